@@ -1,0 +1,375 @@
+"""Benchmark of the Veda block-sparse attention hot path on B200.
+
+One step = one pass of the whole path (permute Q/K/V, pool Q/K, block scores, block
+selection, block-sparse attention, unpermute) over the 16:9-clip workload: B=1, 40
+heads, grid 31x30x54 (50,220 tokens), tile (1,8,16), 10% density (90% sparsity).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {veda,reference}]
+
+Prints one JSON line (rank 0). ``value`` is the effective attention throughput of the
+whole step: FLOPs of the visited 128x128 blocks (4*128^3 each: Q K^T and P V) divided
+by the step time, summed over ranks. Per-kernel times come from CUDA events on the
+launching stream inside the timed region. ``--impl reference`` times the fp64 CPU
+oracle on a bounded sample of the same workload (the CPU baseline).
+Under torchrun (N > 1) every rank runs an independent replica ("replicas only": the
+path has no exchange step); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "block-sparse attn ms/call & effective TFLOPS at 90% sparsity; % bf16 peak"
+UNIT = "TFLOP/s"
+FLOP_PER_BLOCK = 4 * 128 ** 3
+WORKLOAD = synth.CLIP16x9
+SCALE = 1.0 / math.sqrt(128)
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+def _dist():
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist, dist.get_rank(), dist.get_world_size()
+    return None, 0, 1
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        loaded = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _visited_blocks(lists) -> int:
+    return int(lists.full_cnt.sum().item() + lists.part_cnt.sum().item())
+
+
+def run_veda(args):
+    from block_sparse_attention_max_b200 import veda as V
+    dist, rank, world = _dist()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = WORKLOAD
+    peaks = _peaks()
+
+    inp = synth.make_inputs(w)
+    hmaps = V.build_tile_map(w.grid, w.head_shapes, w.n_tail, inp.tile_order)
+    maps = hmaps.to(dev)
+    q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+    wq, wk = inp.wq.to(dev), inp.wk.to(dev)
+    B, N, H, D = q.shape
+    bufs = V.PathBuffers.allocate(B, N, H, maps, w.rho, dev)
+    stream = torch.cuda.current_stream()
+
+    ev = {}
+
+    def event():
+        return torch.cuda.Event(enable_timing=True)
+
+    def step(record: bool):
+        marks = [event() for _ in range(7)] if record else None
+        if record:
+            marks[0].record(stream)
+        V.permute_tiles(q, maps, bufs.q_t)
+        V.permute_tiles(k, maps, bufs.k_t)
+        V.permute_tiles(v, maps, bufs.v_t)
+        if record:
+            marks[1].record(stream)
+        V.tile_pool(bufs.q_t, maps, bufs.pooled_q)
+        V.tile_pool(bufs.k_t, maps, bufs.pooled_k)
+        if record:
+            marks[2].record(stream)
+        V.block_scores(bufs.pooled_q, bufs.pooled_k, wq, wk, bufs.scores, bufs.workspace)
+        if record:
+            marks[3].record(stream)
+        V.select_blocks(bufs.scores, maps, w.rho, bufs.lists.stride, bufs.lists)
+        if record:
+            marks[4].record(stream)
+        V.block_sparse_attn_fwd(bufs.q_t, bufs.k_t, bufs.v_t, maps, bufs.lists, SCALE, bufs.o_t, bufs.lse)
+        if record:
+            marks[5].record(stream)
+        V.unpermute(bufs.o_t, maps, N, bufs.o)
+        if record:
+            marks[6].record(stream)
+        return marks
+
+    for _ in range(args.warmup):
+        step(False)
+    V.check_device_status()
+    blocks = _visited_blocks(bufs.lists)
+    flop_step = blocks * FLOP_PER_BLOCK
+    launches_per_step = 3 + 2 + 2 + 1 + 1 + 1
+
+    clocks = Clocks(dev.index)
+    clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = event(), event()
+    t0.record(stream)
+    all_marks = [step(True) for _ in range(args.steps)]
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    V.check_device_status()
+    ms_total = t0.elapsed_time(t1)
+    stage_names = ["permute_qkv", "pool_qk", "scores", "select", "attention", "unpermute"]
+    stage_ms = {n: statistics.mean(m[i].elapsed_time(m[i + 1]) for m in all_marks)
+                for i, n in enumerate(stage_names)}
+    if dist:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+
+    # end-to-end through the public API with host buffers (pinned), copies inside the region
+    qh, kh, vh = (t.pin_memory() for t in (inp.q, inp.k, inp.v))
+    wqh, wkh = inp.wq.pin_memory(), inp.wk.pin_memory()
+    oh = torch.empty((B, N, H, D), dtype=torch.bfloat16).pin_memory()
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wqd, wkd = torch.empty_like(wq), torch.empty_like(wk)
+
+    def e2e_step():
+        for dst, src in ((qd, qh), (kd, kh), (vd, vh), (wqd, wqh), (wkd, wkh)):
+            dst.copy_(src, non_blocking=True)
+        V.sparse_attention(qd, kd, vd, wqd, wkd, maps, w.rho, SCALE, buffers=bufs)
+        oh.copy_(bufs.o, non_blocking=True)
+
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    e_steps = max(3, min(args.steps, 10))
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = event(), event()
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1) / e_steps
+    if dist:
+        t = torch.tensor([e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    V.check_device_status()
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, wqh, wkh))
+    d2h = oh.numel() * oh.element_size()
+
+    attn_ms = stage_ms["attention"]
+    attn_tflops = flop_step / (attn_ms * 1e-3) / 1e12
+    nbytes = N * H * D * 2
+    hbm = {
+        "permute_GBps": 3 * 2 * nbytes / (stage_ms["permute_qkv"] * 1e-3) / 1e9,
+        "pool_GBps": (2 * nbytes + 2 * w.nT * H * 3 * D * 4) / (stage_ms["pool_qk"] * 1e-3) / 1e9,
+        "unpermute_GBps": 2 * nbytes / (stage_ms["unpermute"] * 1e-3) / 1e9,
+    }
+    for kname in list(hbm):
+        hbm[kname.replace("_GBps", "_frac")] = hbm[kname] / peaks["hbm"]
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "attn_fwd_clip16x9_traffic.json")
+    if os.path.exists(prof):
+        try:
+            traffic = json.load(open(prof)).get("dram_bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    line = {
+        "metric": METRIC, "value": world * flop_step / (ms_step * 1e-3) / 1e12, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded smoothed-field Q/K, N(0,1) V, random-init projections)",
+        "config": {"workload": "clip16x9: B=1 H=40 grid 31x30x54 (50220 tokens) tile (1,8,16), "
+                               "nT=496, density 1/10", "global_batch": world * B, "seq_len": N,
+                   "parallelism": f"replicas x{world}", "visited_blocks": blocks,
+                   "l2": "inputs larger than L2 (Q/K/V 1.54 GB raster + 1.95 GB tiled per step)"},
+        "attn_ms_per_call": attn_ms, "attn_tflops": attn_tflops,
+        "attn_frac_bf16_peak": attn_tflops / peaks["bf16_sus"],
+        "stage_ms": stage_ms, "hbm_stages": hbm,
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peaks["bf16_sus"],
+                     "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_sus"], "traffic": traffic,
+                     "kernel": "attn_fwd_kernel",
+                     "peak_note": f"{peaks['source']} sustained dense bf16 (kernel timed inside a long step)"},
+        "e2e": {"value": world * flop_step / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds, inp)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del bufs
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _oracle_sample(inp, heads, rows_per_head):
+    """The oracle's six steps on some heads of the workload, attention on some query tiles.
+
+    Returns (visited-block FLOPs processed, seconds)."""
+    from oracle import veda_oracle as O
+    w = WORKLOAD
+    t0 = time.perf_counter()
+    f = lambda t: t[:, :, heads].double().numpy()
+    q, k, v = f(inp.q), f(inp.k), f(inp.v)
+    maps = [O.tile_map(w.grid, w.head_shapes[h], w.n_tail) for h in heads]
+    slots, nv, seg = O.stack_maps(maps, w.nT)
+    qt, kt, vt = O.permute(q, slots), O.permute(k, slots), O.permute(v, slots)
+    pq, pk = O.pool(qt, nv), O.pool(kt, nv)
+    S = O.scores(pq, pk, inp.wq[heads].double().numpy(), inp.wk[heads].double().numpy())
+    lists = O.select(S, nv, seg, [len(m.n_valid) for m in maps], w.rho)
+    rows = [(0, j, r) for j in range(len(heads)) for r in range(rows_per_head)]
+    o_t, _ = O.attention(qt, kt, vt, nv, lists, SCALE, rows=rows)
+    O.unpermute(np.nan_to_num(o_t), slots, w.N)
+    dt = time.perf_counter() - t0
+    blocks = sum(len(lists.full[0][j][r]) + len(lists.partial[0][j][r]) for (_, j, r) in rows)
+    return blocks * FLOP_PER_BLOCK, dt
+
+
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(seconds: float, inp):
+    # whole path on one head, attention on as many query tiles as fit the time budget
+    flop, dt = _oracle_sample(inp, [0], 16)
+    per_row = dt / 16
+    rows = int(max(16, min(WORKLOAD.nT, seconds / max(per_row, 1e-3))))
+    flop, dt = _oracle_sample(inp, [0], rows)
+    return {"value": flop / dt / 1e12, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+            "sample": f"fp64 oracle, all six steps on head 0 of 40, attention on {rows} of 496 "
+                      f"query tiles ({dt:.1f} s); value = visited-block FLOPs / CPU time"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    inp = synth.make_inputs(WORKLOAD)
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        _oracle_sample(inp, [0], max(1, rows // 4))
+    flops, secs = 0, 0.0
+    for _ in range(args.steps):
+        f, dt = _oracle_sample(inp, [0], rows)
+        flops += f
+        secs += dt
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same seeded inputs as the CUDA arm)",
+        "config": {"workload": "clip16x9: B=1 H=40 grid 31x30x54 (50220 tokens) tile (1,8,16), "
+                               "nT=496, density 1/10", "global_batch": 1, "seq_len": WORKLOAD.N,
+                   "parallelism": "cpu"},
+        "cpu_baseline": {"kind": "oracle", "cores": _cores(), "value": value, "unit": UNIT,
+                         "sample": f"each step: fp64 oracle, all six steps on head 0 of 40, "
+                                   f"attention on {rows} of 496 query tiles"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["veda", "reference"], default="veda")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=24)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "veda":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_veda(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,340 @@
+// veda_lib.cu -- the C ABI of include/veda.h: argument checks, launch configuration,
+// tensor-map encoding and the per-device status word. Kernels live in k_*.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "../../include/veda.h"
+#include "k_attn.cuh"
+#include "k_gather.cuh"
+#include "k_scores.cuh"
+#include "k_select.cuh"
+#include "veda_ptx.cuh"
+
+namespace veda {
+
+namespace {
+thread_local std::string t_last_error;
+
+struct DeviceInfo {
+  bool probed = false;
+  bool supported = false;
+  int sms = 0;
+  bool attrs_set = false;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+// Signature of the driver's cuTensorMapEncodeTiled (obtained through the runtime's
+// driver entry-point query, so the library needs no link against libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+}  // namespace
+
+void set_last_error(const std::string& msg) { t_last_error = msg; }
+
+namespace {
+
+veda_status fail(veda_status st, const std::string& msg) {
+  set_last_error(msg);
+  return st;
+}
+
+veda_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(VEDA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+// Current device: must be compute capability 10.0 (B200). Sets one-time kernel attributes.
+veda_status current_device(int& sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(VEDA_ERR_UNSUPPORTED, "device ordinal out of range");
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    d.supported = (major == 10 && minor == 0);
+    d.probed = true;
+  }
+  if (!d.supported)
+    return fail(VEDA_ERR_UNSUPPORTED, "the kernels are built for sm_100a (compute capability 10.0) only");
+  if (!d.attrs_set) {
+    struct { const void* f; int bytes; } attrs[] = {
+        {reinterpret_cast<const void*>(permute_kernel), kPermStages * static_cast<int>(kTileBytes) + 1024},
+        {reinterpret_cast<const void*>(unpermute_kernel), kUnpermStages * static_cast<int>(kTileBytes) + 1024},
+        {reinterpret_cast<const void*>(pool_kernel), kPoolStages * static_cast<int>(kTileBytes) + 1024},
+        {reinterpret_cast<const void*>(attn::attn_fwd_kernel), static_cast<int>(attn::kSmemBytes)},
+    };
+    for (auto& x : attrs) {
+      e = cudaFuncSetAttribute(x.f, cudaFuncAttributeMaxDynamicSharedMemorySize, x.bytes);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    }
+    d.attrs_set = true;
+  }
+  sms = d.sms;
+  return VEDA_OK;
+}
+
+veda_status get_encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return VEDA_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
+  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  return VEDA_OK;
+}
+
+// 2D map over rows of 128 bf16 (256 B): box 64 columns x 128 rows, 128-byte swizzle.
+veda_status encode_rows(CUtensorMap& m, const void* base, uint64_t rows) {
+  const cuuint64_t dims[2] = {128, rows};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(r) + ")");
+  return VEDA_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+veda_status launched(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return VEDA_OK;
+}
+
+int grid_for(int64_t units, int sms, int per_sm) {
+  const int64_t g = static_cast<int64_t>(sms) * per_sm;
+  return static_cast<int>(units < g ? units : g);
+}
+
+}  // namespace
+}  // namespace veda
+
+using namespace veda;
+
+extern "C" {
+
+int32_t veda_abi_version(void) { return VEDA_ABI_VERSION; }
+
+const char* veda_status_string(veda_status s) {
+  switch (s) {
+    case VEDA_OK: return "ok";
+    case VEDA_ERR_INVALID_ARG: return "invalid argument";
+    case VEDA_ERR_UNSUPPORTED: return "unsupported device or shape";
+    case VEDA_ERR_CUDA: return "CUDA error";
+    case VEDA_ERR_TIMEOUT: return "a kernel wait timed out";
+    case VEDA_ERR_DEVICE_CHECK: return "a kernel found invalid data";
+  }
+  return "unknown status";
+}
+
+const char* veda_last_error(void) { return t_last_error.c_str(); }
+
+veda_status veda_permute_tiles(const void* x, void* x_tiled, const int32_t* tile_map, int32_t B,
+                               int32_t N, int32_t H, int32_t D, int32_t Npad, veda_stream_t stream) {
+  if (!x || !x_tiled || !tile_map || B <= 0 || N <= 0 || H <= 0 || Npad <= 0 || Npad % 128)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_permute_tiles: bad pointer or size");
+  if (D != 128) return fail(VEDA_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (!aligned(x, 16) || !aligned(x_tiled, 16)) return fail(VEDA_ERR_INVALID_ARG, "veda_permute_tiles: buffers must be 16-byte aligned");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  GatherArgs a{static_cast<const uint8_t*>(x), static_cast<uint8_t*>(x_tiled), tile_map, B, N, H, Npad,
+               Npad / 128, static_cast<int64_t>(B) * H * (Npad / 128)};
+  permute_kernel<<<grid_for(a.units, sms, 1), 32, kPermStages * kTileBytes + 1024,
+                   reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  return launched("permute_kernel");
+}
+
+veda_status veda_unpermute(const void* o_tiled, void* o, const int32_t* tile_map, int32_t B, int32_t N,
+                           int32_t H, int32_t D, int32_t Npad, veda_stream_t stream) {
+  if (!o_tiled || !o || !tile_map || B <= 0 || N <= 0 || H <= 0 || Npad <= 0 || Npad % 128)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_unpermute: bad pointer or size");
+  if (D != 128) return fail(VEDA_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (!aligned(o, 16) || !aligned(o_tiled, 16)) return fail(VEDA_ERR_INVALID_ARG, "veda_unpermute: buffers must be 16-byte aligned");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  GatherArgs a{static_cast<const uint8_t*>(o_tiled), static_cast<uint8_t*>(o), tile_map, B, N, H, Npad,
+               Npad / 128, static_cast<int64_t>(B) * H * (Npad / 128)};
+  unpermute_kernel<<<grid_for(a.units, sms, 1), 32, kUnpermStages * kTileBytes + 1024,
+                     reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  return launched("unpermute_kernel");
+}
+
+veda_status veda_tile_pool(const void* x_tiled, const int32_t* tile_valid, float* pooled, int32_t B,
+                           int32_t H, int32_t nT, int32_t D, veda_stream_t stream) {
+  if (!x_tiled || !tile_valid || !pooled || B <= 0 || H <= 0 || nT <= 0)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_tile_pool: bad pointer or size");
+  if (D != 128) return fail(VEDA_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (!aligned(x_tiled, 16) || !aligned(pooled, 4)) return fail(VEDA_ERR_INVALID_ARG, "veda_tile_pool: misaligned buffer");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  PoolArgs a{static_cast<const uint8_t*>(x_tiled), tile_valid, pooled, B, H, nT,
+             static_cast<int64_t>(B) * H * nT};
+  pool_kernel<<<grid_for(a.units, sms, 1), kPoolThreads, kPoolStages * kTileBytes + 1024,
+                reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  return launched("pool_kernel");
+}
+
+size_t veda_block_scores_workspace_bytes(int32_t B, int32_t H, int32_t nT, int32_t D) {
+  if (B <= 0 || H <= 0 || nT <= 0 || D <= 0) return 0;
+  return static_cast<size_t>(2) * B * H * nT * D * sizeof(float);
+}
+
+veda_status veda_block_scores(const float* pooled_q, const float* pooled_k, const float* Wq, const float* Wk,
+                              float* scores, void* workspace, size_t workspace_bytes, int32_t B, int32_t H,
+                              int32_t nT, int32_t D, veda_stream_t stream) {
+  if (!pooled_q || !pooled_k || !Wq || !Wk || !scores || !workspace || B <= 0 || H <= 0 || nT <= 0)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_scores: bad pointer or size");
+  if (D != 128) return fail(VEDA_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (workspace_bytes < veda_block_scores_workspace_bytes(B, H, nT, D))
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_scores: workspace too small");
+  if (!aligned(pooled_q, 16) || !aligned(pooled_k, 16) || !aligned(Wq, 16) || !aligned(Wk, 16) ||
+      !aligned(workspace, 256))
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_scores: misaligned buffer");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* hat = static_cast<float*>(workspace);             // [2][B][H][nT][128]
+  const int64_t per = static_cast<int64_t>(nT) * 128;
+  // projection: hat[which] = mean + pooled . W^T   (M = nT, N = 128, K = 384)
+  NtGemmArgs p{};
+  p.a0[0] = pooled_q; p.a0[1] = pooled_k;
+  p.b0[0] = Wq; p.b0[1] = Wk;
+  p.r0[0] = pooled_q; p.r0[1] = pooled_k;                  // mean = first 128 of each row
+  p.c0 = hat;
+  p.a_bh = static_cast<int64_t>(nT) * 384; p.b_h = 128 * 384; p.b_b = 0; p.r_bh = p.a_bh; p.c_z = per;
+  p.lda = 384; p.ldb = 384; p.ldr = 384; p.ldc = 128;
+  p.M = nT; p.N = 128; p.K = 384; p.B = B; p.H = H;
+  dim3 gp(128 / kGemmBN, (nT + kGemmBM - 1) / kGemmBM, 2 * B * H);
+  nt_gemm_kernel<<<gp, kGemmThreads, 0, s>>>(p);
+  st = launched("projection");
+  if (st != VEDA_OK) return st;
+  // scores = qhat . khat^T  (M = N = nT, K = 128)
+  NtGemmArgs q{};
+  q.a0[0] = hat; q.a0[1] = hat;
+  q.b0[0] = hat + static_cast<int64_t>(B) * H * per; q.b0[1] = q.b0[0];
+  q.r0[0] = nullptr; q.r0[1] = nullptr;
+  q.c0 = scores;
+  q.a_bh = per; q.b_h = per; q.b_b = static_cast<int64_t>(H) * per; q.r_bh = 0;
+  q.c_z = static_cast<int64_t>(nT) * nT;
+  q.lda = 128; q.ldb = 128; q.ldr = 0; q.ldc = nT;
+  q.M = nT; q.N = nT; q.K = 128; q.B = B; q.H = H;
+  dim3 gq((nT + kGemmBN - 1) / kGemmBN, (nT + kGemmBM - 1) / kGemmBM, B * H);
+  nt_gemm_kernel<<<gq, kGemmThreads, 0, s>>>(q);
+  return launched("scores");
+}
+
+veda_status veda_select_blocks(const float* scores, const int32_t* tile_valid, const int32_t* tile_segment,
+                               const int32_t* nT_per_head, int32_t n_segments, const int32_t* rho_num,
+                               const int32_t* rho_den, int32_t* full_cnt, int32_t* full_idx, int32_t* part_cnt,
+                               int32_t* part_idx, int32_t list_stride, int32_t B, int32_t H, int32_t nT,
+                               veda_stream_t stream) {
+  if (!scores || !tile_valid || !tile_segment || !nT_per_head || !rho_num || !rho_den || !full_cnt ||
+      !full_idx || !part_cnt || !part_idx || B <= 0 || H <= 0 || nT <= 0)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_select_blocks: bad pointer or size");
+  if (nT > VEDA_MAX_TILES) return fail(VEDA_ERR_INVALID_ARG, "veda_select_blocks: nT above VEDA_MAX_TILES");
+  if (n_segments < 1 || n_segments > VEDA_MAX_SEGMENTS)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_select_blocks: n_segments out of range");
+  int64_t bound = 1;
+  for (int s = 0; s < n_segments; ++s) {
+    if (rho_den[s] < 1 || rho_num[s] < 0 || rho_num[s] > rho_den[s])
+      return fail(VEDA_ERR_INVALID_ARG, "veda_select_blocks: density must be num/den with 0 <= num <= den");
+    bound += (static_cast<int64_t>(nT) * rho_num[s] + rho_den[s] - 1) / rho_den[s];
+  }
+  if (bound > nT) bound = nT;
+  if (list_stride < bound)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_select_blocks: list_stride below the largest possible row budget");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  SelectArgs a{};
+  a.scores = scores; a.valid = tile_valid; a.segment = tile_segment; a.nT_per_head = nT_per_head;
+  a.full_cnt = full_cnt; a.full_idx = full_idx; a.part_cnt = part_cnt; a.part_idx = part_idx;
+  a.stride = list_stride; a.B = B; a.H = H; a.nT = nT; a.n_seg = n_segments;
+  for (int s = 0; s < kMaxSeg; ++s) {
+    a.rho_num[s] = s < n_segments ? rho_num[s] : 0;
+    a.rho_den[s] = s < n_segments ? rho_den[s] : 1;
+  }
+  const int64_t rows = static_cast<int64_t>(B) * H * nT;
+  if (rows > INT32_MAX) return fail(VEDA_ERR_INVALID_ARG, "veda_select_blocks: too many rows");
+  select_kernel<<<static_cast<unsigned>(rows), kSelThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  return launched("select_kernel");
+}
+
+veda_status veda_block_sparse_attn_fwd(const void* q, const void* k, const void* v, const int32_t* tile_valid,
+                                       const int32_t* full_cnt, const int32_t* full_idx, const int32_t* part_cnt,
+                                       const int32_t* part_idx, int32_t list_stride, float softmax_scale, void* o,
+                                       float* lse, int32_t B, int32_t H, int32_t nT, int32_t D,
+                                       veda_stream_t stream) {
+  if (!q || !k || !v || !tile_valid || !full_cnt || !full_idx || !part_cnt || !part_idx || !o || B <= 0 ||
+      H <= 0 || nT <= 0 || list_stride <= 0)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_sparse_attn_fwd: bad pointer or size");
+  if (D != 128) return fail(VEDA_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_sparse_attn_fwd: softmax_scale must be positive and finite");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16))
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_sparse_attn_fwd: Q/K/V/O must be 16-byte aligned");
+  const int64_t rows = static_cast<int64_t>(B) * H * nT * 128;
+  if (rows > INT32_MAX) return fail(VEDA_ERR_INVALID_ARG, "veda_block_sparse_attn_fwd: too many rows");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  if ((st = get_encoder()) != VEDA_OK) return st;
+  CUtensorMap tq, tk, tv;
+  if ((st = encode_rows(tq, q, rows)) != VEDA_OK) return st;
+  if ((st = encode_rows(tk, k, rows)) != VEDA_OK) return st;
+  if ((st = encode_rows(tv, v, rows)) != VEDA_OK) return st;
+  attn::Args a{};
+  a.valid = tile_valid; a.full_cnt = full_cnt; a.full_idx = full_idx; a.part_cnt = part_cnt; a.part_idx = part_idx;
+  a.o = static_cast<__nv_bfloat16*>(o); a.lse = lse;
+  a.stride = list_stride; a.H = H; a.nT = nT;
+  a.items = static_cast<int64_t>(B) * H * nT;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  attn::attn_fwd_kernel<<<grid_for(a.items, sms, 1), attn::kThreads, attn::kSmemBytes,
+                          reinterpret_cast<cudaStream_t>(stream)>>>(tq, tk, tv, a);
+  return launched("attn_fwd_kernel");
+}
+
+veda_status veda_check_device_status(veda_stream_t stream, uint32_t* detail) {
+  if (detail) *detail = 0;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  uint32_t v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "read status word");
+  if (v) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "clear status word");
+  }
+  if (detail) *detail = v;
+  if (v & ST_TIMEOUT) return fail(VEDA_ERR_TIMEOUT, "a kernel wait ran out (site " + std::to_string((v >> 8) & 0xff) + ")");
+  if (v) return fail(VEDA_ERR_DEVICE_CHECK, "a kernel flagged invalid data (bits " + std::to_string(v & 0xff) + ")");
+  return VEDA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,362 @@
+"""ctypes binding of libveda.so (include/veda.h) -- argument marshalling only.
+
+Every step of the path runs in the library's CUDA kernels; this module only turns
+torch tensors into pointers and sizes, allocates outputs with torch, and raises when
+a call returns an error. There is no fallback: if the library is missing or the device
+is not a B200 (compute capability 10.0), calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libveda.so")
+
+VEDA_OK = 0
+STATUS_NAMES = {0: "VEDA_OK", 1: "VEDA_ERR_INVALID_ARG", 2: "VEDA_ERR_UNSUPPORTED",
+                3: "VEDA_ERR_CUDA", 4: "VEDA_ERR_TIMEOUT", 5: "VEDA_ERR_DEVICE_CHECK"}
+
+EXPORTED = (
+    "veda_abi_version", "veda_status_string", "veda_last_error", "veda_geometry_sizes",
+    "veda_build_tile_map", "veda_permute_tiles", "veda_tile_pool",
+    "veda_block_scores_workspace_bytes", "veda_block_scores", "veda_select_blocks",
+    "veda_block_sparse_attn_fwd", "veda_unpermute", "veda_check_device_status",
+)
+
+
+class VedaError(RuntimeError):
+    def __init__(self, call: str, status: int, message: str):
+        super().__init__(f"{call} -> {STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class TileShape(ctypes.Structure):
+    _fields_ = [("t", ctypes.c_int32), ("h", ctypes.c_int32), ("w", ctypes.c_int32)]
+
+
+class Geometry(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int32), ("T", ctypes.c_int32), ("Hg", ctypes.c_int32),
+                ("Wg", ctypes.c_int32), ("n_tail", ctypes.c_int32),
+                ("head_shape", ctypes.POINTER(TileShape)),
+                ("tile_order", ctypes.POINTER(ctypes.c_int32)),
+                ("order_stride", ctypes.c_int32)]
+
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_F = ctypes.c_float
+_SIG = {
+    "veda_abi_version": (_I, []),
+    "veda_status_string": (ctypes.c_char_p, [_I]),
+    "veda_last_error": (ctypes.c_char_p, []),
+    "veda_geometry_sizes": (_I, [ctypes.POINTER(Geometry), _P, _P, _P]),
+    "veda_build_tile_map": (_I, [ctypes.POINTER(Geometry), _P, _P, _P, _P]),
+    "veda_permute_tiles": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "veda_tile_pool": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
+    "veda_block_scores_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
+    "veda_block_scores": (_I, [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _P]),
+    "veda_select_blocks": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "veda_block_sparse_attn_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _F, _P, _P, _I, _I,
+                                        _I, _I, _P]),
+    "veda_unpermute": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "veda_check_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library. Raises if libveda.so has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m block_sparse_attention_max_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIG.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(call: str, status: int) -> None:
+    if status != VEDA_OK:
+        msg = lib().veda_last_error().decode(errors="replace")
+        raise VedaError(call, status, msg)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str, cuda: bool = True) -> None:
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+
+
+# ---------------------------------------------------------------------------------------
+# geometry (host)
+# ---------------------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class TileMaps:
+    """Host tile maps of one geometry (numpy int32)."""
+    tile_map: np.ndarray       # [H, Npad]
+    tile_valid: np.ndarray     # [H, nT]
+    tile_segment: np.ndarray   # [H, nT]
+    nT_per_head: np.ndarray    # [H]
+    N: int
+    nT: int
+    Npad: int
+
+    def to(self, device) -> "DeviceMaps":
+        f = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        return DeviceMaps(f(self.tile_map), f(self.tile_valid), f(self.tile_segment),
+                          f(self.nT_per_head), self.N, self.nT, self.Npad)
+
+
+@dataclasses.dataclass
+class DeviceMaps:
+    tile_map: torch.Tensor
+    tile_valid: torch.Tensor
+    tile_segment: torch.Tensor
+    nT_per_head: torch.Tensor
+    N: int
+    nT: int
+    Npad: int
+
+
+def _geometry(grid, head_shapes, n_tail, tile_order):
+    H = len(head_shapes)
+    shapes = (TileShape * H)(*[TileShape(*map(int, s)) for s in head_shapes])
+    keep = [shapes]
+    g = Geometry(H, int(grid[0]), int(grid[1]), int(grid[2]), int(n_tail), shapes, None, 0)
+    if tile_order is not None:
+        order = np.ascontiguousarray(np.asarray(tile_order, dtype=np.int32))
+        keep.append(order)
+        g.tile_order = order.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+        g.order_stride = order.shape[1]
+    return g, keep
+
+
+def geometry_sizes(grid, head_shapes, n_tail=0) -> Tuple[int, int, int]:
+    g, _keep = _geometry(grid, head_shapes, n_tail, None)
+    N, nT, Npad = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check("veda_geometry_sizes", lib().veda_geometry_sizes(
+        ctypes.byref(g), ctypes.addressof(N), ctypes.addressof(nT), ctypes.addressof(Npad)))
+    return N.value, nT.value, Npad.value
+
+
+def build_tile_map(grid, head_shapes, n_tail=0, tile_order=None) -> TileMaps:
+    g, _keep = _geometry(grid, head_shapes, n_tail, tile_order)
+    N, nT, Npad = geometry_sizes(grid, head_shapes, n_tail)
+    H = len(head_shapes)
+    tm = np.empty((H, Npad), np.int32)
+    tv = np.empty((H, nT), np.int32)
+    ts = np.empty((H, nT), np.int32)
+    nph = np.empty((H,), np.int32)
+    _check("veda_build_tile_map", lib().veda_build_tile_map(
+        ctypes.byref(g), tm.ctypes.data, tv.ctypes.data, ts.ctypes.data, nph.ctypes.data))
+    return TileMaps(tm, tv, ts, nph, N, nT, Npad)
+
+
+# ---------------------------------------------------------------------------------------
+# device steps
+# ---------------------------------------------------------------------------------------
+
+def permute_tiles(x: torch.Tensor, maps: DeviceMaps, out: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    _need(x, torch.bfloat16, "x")
+    B, N, H, D = x.shape
+    if out is None:
+        out = torch.empty((B, H, maps.Npad, D), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    _check("veda_permute_tiles", lib().veda_permute_tiles(
+        _ptr(x), _ptr(out), _ptr(maps.tile_map), B, N, H, D, maps.Npad, _stream(stream)))
+    return out
+
+
+def tile_pool(x_tiled: torch.Tensor, maps: DeviceMaps, out: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    _need(x_tiled, torch.bfloat16, "x_tiled")
+    B, H, Npad, D = x_tiled.shape
+    nT = Npad // 128
+    if out is None:
+        out = torch.empty((B, H, nT, 3, D), dtype=torch.float32, device=x_tiled.device)
+    _need(out, torch.float32, "out")
+    _check("veda_tile_pool", lib().veda_tile_pool(
+        _ptr(x_tiled), _ptr(maps.tile_valid), _ptr(out), B, H, nT, D, _stream(stream)))
+    return out
+
+
+def block_scores_workspace_bytes(B: int, H: int, nT: int, D: int = 128) -> int:
+    return int(lib().veda_block_scores_workspace_bytes(B, H, nT, D))
+
+
+def block_scores(pooled_q: torch.Tensor, pooled_k: torch.Tensor, wq: torch.Tensor,
+                 wk: torch.Tensor, out: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    for t, n in ((pooled_q, "pooled_q"), (pooled_k, "pooled_k"), (wq, "wq"), (wk, "wk")):
+        _need(t, torch.float32, n)
+    B, H, nT, _, D = pooled_q.shape
+    if out is None:
+        out = torch.empty((B, H, nT, nT), dtype=torch.float32, device=pooled_q.device)
+    nbytes = block_scores_workspace_bytes(B, H, nT, D)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=pooled_q.device)
+    _check("veda_block_scores", lib().veda_block_scores(
+        _ptr(pooled_q), _ptr(pooled_k), _ptr(wq), _ptr(wk), _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), B, H, nT, D, _stream(stream)))
+    return out
+
+
+def list_stride_for(nT: int, rho: Sequence[Tuple[int, int]]) -> int:
+    """Smallest list_stride veda_select_blocks accepts for these densities."""
+    bound = 1 + sum(-(-nT * p // q) for p, q in rho)
+    return min(nT, bound)
+
+
+@dataclasses.dataclass
+class BlockLists:
+    full_cnt: torch.Tensor    # [B, H, nT] int32
+    full_idx: torch.Tensor    # [B, H, nT, stride] int32
+    part_cnt: torch.Tensor
+    part_idx: torch.Tensor
+    stride: int
+
+
+def select_blocks(scores: torch.Tensor, maps: DeviceMaps, rho: Sequence[Tuple[int, int]],
+                  list_stride: Optional[int] = None, out: Optional[BlockLists] = None,
+                  stream=None) -> BlockLists:
+    _need(scores, torch.float32, "scores")
+    B, H, nT, _ = scores.shape
+    stride = list_stride or list_stride_for(nT, rho)
+    if out is None:
+        dev = scores.device
+        out = BlockLists(torch.empty((B, H, nT), dtype=torch.int32, device=dev),
+                         torch.zeros((B, H, nT, stride), dtype=torch.int32, device=dev),
+                         torch.empty((B, H, nT), dtype=torch.int32, device=dev),
+                         torch.zeros((B, H, nT, stride), dtype=torch.int32, device=dev), stride)
+    num = (ctypes.c_int32 * len(rho))(*[int(p) for p, _ in rho])
+    den = (ctypes.c_int32 * len(rho))(*[int(q) for _, q in rho])
+    _check("veda_select_blocks", lib().veda_select_blocks(
+        _ptr(scores), _ptr(maps.tile_valid), _ptr(maps.tile_segment), _ptr(maps.nT_per_head),
+        len(rho), ctypes.addressof(num), ctypes.addressof(den), _ptr(out.full_cnt),
+        _ptr(out.full_idx), _ptr(out.part_cnt), _ptr(out.part_idx), out.stride, B, H, nT,
+        _stream(stream)))
+    return out
+
+
+def block_sparse_attn_fwd(q_t: torch.Tensor, k_t: torch.Tensor, v_t: torch.Tensor,
+                          maps: DeviceMaps, lists: BlockLists, scale: float,
+                          out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                          want_lse: bool = True, stream=None):
+    for t, n in ((q_t, "q"), (k_t, "k"), (v_t, "v")):
+        _need(t, torch.bfloat16, n)
+    B, H, Npad, D = q_t.shape
+    nT = Npad // 128
+    if out is None:
+        out = torch.empty_like(q_t)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, Npad), dtype=torch.float32, device=q_t.device)
+    _check("veda_block_sparse_attn_fwd", lib().veda_block_sparse_attn_fwd(
+        _ptr(q_t), _ptr(k_t), _ptr(v_t), _ptr(maps.tile_valid), _ptr(lists.full_cnt),
+        _ptr(lists.full_idx), _ptr(lists.part_cnt), _ptr(lists.part_idx), lists.stride,
+        float(scale), _ptr(out), _ptr(lse), B, H, nT, D, _stream(stream)))
+    return out, lse
+
+
+def unpermute(o_t: torch.Tensor, maps: DeviceMaps, N: int, out: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    _need(o_t, torch.bfloat16, "o_tiled")
+    B, H, Npad, D = o_t.shape
+    if out is None:
+        out = torch.empty((B, N, H, D), dtype=torch.bfloat16, device=o_t.device)
+    _check("veda_unpermute", lib().veda_unpermute(
+        _ptr(o_t), _ptr(out), _ptr(maps.tile_map), B, N, H, D, Npad, _stream(stream)))
+    return out
+
+
+def check_device_status(stream=None) -> int:
+    """Synchronise the stream and raise if a kernel recorded an error. Returns the raw bits."""
+    detail = ctypes.c_uint32(0)
+    st = lib().veda_check_device_status(_stream(stream), ctypes.byref(detail))
+    _check("veda_check_device_status", st)
+    return detail.value
+
+
+# ---------------------------------------------------------------------------------------
+# the whole path
+# ---------------------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class PathBuffers:
+    """Device buffers of one attention call (reusable across calls of the same shape)."""
+    q_t: torch.Tensor
+    k_t: torch.Tensor
+    v_t: torch.Tensor
+    pooled_q: torch.Tensor
+    pooled_k: torch.Tensor
+    scores: torch.Tensor
+    workspace: torch.Tensor
+    lists: BlockLists
+    o_t: torch.Tensor
+    lse: torch.Tensor
+    o: torch.Tensor
+
+    @staticmethod
+    def allocate(B: int, N: int, H: int, maps: DeviceMaps, rho, device) -> "PathBuffers":
+        nT, Npad, D = maps.nT, maps.Npad, 128
+        bf = dict(dtype=torch.bfloat16, device=device)
+        f32 = dict(dtype=torch.float32, device=device)
+        stride = list_stride_for(nT, rho)
+        i32 = dict(dtype=torch.int32, device=device)
+        lists = BlockLists(torch.zeros((B, H, nT), **i32), torch.zeros((B, H, nT, stride), **i32),
+                           torch.zeros((B, H, nT), **i32), torch.zeros((B, H, nT, stride), **i32),
+                           stride)
+        return PathBuffers(
+            torch.empty((B, H, Npad, D), **bf), torch.empty((B, H, Npad, D), **bf),
+            torch.empty((B, H, Npad, D), **bf), torch.empty((B, H, nT, 3, D), **f32),
+            torch.empty((B, H, nT, 3, D), **f32), torch.empty((B, H, nT, nT), **f32),
+            torch.empty(block_scores_workspace_bytes(B, H, nT, D), dtype=torch.uint8, device=device),
+            lists, torch.empty((B, H, Npad, D), **bf), torch.empty((B, H, Npad), **f32),
+            torch.empty((B, N, H, D), **bf))
+
+
+def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, wq: torch.Tensor,
+                     wk: torch.Tensor, maps: DeviceMaps, rho: Sequence[Tuple[int, int]],
+                     scale: float, buffers: Optional[PathBuffers] = None, stream=None):
+    """All six steps on raster Q/K/V [B, N, H, 128] (bf16, on the device).
+
+    Returns the PathBuffers holding every intermediate; ``.o`` is the raster output.
+    """
+    B, N, H, D = q.shape
+    bufs = buffers or PathBuffers.allocate(B, N, H, maps, rho, q.device)
+    permute_tiles(q, maps, bufs.q_t, stream)
+    permute_tiles(k, maps, bufs.k_t, stream)
+    permute_tiles(v, maps, bufs.v_t, stream)
+    tile_pool(bufs.q_t, maps, bufs.pooled_q, stream)
+    tile_pool(bufs.k_t, maps, bufs.pooled_k, stream)
+    block_scores(bufs.pooled_q, bufs.pooled_k, wq, wk, bufs.scores, bufs.workspace, stream)
+    select_blocks(bufs.scores, maps, rho, bufs.lists.stride, bufs.lists, stream)
+    block_sparse_attn_fwd(bufs.q_t, bufs.k_t, bufs.v_t, maps, bufs.lists, scale, bufs.o_t,
+                          bufs.lse, stream=stream)
+    unpermute(bufs.o_t, maps, N, bufs.o, stream)
+    return bufs

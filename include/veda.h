@@ -1,0 +1,257 @@
+/*
+ * veda.h -- C ABI of the Veda block-sparse attention hot path for NVIDIA B200 (sm_100a).
+ *
+ * The path (per attention call), as described on the "Miowtion" README (bullet
+ * "Sparse acceleration (Veda)"; Key Features / Veda sparse attention) and on
+ * "Deploying this checkpoint" (preamble; section 2, SM90 and SM100 paragraphs):
+ *
+ *   1. veda_permute_tiles          raster tokens -> 3D tiles of 128 tokens
+ *   2. veda_tile_pool              mean / max / min of every Q and K tile
+ *   3. veda_block_scores           per-head residual projection, (q tile, k tile) scores
+ *   4. veda_select_blocks          Bresenham budgets, forced diagonal, full/partial lists
+ *   5. veda_block_sparse_attn_fwd  attention over the listed key tiles only
+ *   6. veda_unpermute              tiles -> raster order
+ *
+ * Conventions shared by every call:
+ *  - Ownership: the caller allocates and owns every buffer. Pointers named *_dev or
+ *    documented as "device" must be device memory of the current CUDA device; the
+ *    library allocates no device memory of its own (its status word is a static
+ *    __device__ variable) and keeps no pointer after a call returns.
+ *  - Synchrony: device calls only enqueue work on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream) and return. Argument errors are detected on the host
+ *    before anything is launched. Errors found by a kernel (bad index, NaN score,
+ *    bounded wait that ran out) are recorded in a per-device status word and are
+ *    reported by veda_check_device_status().
+ *  - Architecture: every device call returns VEDA_ERR_UNSUPPORTED on a device other
+ *    than compute capability 10.0 (B200) and for head_dim != 128. There is no dense,
+ *    CPU or other fallback.
+ *  - Types: Q/K/V/O are bf16 (uint16 storage); pooled features, projection weights,
+ *    scores and LSE are fp32; indices and counts are int32. All arrays are dense
+ *    row-major with the shapes given below.
+ *  - Shapes: B batch, H heads, D = 128 head_dim, N raster tokens, nT tiles per head
+ *    (the maximum over heads), Npad = nT * 128 tile slots per head.
+ */
+#ifndef VEDA_H_
+#define VEDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define VEDA_API __attribute__((visibility("default")))
+#else
+#define VEDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VEDA_ABI_VERSION 1
+#define VEDA_TILE 128          /* tokens per tile and rows per query tile */
+#define VEDA_MAX_SEGMENTS 4    /* key segments with their own budget */
+#define VEDA_MAX_TILES 2048    /* tiles per head accepted by veda_select_blocks */
+
+typedef struct CUstream_st* veda_stream_t;   /* same type as cudaStream_t */
+
+typedef enum veda_status {
+  VEDA_OK = 0,
+  VEDA_ERR_INVALID_ARG = 1,   /* a pointer, size or geometry argument is invalid */
+  VEDA_ERR_UNSUPPORTED = 2,   /* not a compute-capability 10.0 device, or head_dim != 128 */
+  VEDA_ERR_CUDA = 3,          /* a CUDA runtime call failed (see veda_last_error()) */
+  VEDA_ERR_TIMEOUT = 4,       /* a kernel's bounded wait ran out; it stopped early */
+  VEDA_ERR_DEVICE_CHECK = 5,  /* a kernel found a bad index, count or NaN score */
+} veda_status;
+
+/* One 3D tile shape; t*h*w must equal 128 ("3D tiles of 128 tokens"). */
+typedef struct veda_tile_shape {
+  int32_t t, h, w;
+} veda_tile_shape;
+
+/*
+ * Token geometry of one attention call (host memory, read during the call only).
+ * "Miowtion" README, Key Features / Veda sparse attention: up to two (t, h, w) tile
+ * shapes per layer (per head), padded grids with valid-prefix tiles, segmented
+ * reference/target budgets; NEWS 2026/09/23: per-head dynamic tile permutations.
+ *   H            heads
+ *   T, Hg, Wg    video grid (raster index of token (t,h,w) = (t*Hg + h)*Wg + w)
+ *   n_tail       appended 1D tokens (e.g. audio), raster indices T*Hg*Wg + j
+ *   head_shape   [H] tile shape of each head
+ *   tile_order   NULL, or [H][order_stride]: head h's position p holds its video tile
+ *                tile_order[h*order_stride + p] of the raster tile enumeration (the
+ *                first n_video_tiles(h) entries must be a permutation)
+ */
+typedef struct veda_geometry {
+  int32_t H;
+  int32_t T, Hg, Wg;
+  int32_t n_tail;
+  const veda_tile_shape* head_shape;
+  const int32_t* tile_order;
+  int32_t order_stride;
+} veda_geometry;
+
+/* Library ABI version (VEDA_ABI_VERSION). */
+VEDA_API int32_t veda_abi_version(void);
+
+/* Static description of a status code. Never NULL. */
+VEDA_API const char* veda_status_string(veda_status s);
+
+/* Message of the last failing call on this host thread ("" if none). Never NULL. */
+VEDA_API const char* veda_last_error(void);
+
+/*
+ * Sizes implied by a geometry (host only, no CUDA). Outputs (any may be NULL):
+ *   N        raster tokens T*Hg*Wg + n_tail
+ *   nT_max   tiles per head, maximum over heads (video tiles of the padded grid
+ *            plus ceil(n_tail/128) tail tiles)
+ *   Npad_max nT_max * 128
+ * Returns VEDA_ERR_INVALID_ARG for a NULL geometry, negative sizes or a tile shape
+ * whose volume is not 128.
+ */
+VEDA_API veda_status veda_geometry_sizes(const veda_geometry* g, int32_t* N, int32_t* nT_max,
+                                int32_t* Npad_max);
+
+/*
+ * Step 1 plan: slot -> raster-token map of every head (host only, no CUDA).
+ * "Miowtion" README, bullet "Sparse acceleration (Veda)" (tokens permuted into 3D
+ * tiles of 128) and Key Features (padded grids with valid-prefix tiles). Each head's
+ * grid is padded to a multiple of its tile shape; tiles are enumerated in raster
+ * order of their tile coordinates (then reordered by tile_order); inside a tile the
+ * valid tokens come first, in local (t,h,w) raster order; tail tokens follow as 1D
+ * tiles of 128. Video tiles are key segment 0, tail tiles segment 1.
+ * Outputs (host memory, caller-allocated):
+ *   tile_map     [H][Npad_max] raster token of each slot, -1 for a pad slot
+ *   tile_valid   [H][nT_max]   valid tokens of each tile (0 past the head's tiles)
+ *   tile_segment [H][nT_max]   key segment of each tile
+ *   nT_per_head  [H]           tiles of each head
+ */
+VEDA_API veda_status veda_build_tile_map(const veda_geometry* g, int32_t* tile_map, int32_t* tile_valid,
+                                int32_t* tile_segment, int32_t* nT_per_head);
+
+/*
+ * Step 1: gather raster tokens into tile order (device).
+ *   x        [B][N][H][D] bf16, raster order
+ *   x_tiled  [B][H][Npad][D] bf16; slot s of head h receives x[b][tile_map[h][s]][h],
+ *            or zeros when tile_map[h][s] < 0
+ *   tile_map [H][Npad] int32 (device), values in [-1, N)
+ * Out-of-range map entries are skipped (the slot is zeroed) and flagged as
+ * VEDA_ERR_DEVICE_CHECK in the status word. x and x_tiled must not overlap.
+ */
+VEDA_API veda_status veda_permute_tiles(const void* x, void* x_tiled, const int32_t* tile_map,
+                               int32_t B, int32_t N, int32_t H, int32_t D, int32_t Npad,
+                               veda_stream_t stream);
+
+/*
+ * Step 2: mean, max and min of every tile over its valid slots, per channel (device).
+ * "Miowtion" README, Key Features / Veda sparse attention: mean/max/min pooling.
+ *   x_tiled    [B][H][nT*128][D] bf16 (output of step 1)
+ *   tile_valid [H][nT] int32 (device), each in [0, 128]; a tile with 0 pools to zeros
+ *   pooled     [B][H][nT][3][D] fp32: [..][0][:] mean, [1] max, [2] min
+ * Sums are accumulated in fp32.
+ */
+VEDA_API veda_status veda_tile_pool(const void* x_tiled, const int32_t* tile_valid, float* pooled,
+                           int32_t B, int32_t H, int32_t nT, int32_t D, veda_stream_t stream);
+
+/* Workspace bytes veda_block_scores needs (the projected features of Q and K tiles). */
+VEDA_API size_t veda_block_scores_workspace_bytes(int32_t B, int32_t H, int32_t nT, int32_t D);
+
+/*
+ * Step 3: score every (query tile, key tile) pair (device).
+ * "Miowtion" README, bullet "Sparse acceleration (Veda)": a small per-head predictor
+ * scores (query tile, key tile) pairs; Key Features: "mean/max/min pooling + per-head
+ * residual projection". For head h with f = [mean; max; min] (3D values):
+ *   qhat_i = mean_q,i + Wq[h] f_q,i      khat_j = mean_k,j + Wk[h] f_k,j
+ *   scores[b][h][i][j] = qhat_i . khat_j
+ *   pooled_q, pooled_k  [B][H][nT][3][D] fp32 (output of step 2)
+ *   Wq, Wk              [H][D][3D] fp32
+ *   scores              [B][H][nT][nT] fp32
+ *   workspace           device scratch of >= veda_block_scores_workspace_bytes(...)
+ *                       bytes, 256-byte aligned; clobbered
+ * Products are accumulated in fp32.
+ */
+VEDA_API veda_status veda_block_scores(const float* pooled_q, const float* pooled_k, const float* Wq,
+                              const float* Wk, float* scores, void* workspace,
+                              size_t workspace_bytes, int32_t B, int32_t H, int32_t nT, int32_t D,
+                              veda_stream_t stream);
+
+/*
+ * Step 4: block lists of every query tile (device).
+ * "Miowtion" README, Key Features / Veda sparse attention: equal-kernel-cost budgets
+ * with Bresenham rounding, forced diagonal tiles, segmented budgets, full/partial
+ * block lists; "Deploying this checkpoint", section 2 (SM90): the block mask is
+ * packed into full/partial index lists.
+ * For head h with n = nT_per_head[h] tiles and segment s holding nK_s of them, row
+ * r < n takes k_rs = floor((r+1) nK_s p_s/q_s) - floor(r nK_s p_s/q_s) key tiles of
+ * segment s (exact integer arithmetic; rho_s = rho_num[s]/rho_den[s]). In the row's
+ * own segment k is raised to at least 1 and the diagonal tile r is taken first; the
+ * other tiles are taken by score, highest first, equal scores (-0 == +0) to the lower
+ * index. The chosen set is sorted ascending and split into full tiles
+ * (tile_valid == 128) and partial tiles. Rows r >= n get empty lists.
+ *   scores        [B][H][nT][nT] fp32 (device); a NaN among a row's candidates is
+ *                 flagged VEDA_ERR_DEVICE_CHECK and ranked last
+ *   tile_valid, tile_segment  [H][nT] int32 (device); segments in [0, n_segments)
+ *   nT_per_head   [H] int32 (device), each in [0, nT]
+ *   rho_num, rho_den  [n_segments] int32 (HOST), 0 <= num <= den, den >= 1
+ *   full_cnt, part_cnt  [B][H][nT] int32 (device, out)
+ *   full_idx, part_idx  [B][H][nT][list_stride] int32 (device, out); the first cnt
+ *                 entries of a row are valid, the rest are left untouched
+ *   list_stride   entries per row; must be >= min(nT, sum_s ceil(nT*rho_s) + 1)
+ * Limits: nT <= VEDA_MAX_TILES, 1 <= n_segments <= VEDA_MAX_SEGMENTS.
+ */
+VEDA_API veda_status veda_select_blocks(const float* scores, const int32_t* tile_valid,
+                               const int32_t* tile_segment, const int32_t* nT_per_head,
+                               int32_t n_segments, const int32_t* rho_num, const int32_t* rho_den,
+                               int32_t* full_cnt, int32_t* full_idx, int32_t* part_cnt,
+                               int32_t* part_idx, int32_t list_stride, int32_t B, int32_t H,
+                               int32_t nT, veda_stream_t stream);
+
+/*
+ * Step 5: block-sparse attention forward (device).
+ * "Deploying this checkpoint", preamble (attention only visits the selected key
+ * tiles) and section 2 (128 x 128 tiles at head_dim 128, one 128-row query tile per
+ * block row); "Miowtion" README, Key Features (full/partial block lists, a single
+ * mask function on partial blocks). For every (b, h, query tile r), with rows
+ * i in [r*128, r*128+128) (pad rows included):
+ *   o[i] = sum_j softmax_j(scale * q_i . k_j) v_j
+ * over the valid slots (slot < tile_valid) of the key tiles listed in full_idx and
+ * part_idx for that row; online softmax, fp32 scores/accumulators, bf16 output.
+ *   q, k, v       [B][H][nT*128][128] bf16 (device, output of step 1), 16-byte aligned
+ *   tile_valid    [H][nT] int32 (device)
+ *   full_cnt/idx, part_cnt/idx  as produced by step 4 (device); key indices in [0, nT)
+ *   o             [B][H][nT*128][128] bf16 (device, out); rows with no key tile get 0
+ *   lse           NULL or [B][H][nT*128] fp32 (device, out): natural-log sum of
+ *                 exp(scale * q.k) over the visited keys; -inf for rows with none
+ * Out-of-range key indices or counts are flagged VEDA_ERR_DEVICE_CHECK and that
+ * query tile's output is zeroed.
+ */
+VEDA_API veda_status veda_block_sparse_attn_fwd(const void* q, const void* k, const void* v,
+                                       const int32_t* tile_valid, const int32_t* full_cnt,
+                                       const int32_t* full_idx, const int32_t* part_cnt,
+                                       const int32_t* part_idx, int32_t list_stride,
+                                       float softmax_scale, void* o, float* lse, int32_t B,
+                                       int32_t H, int32_t nT, int32_t D, veda_stream_t stream);
+
+/*
+ * Step 6: scatter tile-order rows back to raster order (device).
+ *   o_tiled  [B][H][Npad][D] bf16
+ *   o        [B][N][H][D] bf16; o[b][tile_map[h][s]][h] = o_tiled[b][h][s] for every
+ *            slot with tile_map[h][s] >= 0; pad slots are dropped. Raster rows that no
+ *            slot maps to are left untouched.
+ *   tile_map [H][Npad] int32 (device)
+ */
+VEDA_API veda_status veda_unpermute(const void* o_tiled, void* o, const int32_t* tile_map, int32_t B,
+                           int32_t N, int32_t H, int32_t D, int32_t Npad, veda_stream_t stream);
+
+/*
+ * Synchronise `stream`, then read and clear the current device's status word.
+ * Returns VEDA_OK, VEDA_ERR_TIMEOUT, VEDA_ERR_DEVICE_CHECK or VEDA_ERR_CUDA.
+ * detail (may be NULL) receives the raw status bits (see VEDA_STATUS_* in the
+ * library source) -- 0 when clean.
+ */
+VEDA_API veda_status veda_check_device_status(veda_stream_t stream, uint32_t* detail);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* VEDA_H_ */

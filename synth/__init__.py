@@ -235,17 +235,24 @@ def make_inputs(w: Workload, heads: Optional[Sequence[int]] = None) -> Inputs:
         v = _rng(1000 * w.wid + 4).standard_normal((B, N, len(hs), D), dtype=np.float32)
     wq = (0.02 * _rng(1000 * w.wid + 5).standard_normal((H, D, 3 * D), dtype=np.float32))[hs]
     wk = (0.02 * _rng(1000 * w.wid + 6).standard_normal((H, D, 3 * D), dtype=np.float32))[hs]
-    order = None
-    if w.shuffle_heads:
-        g = _rng(1000 * w.wid + 7)
-        order = np.full((H, w.nT), -1, dtype=np.int32)
-        for h in range(H):
-            nv = w.video_tiles(w.head_shapes[h])
-            order[h, :nv] = g.permutation(nv).astype(np.int32)
+    order = tile_orders(w)
+    if order is not None:
         order = order[hs]
     return Inputs(_to_bf16(q), _to_bf16(k), _to_bf16(v),
                   torch.from_numpy(np.ascontiguousarray(wq)),
                   torch.from_numpy(np.ascontiguousarray(wk)), order)
+
+
+def tile_orders(w: Workload) -> Optional[np.ndarray]:
+    """Seeded per-head tile orders [H, nT] (first n_video_tiles entries used), or None."""
+    if not w.shuffle_heads:
+        return None
+    g = _rng(1000 * w.wid + 7)
+    order = np.full((w.H, w.nT), -1, dtype=np.int32)
+    for h in range(w.H):
+        nv = w.video_tiles(w.head_shapes[h])
+        order[h, :nv] = g.permutation(nv).astype(np.int32)
+    return order
 
 
 def head_subset(w: Workload, heads: Sequence[int]) -> Workload:

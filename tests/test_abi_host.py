@@ -1,0 +1,94 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol include/veda.h
+declares, its host-side tile maps match the oracle's bit for bit, and device calls
+validate their arguments before touching CUDA (and never fall back to anything)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import veda_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+veda = pytest.importorskip("block_sparse_attention_max_b200.veda")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from block_sparse_attention_max_b200 import build
+    build.build()
+    return veda.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "veda.h")).read()
+    return sorted(set(re.findall(r"VEDA_API\s+[\w\s\*]+?\b(veda_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared()
+    assert len(names) == 13
+    assert sorted(veda.EXPORTED) == names
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.veda_abi_version() == 1
+    assert L.veda_status_string(0) == b"ok"
+
+
+@pytest.mark.parametrize("w", [synth.TINY, synth.SMALL, synth.CLIP16x9, synth.MIXED])
+def test_tile_map_matches_oracle(L, w):
+    inp_order = synth.tile_orders(w)
+    maps = veda.build_tile_map(w.grid, w.head_shapes, w.n_tail, inp_order)
+    assert (maps.N, maps.nT, maps.Npad) == (w.N, w.nT, w.Npad)
+    om = [O.tile_map(w.grid, w.head_shapes[h], w.n_tail, None if inp_order is None else inp_order[h])
+          for h in range(w.H)]
+    slots, nv, seg = O.stack_maps(om, w.nT)
+    assert (maps.tile_map == slots).all()
+    assert (maps.tile_valid == nv).all()
+    assert (maps.tile_segment == seg).all()
+    assert (maps.nT_per_head == [len(m.n_valid) for m in om]).all()
+
+
+def test_tile_map_ragged_heads_and_rejections(L):
+    shapes = [(1, 8, 16), (2, 8, 8), (4, 4, 8)]
+    maps = veda.build_tile_map((5, 8, 16), shapes, 0)
+    assert list(maps.nT_per_head) == [5, 6, 8] and maps.nT == 8
+    om = [O.tile_map((5, 8, 16), s) for s in shapes]
+    slots, nv, seg = O.stack_maps(om, 8)
+    assert (maps.tile_map == slots).all() and (maps.tile_valid == nv).all()
+    with pytest.raises(veda.VedaError):
+        veda.build_tile_map((4, 8, 16), [(2, 8, 16)], 0)          # not 128 tokens
+    with pytest.raises(veda.VedaError):
+        veda.build_tile_map((4, 8, 16), [(1, 8, 16)], 0, np.zeros((1, 4), np.int32))  # not a permutation
+
+
+def test_device_calls_validate_before_cuda(L):
+    INVALID, UNSUPPORTED = 1, 2
+    assert L.veda_permute_tiles(None, None, None, 1, 1, 1, 128, 128, None) == INVALID
+    assert L.veda_permute_tiles(16, 16, 16, 1, 1, 1, 64, 128, None) == UNSUPPORTED
+    assert L.veda_permute_tiles(16, 16, 16, 1, 1, 1, 128, 100, None) == INVALID
+    assert L.veda_tile_pool(None, None, None, 1, 1, 1, 128, None) == INVALID
+    assert L.veda_block_scores(16, 16, 16, 16, 16, 256, 0, 1, 1, 4, 128, None) == INVALID  # workspace too small
+    num = (ctypes.c_int32 * 1)(1)
+    den = (ctypes.c_int32 * 1)(0)
+    assert L.veda_select_blocks(16, 16, 16, 16, 1, ctypes.addressof(num), ctypes.addressof(den),
+                                16, 16, 16, 16, 4, 1, 1, 4, None) == INVALID          # den = 0
+    den[0] = 2
+    assert L.veda_select_blocks(16, 16, 16, 16, 1, ctypes.addressof(num), ctypes.addressof(den),
+                                16, 16, 16, 16, 1, 1, 1, 8, None) == INVALID          # stride too small
+    assert L.veda_block_sparse_attn_fwd(16, 16, 16, 16, 16, 16, 16, 16, 4, -1.0, 16, None,
+                                        1, 1, 4, 128, None) == INVALID                 # bad scale
+    assert L.veda_block_sparse_attn_fwd(8, 16, 16, 16, 16, 16, 16, 16, 4, 0.1, 16, None,
+                                        1, 1, 4, 128, None) == INVALID                 # misaligned q
+    assert veda.block_scores_workspace_bytes(1, 2, 4) == 2 * 2 * 4 * 128 * 4
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_no_device_means_error_not_fallback(L):
+    # well-formed arguments reach the device query, which fails without a GPU
+    st = L.veda_permute_tiles(256, 256, 256, 1, 128, 1, 128, 128, None)
+    assert st in (2, 3)
+    assert L.veda_check_device_status(None, None) == 3

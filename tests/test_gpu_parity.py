@@ -1,0 +1,242 @@
+"""GPU parity: every step of the CUDA library against the fp64 oracle, through the C ABI.
+
+Stage tests feed both sides the same seeded inputs (the oracle's own output of the
+previous step, never the GPU's -- except the block selection, which the parity rule
+feeds the GPU's fp32 scores). The end-to-end tests run the public ``sparse_attention``
+path and compare every intermediate. Full-size workloads compare sampled heads and
+query tiles, in the launch configuration the benchmark times.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import veda_oracle as O
+import parity as P
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from block_sparse_attention_max_b200 import build
+    build.build()
+    V = P.veda()
+    V.lib()
+    yield
+    V.check_device_status()
+
+
+def _stage_run(w: synth.Workload, heads=None, rows=None, attn_rows=None):
+    """Stage-by-stage parity on workload w. heads: oracle heads checked (all if None)."""
+    V = P.veda()
+    inp = synth.make_inputs(w)
+    orders = inp.tile_order
+    slots, nv, seg, nTh = P.oracle_maps(w, orders)
+    hm = V.build_tile_map(w.grid, w.head_shapes, w.n_tail, orders)
+    assert (hm.tile_map == slots).all() and (hm.tile_valid == nv).all()
+    maps = hm.to(DEV)
+    hs = list(range(w.H)) if heads is None else list(heads)
+
+    # 1. permute: bit-exact
+    q_d, k_d, v_d = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    qt = V.permute_tiles(q_d, maps)
+    kt = V.permute_tiles(k_d, maps)
+    vt = V.permute_tiles(v_d, maps)
+    V.check_device_status()
+    xq = P.f64(inp.q[:, :, hs])
+    oq = O.permute(xq, slots[hs])
+    assert np.array_equal(P.f64(qt[:, hs]), oq), "permute differs"
+    ok_ = O.permute(P.f64(inp.k[:, :, hs]), slots[hs])
+    ov_ = O.permute(P.f64(inp.v[:, :, hs]), slots[hs])
+
+    # 2. pool (input: the oracle's tiles, as bf16 -- the same bytes)
+    pq_g = V.tile_pool(qt, maps)
+    pk_g = V.tile_pool(kt, maps)
+    pq_o = O.pool(oq, nv[hs])
+    pk_o = O.pool(ok_, nv[hs])
+    for g_, o_ in ((P.f64(pq_g[:, hs]), pq_o), (P.f64(pk_g[:, hs]), pk_o)):
+        assert np.array_equal(g_[..., 1:, :], o_[..., 1:, :]), "max/min differ"
+        assert np.allclose(g_[..., 0, :], o_[..., 0, :], rtol=1e-5, atol=1e-6), "mean differs"
+
+    # 3. scores from the oracle's pooled features rounded to fp32 (both sides)
+    pq32 = torch.from_numpy(pq_o.astype(np.float32))
+    pk32 = torch.from_numpy(pk_o.astype(np.float32))
+    wq, wk = inp.wq[hs].contiguous(), inp.wk[hs].contiguous()
+    S_g = V.block_scores(pq32.to(DEV), pk32.to(DEV), wq.to(DEV), wk.to(DEV))
+    S_o = O.scores(pq32.double().numpy(), pk32.double().numpy(), P.f64(wq), P.f64(wk))
+    err = P.score_errors(P.f64(S_g), S_o)
+    assert err <= P.SCORE_RTOL, f"score error {err}"
+
+    # 4. selection on the GPU's fp32 scores: bit-exact against the oracle's selection
+    sub = synth.head_subset(w, hs)
+    sub_maps = V.build_tile_map(sub.grid, sub.head_shapes, sub.n_tail,
+                                None if orders is None else orders[hs]).to(DEV)
+    lists_g = V.select_blocks(S_g, sub_maps, w.rho)
+    V.check_device_status()
+    S_g64 = P.f64(S_g)
+    lists_o = O.select(S_g64, nv[hs], seg[hs], [nTh[h] for h in hs], w.rho)
+    bad, total = P.gpu_lists_equal(lists_g, lists_o, range(len(hs)), rows)
+    assert bad == 0, f"{bad}/{total} block lists differ"
+    # budget invariants on the GPU lists
+    fc = lists_g.full_cnt.cpu().numpy() + lists_g.part_cnt.cpu().numpy()
+    for j, h in enumerate(hs):
+        k = O.budgets(nTh[h], seg[h], w.rho).sum(axis=1)
+        assert (fc[:, j, :nTh[h]] == k[None, :]).all()
+
+    # 5. attention with the oracle's lists (selection on the oracle's fp64 scores)
+    lists_ref = O.select(S_o, nv[hs], seg[hs], [nTh[h] for h in hs], w.rho)
+    stride = V.list_stride_for(w.nT, w.rho)
+    lists_dev = P.lists_to_device(lists_ref, w.B, len(hs), w.nT, stride, DEV)
+    qs = torch.from_numpy(oq).to(torch.bfloat16).to(DEV)
+    ks = torch.from_numpy(ok_).to(torch.bfloat16).to(DEV)
+    vs = torch.from_numpy(ov_).to(torch.bfloat16).to(DEV)
+    o_g, lse_g = V.block_sparse_attn_fwd(qs, ks, vs, sub_maps, lists_dev, P.SCALE)
+    V.check_device_status()
+    todo = attn_rows or [(b, j, r) for b in range(w.B) for j in range(len(hs)) for r in range(w.nT)]
+    o_o, lse_o = O.attention(oq, ok_, ov_, nv[hs], lists_ref, P.SCALE, rows=todo)
+    o_g64, lse_g64 = P.f64(o_g), P.f64(lse_g)
+    diffs, lse_d = [], []
+    for (b, j, r) in todo:
+        sl = slice(r * 128, (r + 1) * 128)
+        if r >= nTh[hs[j]]:
+            assert (o_g64[b, j, sl] == 0).all() and np.isneginf(lse_g64[b, j, sl]).all()
+            continue
+        diffs.append(np.abs(o_g64[b, j, sl] - o_o[b, j, sl]))
+        lse_d.append(np.abs(lse_g64[b, j, sl] - lse_o[b, j, sl]).max())
+    d = np.concatenate([x.ravel() for x in diffs])
+    assert d.max() <= P.ATTN_MAX_ABS and d.mean() <= P.ATTN_MEAN_ABS, (d.max(), d.mean())
+    assert max(lse_d) < 2e-3
+
+    # 6. unpermute of a seeded random tile tensor: bit-exact on valid rows
+    g = torch.Generator().manual_seed(99)
+    ot = torch.randn((w.B, w.H, w.Npad, 128), generator=g).to(torch.bfloat16)
+    o_r = V.unpermute(ot.to(DEV), maps, w.N)
+    V.check_device_status()
+    ref = O.unpermute(P.f64(ot[:, hs]), slots[hs], w.N)
+    assert np.array_equal(P.f64(o_r[:, :, hs]), ref), "unpermute differs"
+    return dict(d_max=float(d.max()), d_mean=float(d.mean()), score_err=err)
+
+
+def test_stages_tiny():
+    _stage_run(synth.TINY)
+
+
+def test_stages_small():
+    _stage_run(synth.SMALL)
+
+
+def test_stages_mixed_segments_and_shuffled_heads():
+    rng = np.random.default_rng(4)
+    heads = [0, 5, 16, 27]
+    rows = [(0, j, int(r)) for j in range(4) for r in rng.choice(229, 12, replace=False)]
+    rows += [(0, j, r) for j in range(4) for r in (224, 228)]     # audio query tiles
+    _stage_run(synth.MIXED, heads=heads, attn_rows=rows)
+
+
+def test_stages_ragged_heads_and_empty_rows():
+    # three tile shapes give 5, 6 and 8 tiles per head: rows past a head's tiles are empty,
+    # the grid is padded in t, and the tail makes a partial last tile
+    w = synth.Workload("ragged", 9, B=2, H=3, grid=(5, 8, 16),
+                       head_shapes=((1, 8, 16), (2, 8, 8), (4, 4, 8)), n_tail=77,
+                       rho=((1, 3), (1, 2)))
+    _stage_run(w)
+
+
+def test_stages_length_sweep_shortest():
+    _stage_run(synth.sweep_length(5), heads=[0, 17, 39],
+               attn_rows=[(0, j, r) for j in range(3) for r in (0, 1, 40, 79)])
+
+
+def test_full_density_equals_dense_attention():
+    # at 100% density the tiled sparse path (whole public API) is dense softmax attention
+    V = P.veda()
+    w = synth.Workload("dense", 10, B=1, H=2, grid=(3, 9, 20),
+                       head_shapes=((1, 8, 16), (2, 8, 8)), rho=((1, 1),), field=False)
+    inp = synth.make_inputs(w)
+    maps = V.build_tile_map(w.grid, w.head_shapes).to(DEV)
+    bufs = V.sparse_attention(inp.q.to(DEV), inp.k.to(DEV), inp.v.to(DEV), inp.wq.to(DEV),
+                              inp.wk.to(DEV), maps, w.rho, P.SCALE)
+    V.check_device_status()
+    od, _ = O.dense_attention_raster(P.f64(inp.q), P.f64(inp.k), P.f64(inp.v), P.SCALE)
+    dmax, dmean = P.attn_errors(P.f64(bufs.o), od)
+    assert dmax <= P.ATTN_MAX_ABS and dmean <= P.ATTN_MEAN_ABS, (dmax, dmean)
+
+
+def _end_to_end(w, heads=None, rows=None, attn_rows=None):
+    """Public API on the whole workload; every intermediate checked on some heads."""
+    V = P.veda()
+    inp = synth.make_inputs(w)
+    orders = inp.tile_order
+    slots, nv, seg, nTh = P.oracle_maps(w, orders)
+    maps = V.build_tile_map(w.grid, w.head_shapes, w.n_tail, orders).to(DEV)
+    bufs = V.sparse_attention(inp.q.to(DEV), inp.k.to(DEV), inp.v.to(DEV), inp.wq.to(DEV),
+                              inp.wk.to(DEV), maps, w.rho, P.SCALE)
+    V.check_device_status()
+    hs = list(range(w.H)) if heads is None else list(heads)
+    q64, k64, v64 = (P.f64(t[:, :, hs]) for t in (inp.q, inp.k, inp.v))
+    qt, kt, vt = (O.permute(x, slots[hs]) for x in (q64, k64, v64))
+    assert np.array_equal(P.f64(bufs.q_t[:, hs]), qt)
+    pq, pk = O.pool(qt, nv[hs]), O.pool(kt, nv[hs])
+    assert np.allclose(P.f64(bufs.pooled_q[:, hs]), pq, rtol=1e-5, atol=1e-6)
+    assert np.allclose(P.f64(bufs.pooled_k[:, hs]), pk, rtol=1e-5, atol=1e-6)
+    S_o = O.scores(pq, pk, P.f64(inp.wq[hs]), P.f64(inp.wk[hs]))
+    S_g = P.f64(bufs.scores[:, hs])
+    err = P.score_errors(S_g, S_o)
+    assert err <= P.SCORE_RTOL, err
+    lists_o = O.select(S_g, nv[hs], seg[hs], [nTh[h] for h in hs], w.rho)
+    bad, total = P.gpu_lists_equal(bufs.lists, lists_o, hs, rows)
+    assert bad == 0, f"{bad}/{total} lists differ"
+    # how often does fp64 selection pick differently (near-ties)? reported, not asserted
+    lists_64 = O.select(S_o, nv[hs], seg[hs], [nTh[h] for h in hs], w.rho)
+    bad64, _ = P.gpu_lists_equal(bufs.lists, lists_64, hs, rows)
+    todo = attn_rows or [(b, j, r) for b in range(w.B) for j in range(len(hs)) for r in range(nTh[hs[j]])]
+    o_t, _ = O.attention(qt, kt, vt, nv[hs], lists_o, P.SCALE, rows=todo)
+    o_g = P.f64(bufs.o_t[:, hs])
+    diffs = [np.abs(o_g[b, j, r * 128:(r + 1) * 128] - o_t[b, j, r * 128:(r + 1) * 128]) for (b, j, r) in todo]
+    d = np.concatenate([x.ravel() for x in diffs])
+    assert d.max() <= P.ATTN_MAX_ABS and d.mean() <= P.ATTN_MEAN_ABS, (d.max(), d.mean())
+    # raster output = unpermute of the tiled output (valid slots of the checked heads)
+    o_r = P.f64(bufs.o[:, :, hs])
+    assert np.array_equal(o_r, O.unpermute(P.f64(bufs.o_t[:, hs]), slots[hs], w.N))
+    return dict(lists_fp64_mismatch=bad64, total=total)
+
+
+def test_end_to_end_tiny():
+    _end_to_end(synth.TINY)
+
+
+def test_end_to_end_small():
+    r = _end_to_end(synth.SMALL)
+    assert r["lists_fp64_mismatch"] <= r["total"] // 20
+
+
+def test_end_to_end_clip16x9_full_size():
+    # the benchmark's workload and launch configuration; sampled heads and query tiles
+    rng = np.random.default_rng(3)
+    heads = [0, 13, 39]
+    rows = [int(r) for r in rng.choice(496, 40, replace=False)] + [0, 1, 495]
+    attn = [(0, j, r) for j in range(3) for r in rows[:8] + [0, 495]]
+    r = _end_to_end(synth.CLIP16x9, heads=heads, rows=rows, attn_rows=attn)
+    assert r["lists_fp64_mismatch"] <= r["total"] // 10
+
+
+def test_device_check_flags_bad_lists_without_fault():
+    # an out-of-range key index is caught by the kernel's own bounds check: it reads a
+    # valid tile instead, records VEDA_ERR_DEVICE_CHECK and the call returns normally
+    V = P.veda()
+    w = synth.TINY
+    inp = synth.make_inputs(w)
+    maps = V.build_tile_map(w.grid, w.head_shapes).to(DEV)
+    bufs = V.sparse_attention(inp.q.to(DEV), inp.k.to(DEV), inp.v.to(DEV), inp.wq.to(DEV),
+                              inp.wk.to(DEV), maps, w.rho, P.SCALE)
+    V.check_device_status()
+    bufs.lists.full_idx[0, 0, 1, 0] = 1000
+    V.block_sparse_attn_fwd(bufs.q_t, bufs.k_t, bufs.v_t, maps, bufs.lists, P.SCALE)
+    with pytest.raises(V.VedaError) as e:
+        V.check_device_status()
+    assert e.value.status == 5
+    V.check_device_status()       # the word was cleared
