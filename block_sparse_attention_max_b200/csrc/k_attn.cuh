@@ -172,6 +172,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             return false;
           bool b2;
           const int32_t idx = item_key(a, u, nf, j, b2);
+          if (b2) flag_status(ST_BAD_LIST);   // clamped to tile 0 by item_key
           const int32_t row = static_cast<int32_t>((bh * a.nT + idx) * 128);
           const uint32_t bar = smem_u32(&bars.k_full[st]);
           mbar_arrive_expect_tx(bar, kTileB);
