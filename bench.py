@@ -121,7 +121,7 @@ def run_veda(args):
     from block_sparse_attention_max_b200 import veda as V
     dist, rank, world = _dist()
     dev = torch.device("cuda", torch.cuda.current_device())
-    w = WORKLOAD
+    w = workload(args)
     peaks = _peaks()
 
     inp = synth.make_inputs(w)
@@ -253,10 +253,10 @@ def run_veda(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded smoothed-field Q/K, N(0,1) V, random-init projections)",
-        "config": {"workload": "clip16x9: B=1 H=40 grid 31x30x54 (50220 tokens) tile (1,8,16), "
+        "config": {"workload": f"clip16x9: B=1 H={H} grid 31x30x54 (50220 tokens) tile (1,8,16), "
                                "nT=496, density 1/10", "global_batch": world * B, "seq_len": N,
                    "parallelism": f"replicas x{world}", "visited_blocks": blocks,
-                   "l2": "inputs larger than L2 (Q/K/V 1.54 GB raster + 1.95 GB tiled per step)"},
+                   "l2": f"inputs larger than L2 ({3 * N * H * D * 2 / 1e9:.2f} GB raster Q/K/V per step)"},
         "attn_ms_per_call": attn_ms, "attn_tflops": attn_tflops,
         "attn_frac_bf16_peak": attn_tflops / peaks["bf16_sus"],
         "stage_ms": stage_ms, "hbm_stages": hbm,
@@ -277,6 +277,13 @@ def run_veda(args):
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def workload(args) -> synth.Workload:
+    """The 16:9-clip workload, or the same clip with fewer heads (--heads, for profiling)."""
+    if args.heads == WORKLOAD.H:
+        return WORKLOAD
+    return synth.head_subset(WORKLOAD, list(range(args.heads)))
 
 
 def _oracle_sample(inp, heads, rows_per_head):
@@ -362,6 +369,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=24)
+    ap.add_argument("--heads", type=int, default=WORKLOAD.H,
+                    help="heads of the 16:9 clip to run (default all 40; fewer for profiling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "veda":
         args.warmup = 3
