@@ -248,6 +248,41 @@ veda_status veda_block_scores(const float* pooled_q, const float* pooled_k, cons
   return launched("scores");
 }
 
+// Scratch of veda_block_scores_noalloc: part of the library's device image, so no call
+// ever allocates. Host code must not pass `g_noalloc_scratch` itself to a kernel (on the
+// host it is only a stand-in symbol); its device address is looked up once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[VEDA_NOALLOC_SCORES_BYTES];
+static void* g_noalloc_ptr[kMaxDevices] = {};
+
+veda_status veda_block_scores_noalloc(const float* pooled_q, const float* pooled_k, const float* Wq,
+                                      const float* Wk, float* scores, int32_t B, int32_t H, int32_t nT,
+                                      int32_t D, veda_stream_t stream) {
+  if (B <= 0 || H <= 0 || nT <= 0)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_scores_noalloc: bad size");
+  const size_t need = veda_block_scores_workspace_bytes(B, H, nT, D);
+  if (need > VEDA_NOALLOC_SCORES_BYTES)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_scores_noalloc: 2*B*H*nT*D*4 = " + std::to_string(need) +
+                                          " bytes exceeds the built-in scratch of " +
+                                          std::to_string(VEDA_NOALLOC_SCORES_BYTES) + " bytes");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(VEDA_ERR_UNSUPPORTED, "device ordinal out of range");
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);   // with `dev` current
+      if (e != cudaSuccess || p == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return veda_block_scores(pooled_q, pooled_k, Wq, Wk, scores, scratch, VEDA_NOALLOC_SCORES_BYTES, B, H, nT, D,
+                           stream);
+}
+
 veda_status veda_select_blocks(const float* scores, const int32_t* tile_valid, const int32_t* tile_segment,
                                const int32_t* nT_per_head, int32_t n_segments, const int32_t* rho_num,
                                const int32_t* rho_den, int32_t* full_cnt, int32_t* full_idx, int32_t* part_cnt,

@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "VEDA_OK", 1: "VEDA_ERR_INVALID_ARG", 2: "VEDA_ERR_UNSUPPORTE
 EXPORTED = (
     "veda_abi_version", "veda_status_string", "veda_last_error", "veda_geometry_sizes",
     "veda_build_tile_map", "veda_permute_tiles", "veda_tile_pool",
-    "veda_block_scores_workspace_bytes", "veda_block_scores", "veda_select_blocks",
+    "veda_block_scores_workspace_bytes", "veda_block_scores", "veda_block_scores_noalloc",
+    "veda_select_blocks",
     "veda_block_sparse_attn_fwd", "veda_unpermute", "veda_check_device_status",
 )
 
@@ -63,6 +64,7 @@ _SIG = {
     "veda_tile_pool": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
     "veda_block_scores_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "veda_block_scores": (_I, [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _P]),
+    "veda_block_scores_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "veda_select_blocks": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "veda_block_sparse_attn_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _F, _P, _P, _I, _I,
                                         _I, _I, _P]),
@@ -224,6 +226,26 @@ def block_scores(pooled_q: torch.Tensor, pooled_k: torch.Tensor, wq: torch.Tenso
     _check("veda_block_scores", lib().veda_block_scores(
         _ptr(pooled_q), _ptr(pooled_k), _ptr(wq), _ptr(wk), _ptr(out), _ptr(workspace),
         workspace.numel() * workspace.element_size(), B, H, nT, D, _stream(stream)))
+    return out
+
+
+def block_scores_noalloc(pooled_q: torch.Tensor, pooled_k: torch.Tensor, wq: torch.Tensor,
+                         wk: torch.Tensor, out: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """veda_block_scores_noalloc: same result as block_scores, scratch built into the library.
+
+    For callers that may not allocate device memory (see include/veda.h); ``out`` should
+    then be passed in. Calls sharing a device must not overlap on the GPU.
+    """
+    for t, n in ((pooled_q, "pooled_q"), (pooled_k, "pooled_k"), (wq, "wq"), (wk, "wk")):
+        _need(t, torch.float32, n)
+    B, H, nT, _, D = pooled_q.shape
+    if out is None:
+        out = torch.empty((B, H, nT, nT), dtype=torch.float32, device=pooled_q.device)
+    _need(out, torch.float32, "out")
+    _check("veda_block_scores_noalloc", lib().veda_block_scores_noalloc(
+        _ptr(pooled_q), _ptr(pooled_k), _ptr(wq), _ptr(wk), _ptr(out), B, H, nT, D,
+        _stream(stream)))
     return out
 
 

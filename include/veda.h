@@ -175,6 +175,36 @@ VEDA_API veda_status veda_block_scores(const float* pooled_q, const float* poole
                               veda_stream_t stream);
 
 /*
+ * Allocation-free variant of veda_block_scores (no counterpart on the pages: it only
+ * changes where the scratch memory comes from).
+ *
+ * Some callers cannot hand the library a workspace: a plugin inside a runtime that owns
+ * every device allocation and gives the plugin no allocator, or latency-critical code
+ * that must not call cudaMalloc (it can synchronise the whole device). This entry point
+ * takes the same inputs and outputs as veda_block_scores but uses a scratch array that
+ * is part of the library itself: a static __device__ array of
+ * VEDA_NOALLOC_SCORES_BYTES (32 MiB) that every GPU holds from the moment it loads the
+ * library until the process exits. It calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *   - Limit: 2 * B * H * nT * D * 4 bytes must not exceed VEDA_NOALLOC_SCORES_BYTES
+ *     (B * H * nT <= 32768 at D = 128); larger calls return VEDA_ERR_INVALID_ARG
+ *     without launching anything.
+ *   - Set-up: the first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before
+ *     any stream capture.
+ *   - Sharing: every call on a device uses the same array and leaves its contents
+ *     behind. Nothing in it needs to start at zero (each call overwrites all it reads),
+ *     but calls whose executions overlap on the GPU (different streams without
+ *     ordering, or concurrent host threads) race on it: order them.
+ * Results equal veda_block_scores' for the same inputs.
+ */
+#define VEDA_NOALLOC_SCORES_BYTES (32u * 1024u * 1024u)
+VEDA_API veda_status veda_block_scores_noalloc(const float* pooled_q, const float* pooled_k,
+                                               const float* Wq, const float* Wk, float* scores,
+                                               int32_t B, int32_t H, int32_t nT, int32_t D,
+                                               veda_stream_t stream);
+
+/*
  * Step 4: block lists of every query tile (device).
  * "Miowtion" README, Key Features / Veda sparse attention: equal-kernel-cost budgets
  * with Bresenham rounding, forced diagonal tiles, segmented budgets, full/partial
