@@ -360,6 +360,43 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """Density and length sweep of the attention step (not the contract line): for each
+    configuration, permute/pool/score/select once, then time the attention call alone
+    (CUDA events, median of --steps calls after --warmup). Writes one JSON line per
+    configuration; at 100% density the same kernel runs dense attention."""
+    from block_sparse_attention_max_b200 import veda as V
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = _peaks()
+    cfgs = [synth.sweep_density(p, q) for p, q in synth.SWEEP_DENSITIES]
+    cfgs += [synth.sweep_length(T) for T in synth.SWEEP_FRAMES]
+    for w in cfgs:
+        inp = synth.make_inputs(w)
+        maps = V.build_tile_map(w.grid, w.head_shapes, w.n_tail, inp.tile_order).to(dev)
+        q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+        B, N, H, D = q.shape
+        bufs = V.sparse_attention(q, k, v, inp.wq.to(dev), inp.wk.to(dev), maps, w.rho, SCALE)
+        V.check_device_status()
+        blocks = _visited_blocks(bufs.lists)
+        times = []
+        for it in range(args.warmup + args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            V.block_sparse_attn_fwd(bufs.q_t, bufs.k_t, bufs.v_t, maps, bufs.lists, SCALE, bufs.o_t, bufs.lse)
+            e1.record()
+            torch.cuda.synchronize()
+            if it >= args.warmup:
+                times.append(e0.elapsed_time(e1))
+        V.check_device_status()
+        ms = statistics.median(times)
+        tf = blocks * FLOP_PER_BLOCK / (ms * 1e-3) / 1e12
+        print(json.dumps({"sweep": w.name, "tokens": N, "nT": maps.nT, "density": f"{w.rho[0][0]}/{w.rho[0][1]}",
+                          "visited_blocks": blocks, "attn_ms": ms, "attn_tflops": tf,
+                          "frac_bf16_peak_burst": tf / peaks["bf16"]}), flush=True)
+        del bufs, q, k, v, inp
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -369,6 +406,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=24)
+    ap.add_argument("--sweep", action="store_true",
+                    help="density / length sweep of the attention step (one JSON line per config)")
     ap.add_argument("--heads", type=int, default=WORKLOAD.H,
                     help="heads of the 16:9 clip to run (default all 40; fewer for profiling)")
     args = ap.parse_args()
@@ -376,6 +415,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_veda(args)
 

@@ -292,12 +292,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tc_fence_after();
         float s[128];
         {
-          uint32_t r32[32];
+          // four 32-column loads in flight, one wait
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          const uint32_t sa = tmem + lane_off + kColS + sbuf * 128;
+          tmem_ld32(sa, r0);
+          tmem_ld32(sa + 32, r1);
+          tmem_ld32(sa + 64, r2);
+          tmem_ld32(sa + 96, r3);
+          tmem_wait_ld();
+          reg_fence32(r0); reg_fence32(r1); reg_fence32(r2); reg_fence32(r3);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            tmem_ld32_sync(tmem + lane_off + kColS + sbuf * 128 + c * 32, r32);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r32[i]);
+          for (int i = 0; i < 32; ++i) {
+            s[i] = __uint_as_float(r0[i]);
+            s[32 + i] = __uint_as_float(r1[i]);
+            s[64 + i] = __uint_as_float(r2[i]);
+            s[96 + i] = __uint_as_float(r3[i]);
           }
         }
         int32_t nv = 128;
@@ -313,9 +322,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int i = 0; i < 128; ++i)
             if (i >= nv) s[i] = -INFINITY;
         }
-        float mx = s[0];
+        // row max with eight independent chains (a single chain is 128 dependent steps)
+        float mx8[8];
 #pragma unroll
-        for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+        for (int c = 0; c < 8; ++c) mx8[c] = s[c];
+#pragma unroll
+        for (int i = 8; i < 128; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_blk = mx * a.scale_log2;
         if (j == 0) {
           m = m_blk;
@@ -345,13 +359,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 32)) { stop = true; break; }
           tc_fence_after();
         }
-        float rs = 0.f;
+        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int i = 0; i < 128; ++i) {
           s[i] = ex2_approx(fmaf(s[i], a.scale_log2, -m));
-          rs += s[i];
+          rs8[i & 7] += s[i];
         }
-        l += rs;
+        l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t p32[32];

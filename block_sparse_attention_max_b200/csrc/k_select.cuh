@@ -3,24 +3,26 @@
 //
 // "Miowtion" README, Key Features / Veda sparse attention: equal-kernel-cost budgets
 // with Bresenham rounding, forced diagonal tiles, segmented reference/target budgets,
-// full/partial block lists. One CTA per (batch, head, query row). Every candidate key
-// tile gets one 64-bit key that orders it within its segment:
-//   bits 48..51  segment
-//   bits 16..47  descending-order image of the fp32 score (-0 folded onto +0);
-//                0 is reserved for the diagonal, which therefore comes first
-//   bits  0..15  tile index (equal scores: lower index first)
-// After an ascending bitonic sort the k-th key of each segment is that segment's
-// threshold; a tile is selected when its key is at or below its segment's threshold.
-// Selected tiles are compacted in ascending index order.
+// full/partial block lists.
+//
+// One warp per (batch, head, query row). Each candidate key tile j gets a 32-bit rank
+// image u_j of its score (order-preserving, complemented so that the highest score has
+// the smallest image, -0 folded onto +0, NaN last); the diagonal gets u = 0, below any
+// real score. For every segment s the k_s-th smallest image T_s is found by a radix
+// select (four 8-bit digits, most significant first, one shared-memory histogram per
+// segment and digit). The row then takes every tile with u < T_s and, among the tiles
+// with u == T_s, the lowest indices until k_s are taken -- exactly "score descending,
+// ties to the lower index". Selected tiles are written in ascending index order by
+// ballot compaction, into the full list (tile_valid == 128) or the partial list.
 #pragma once
 
 #include "veda_ptx.cuh"
 
 namespace veda {
 
-constexpr int kSelThreads = 512;
+constexpr int kSelWarps = 2;                   // query rows per CTA
+constexpr int kSelThreads = 32 * kSelWarps;
 constexpr int kSelMaxTiles = 2048;
-constexpr int kSelPerThread = kSelMaxTiles / kSelThreads;   // 4
 constexpr int kMaxSeg = 4;
 
 struct SelectArgs {
@@ -36,8 +38,8 @@ struct SelectArgs {
   int32_t rho_num[kMaxSeg], rho_den[kMaxSeg];
 };
 
-// Order-preserving map of fp32 onto uint32 (ascending), then complemented so that the
-// highest score has the smallest image. -0 is folded onto +0; NaN ranks last.
+// Order-preserving map of fp32 onto uint32 (ascending), complemented so that the highest
+// score has the smallest image; -0 is folded onto +0 and NaN ranks last.
 __device__ __forceinline__ uint32_t score_rank_bits(float f, bool& is_nan) {
   is_nan = f != f;
   if (is_nan) return 0xFFFFFFFFu;
@@ -47,150 +49,168 @@ __device__ __forceinline__ uint32_t score_rank_bits(float f, bool& is_nan) {
   return ~u;   // +inf -> 0x007FFFFF; never 0
 }
 
-__global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectArgs a) {
-  __shared__ uint64_t keys[kSelMaxTiles];
-  __shared__ int32_t seg_count[kMaxSeg];
-  __shared__ int32_t warp_tot[2][kSelThreads / 32];
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
 
-  const int32_t r = blockIdx.x % a.nT;
-  const int32_t bh = blockIdx.x / a.nT;
-  const int32_t h = bh % a.H;
-  const int32_t tid = threadIdx.x;
-  const int64_t row = static_cast<int64_t>(bh) * a.nT + r;
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a) {
+  __shared__ uint32_t s_u[kSelWarps][kSelMaxTiles];
+  __shared__ uint8_t s_seg[kSelWarps][kSelMaxTiles];
+  __shared__ uint32_t s_hist[kSelWarps][kMaxSeg][256];
+
+  const int w = threadIdx.x >> 5;
+  const uint32_t lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kSelWarps + w;
+  if (row >= static_cast<int64_t>(a.B) * a.H * a.nT) return;
+  const int32_t r = static_cast<int32_t>(row % a.nT);
+  const int32_t h = static_cast<int32_t>((row / a.nT) % a.H);
   int32_t n = a.nT_per_head[h];
   if (n < 0 || n > a.nT) {
-    if (tid == 0) flag_status(ST_BAD_LIST);
+    if (lane == 0) flag_status(ST_BAD_LIST);
     n = 0;
   }
-  if (r >= n) {           // past the head's tiles: empty lists
-    if (tid == 0) { a.full_cnt[row] = 0; a.part_cnt[row] = 0; }
+  if (r >= n) {            // past the head's tiles: empty lists
+    if (lane == 0) { a.full_cnt[row] = 0; a.part_cnt[row] = 0; }
     return;
   }
+  const int32_t nseg = a.n_seg;
   const int32_t* seg_h = a.segment + static_cast<int64_t>(h) * a.nT;
   const int32_t* val_h = a.valid + static_cast<int64_t>(h) * a.nT;
   const float* srow = a.scores + row * a.nT;
+  uint32_t* su = s_u[w];
+  uint8_t* ss = s_seg[w];
 
-  if (tid < kMaxSeg) seg_count[tid] = 0;
-  __syncthreads();
-
-  // keys of this thread's tiles (contiguous block of kSelPerThread tiles)
-  int P = 1;
-  while (P < n) P <<= 1;
-  uint64_t mykey[kSelPerThread];
-  int32_t myseg[kSelPerThread];
-  int32_t local_cnt[kMaxSeg] = {0, 0, 0, 0};
-  bool saw_nan = false;
+  // candidates -> shared memory; tiles per segment
+  int32_t cnt[kMaxSeg] = {0, 0, 0, 0};
+  bool saw_nan = false, bad_seg = false;
+  for (int32_t j = static_cast<int32_t>(lane); j < n; j += 32) {
+    int32_t sg = seg_h[j];
+    if (sg < 0 || sg >= nseg) { bad_seg = true; sg = nseg - 1; }
+    bool nan = false;
+    uint32_t u = score_rank_bits(srow[j], nan);
+    saw_nan |= nan;
+    if (j == r) u = 0;
+    su[j] = u;
+    ss[j] = static_cast<uint8_t>(sg);
 #pragma unroll
-  for (int i = 0; i < kSelPerThread; ++i) {
-    const int32_t j = tid * kSelPerThread + i;
-    mykey[i] = ~0ull;
-    myseg[i] = -1;
-    if (j < n) {
-      int32_t sg = seg_h[j];
-      if (sg < 0 || sg >= a.n_seg) { flag_status(ST_BAD_LIST); sg = a.n_seg - 1; }
-      myseg[i] = sg;
-      bool nan = false;
-      uint32_t rank = score_rank_bits(srow[j], nan);
-      saw_nan |= nan;
-      if (j == r) rank = 0;
-      mykey[i] = (static_cast<uint64_t>(sg) << 48) | (static_cast<uint64_t>(rank) << 16) |
-                 static_cast<uint64_t>(j);
-#pragma unroll
-      for (int s = 0; s < kMaxSeg; ++s) local_cnt[s] += (sg == s);
-    }
-    if (j < P) keys[j] = mykey[i];
+    for (int s = 0; s < kMaxSeg; ++s) cnt[s] += (sg == s);
   }
   if (saw_nan) flag_status(ST_NAN_SCORE);
-#pragma unroll
-  for (int s = 0; s < kMaxSeg; ++s)
-    if (local_cnt[s]) atomicAdd(&seg_count[s], local_cnt[s]);
-  __syncthreads();
+  if (bad_seg) flag_status(ST_BAD_LIST);
+  int32_t own = seg_h[r];
+  if (own < 0 || own >= nseg) own = nseg - 1;
 
-  // ascending bitonic sort of keys[0, P)
-  for (int k = 2; k <= P; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int i = tid; i < P; i += kSelThreads) {
-        const int l = i ^ jj;
-        if (l > i) {
-          const uint64_t x = keys[i], y = keys[l];
-          const bool up = (i & k) == 0;
-          if ((x > y) == up) { keys[i] = y; keys[l] = x; }
-        }
-      }
-      __syncthreads();
-    }
-  }
-
-  // budgets of this row (exact integer Bresenham), threshold key per segment: the keys
-  // of segment s occupy sorted positions [start_s, start_s + nK_s)
-  const int32_t own = seg_h[r] < 0 || seg_h[r] >= a.n_seg ? a.n_seg - 1 : seg_h[r];
-  uint64_t thr[kMaxSeg];
-  int32_t budget[kMaxSeg];
-  int32_t start = 0;
+  // budgets of this row (exact integer Bresenham per segment)
+  int32_t k[kMaxSeg], krem[kMaxSeg];
+  uint32_t prefix[kMaxSeg];
 #pragma unroll
   for (int s = 0; s < kMaxSeg; ++s) {
-    thr[s] = 0;
-    budget[s] = 0;
-    if (s < a.n_seg) {
-      const int64_t nK = seg_count[s];
-      const int64_t num = nK * a.rho_num[s];
-      int64_t kk = ((r + 1) * num) / a.rho_den[s] - (static_cast<int64_t>(r) * num) / a.rho_den[s];
+    int32_t nK = cnt[s];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nK += __shfl_xor_sync(0xffffffffu, nK, o);
+    int64_t kk = 0;
+    if (s < nseg) {
+      const int64_t num = static_cast<int64_t>(nK) * a.rho_num[s];
+      kk = ((r + 1) * num) / a.rho_den[s] - (static_cast<int64_t>(r) * num) / a.rho_den[s];
       if (s == own && kk < 1) kk = 1;
       if (kk > nK) kk = nK;
       if (kk < 0) kk = 0;
-      budget[s] = static_cast<int32_t>(kk);
-      if (kk > 0) thr[s] = keys[start + kk - 1];
-      start += static_cast<int32_t>(nK);
     }
+    k[s] = static_cast<int32_t>(kk);
+    krem[s] = k[s];
+    prefix[s] = 0;
+  }
+  __syncwarp();
+
+  // radix select of the k_s-th smallest image per segment
+  for (int d = 3; d >= 0; --d) {
+    const int shift = 8 * d;
+    const uint32_t hi_mask = d == 3 ? 0u : (0xFFFFFFFFu << (shift + 8));
+    for (int i = static_cast<int>(lane); i < nseg * 256; i += 32) (&s_hist[w][0][0])[i] = 0;
+    __syncwarp();
+    for (int32_t j = static_cast<int32_t>(lane); j < n; j += 32) {
+      const uint32_t u = su[j];
+      const int sg = ss[j];
+      if (k[sg] > 0 && (u & hi_mask) == prefix[sg]) atomicAdd(&s_hist[w][sg][(u >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int s = 0; s < kMaxSeg; ++s) {
+      if (s >= nseg || k[s] == 0) continue;       // warp-uniform
+      uint32_t c8[8];
+      uint32_t local = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { c8[i] = s_hist[w][s][lane * 8 + i]; local += c8[i]; }
+      uint32_t incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= static_cast<uint32_t>(o)) incl += x;
+      }
+      uint32_t before = incl - local;
+      int found_bin = -1;
+      uint32_t found_before = 0;
+      const uint32_t want = static_cast<uint32_t>(krem[s]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (found_bin < 0 && before < want && want <= before + c8[i]) {
+          found_bin = static_cast<int>(lane * 8 + i);
+          found_before = before;
+        }
+        before += c8[i];
+      }
+      const uint32_t who = __ballot_sync(0xffffffffu, found_bin >= 0);
+      const int src = who ? __ffs(who) - 1 : 0;
+      found_bin = __shfl_sync(0xffffffffu, found_bin, src);
+      found_before = __shfl_sync(0xffffffffu, found_before, src);
+      if (found_bin >= 0) {
+        prefix[s] |= static_cast<uint32_t>(found_bin) << shift;
+        krem[s] -= static_cast<int32_t>(found_before);
+      }
+    }
+    __syncwarp();
   }
 
-  // selection flags: a tile is taken when its key ranks within its segment's budget
+  // selection and ascending compaction (chunks of 32 tiles in index order)
+  int32_t eq_taken[kMaxSeg] = {0, 0, 0, 0};
   int32_t nf = 0, np = 0;
-  bool selF[kSelPerThread], selP[kSelPerThread];
-#pragma unroll
-  for (int i = 0; i < kSelPerThread; ++i) {
-    const int32_t j = tid * kSelPerThread + i;
-    bool sel = false;
-    if (j < n) {
-      const int32_t sg = myseg[i];
-      sel = budget[sg] > 0 && mykey[i] <= thr[sg];
-    }
-    const bool full = sel && val_h[j] == 128;
-    selF[i] = full;
-    selP[i] = sel && !full;
-    nf += selF[i];
-    np += selP[i];
-  }
-  // block-wide exclusive scan of (nf, np) in thread order
-  const int lane = tid & 31, warp = tid >> 5;
-  int32_t sf = nf, sp = np;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int32_t xf = __shfl_up_sync(0xffffffffu, sf, o);
-    const int32_t xp = __shfl_up_sync(0xffffffffu, sp, o);
-    if (lane >= o) { sf += xf; sp += xp; }
-  }
-  if (lane == 31) { warp_tot[0][warp] = sf; warp_tot[1][warp] = sp; }
-  __syncthreads();
-  int32_t basef = 0, basep = 0, totf = 0, totp = 0;
-  for (int w = 0; w < kSelThreads / 32; ++w) {
-    if (w < warp) { basef += warp_tot[0][w]; basep += warp_tot[1][w]; }
-    totf += warp_tot[0][w];
-    totp += warp_tot[1][w];
-  }
-  int32_t pf = basef + sf - nf, pp = basep + sp - np;
   int32_t* fo = a.full_idx + row * a.stride;
   int32_t* po = a.part_idx + row * a.stride;
+  const uint32_t lt = lanemask_lt();
+  for (int32_t j0 = 0; j0 < n; j0 += 32) {
+    const int32_t j = j0 + static_cast<int32_t>(lane);
+    const bool in = j < n;
+    const int sg = in ? ss[j] : 0;
+    const uint32_t u = in ? su[j] : 0xFFFFFFFFu;
+    const bool take_seg = in && k[sg] > 0;
+    const bool less = take_seg && u < prefix[sg];
+    const bool eq = take_seg && u == prefix[sg];
+    int32_t rank = 0;
+    bool sel = less;
 #pragma unroll
-  for (int i = 0; i < kSelPerThread; ++i) {
-    const int32_t j = tid * kSelPerThread + i;
-    if (selF[i]) { if (pf < a.stride) fo[pf] = j; ++pf; }
-    if (selP[i]) { if (pp < a.stride) po[pp] = j; ++pp; }
+    for (int s = 0; s < kMaxSeg; ++s) {
+      const uint32_t be = __ballot_sync(0xffffffffu, eq && sg == s);
+      if (eq && sg == s) {
+        rank = eq_taken[s] + __popc(be & lt);
+        sel = rank < krem[s];
+      }
+      eq_taken[s] += __popc(be);
+    }
+    const bool full = sel && val_h[in ? j : 0] == 128;
+    const bool part = sel && !full;
+    const uint32_t bf = __ballot_sync(0xffffffffu, full);
+    const uint32_t bp = __ballot_sync(0xffffffffu, part);
+    if (full) { const int32_t p = nf + __popc(bf & lt); if (p < a.stride) fo[p] = j; }
+    if (part) { const int32_t p = np + __popc(bp & lt); if (p < a.stride) po[p] = j; }
+    nf += __popc(bf);
+    np += __popc(bp);
   }
-  if (tid == 0) {
-    if (totf > a.stride || totp > a.stride) flag_status(ST_LIST_OVERFLOW);
-    a.full_cnt[row] = totf < a.stride ? totf : a.stride;
-    a.part_cnt[row] = totp < a.stride ? totp : a.stride;
+  if (lane == 0) {
+    if (nf > a.stride || np > a.stride) flag_status(ST_LIST_OVERFLOW);
+    a.full_cnt[row] = nf < a.stride ? nf : a.stride;
+    a.part_cnt[row] = np < a.stride ? np : a.stride;
   }
 }
 

@@ -26,6 +26,7 @@ struct DeviceInfo {
   bool supported = false;
   int sms = 0;
   bool attrs_set = false;
+  int per_sm_copy = 1, per_sm_unpermute = 1, per_sm_pool = 1;   // resident CTAs per SM
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -74,19 +75,30 @@ veda_status current_device(int& sms) {
     return fail(VEDA_ERR_UNSUPPORTED, "the kernels are built for sm_100a (compute capability 10.0) only");
   if (!d.attrs_set) {
     struct { const void* f; int bytes; } attrs[] = {
-        {reinterpret_cast<const void*>(permute_kernel), kPermStages * static_cast<int>(kTileBytes) + 1024},
-        {reinterpret_cast<const void*>(unpermute_kernel), kUnpermStages * static_cast<int>(kTileBytes) + 1024},
-        {reinterpret_cast<const void*>(pool_kernel), kPoolStages * static_cast<int>(kTileBytes) + 1024},
         {reinterpret_cast<const void*>(attn::attn_fwd_kernel), static_cast<int>(attn::kSmemBytes)},
     };
     for (auto& x : attrs) {
       e = cudaFuncSetAttribute(x.f, cudaFuncAttributeMaxDynamicSharedMemorySize, x.bytes);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     }
+    // persistent grids: as many CTAs as can be resident at once
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_copy, permute_kernel, kCopyThreads, 0)) != cudaSuccess ||
+        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_unpermute, unpermute_kernel, kCopyThreads, 0)) != cudaSuccess ||
+        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_pool, pool_kernel, kPoolThreads, 0)) != cudaSuccess)
+      return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    d.per_sm_copy = d.per_sm_copy < 1 ? 1 : d.per_sm_copy;
+    d.per_sm_unpermute = d.per_sm_unpermute < 1 ? 1 : d.per_sm_unpermute;
+    d.per_sm_pool = d.per_sm_pool < 1 ? 1 : d.per_sm_pool;
     d.attrs_set = true;
   }
   sms = d.sms;
   return VEDA_OK;
+}
+
+const DeviceInfo& device_info() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return g_dev[dev];
 }
 
 veda_status get_encoder() {
@@ -161,7 +173,7 @@ veda_status veda_permute_tiles(const void* x, void* x_tiled, const int32_t* tile
   if (st != VEDA_OK) return st;
   GatherArgs a{static_cast<const uint8_t*>(x), static_cast<uint8_t*>(x_tiled), tile_map, B, N, H, Npad,
                Npad / 128, static_cast<int64_t>(B) * H * (Npad / 128)};
-  permute_kernel<<<grid_for(a.units, sms, 1), 32, kPermStages * kTileBytes + 1024,
+  permute_kernel<<<grid_for(a.units, sms, device_info().per_sm_copy), kCopyThreads, 0,
                    reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return launched("permute_kernel");
 }
@@ -177,7 +189,7 @@ veda_status veda_unpermute(const void* o_tiled, void* o, const int32_t* tile_map
   if (st != VEDA_OK) return st;
   GatherArgs a{static_cast<const uint8_t*>(o_tiled), static_cast<uint8_t*>(o), tile_map, B, N, H, Npad,
                Npad / 128, static_cast<int64_t>(B) * H * (Npad / 128)};
-  unpermute_kernel<<<grid_for(a.units, sms, 1), 32, kUnpermStages * kTileBytes + 1024,
+  unpermute_kernel<<<grid_for(a.units, sms, device_info().per_sm_unpermute), kCopyThreads, 0,
                      reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return launched("unpermute_kernel");
 }
@@ -193,7 +205,8 @@ veda_status veda_tile_pool(const void* x_tiled, const int32_t* tile_valid, float
   if (st != VEDA_OK) return st;
   PoolArgs a{static_cast<const uint8_t*>(x_tiled), tile_valid, pooled, B, H, nT,
              static_cast<int64_t>(B) * H * nT};
-  pool_kernel<<<grid_for(a.units, sms, 1), kPoolThreads, kPoolStages * kTileBytes + 1024,
+  const int64_t pool_ctas = (a.units + kPoolThreads / 32 - 1) / (kPoolThreads / 32);
+  pool_kernel<<<grid_for(pool_ctas, sms, device_info().per_sm_pool), kPoolThreads, 0,
                 reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return launched("pool_kernel");
 }
@@ -316,7 +329,8 @@ veda_status veda_select_blocks(const float* scores, const int32_t* tile_valid, c
   }
   const int64_t rows = static_cast<int64_t>(B) * H * nT;
   if (rows > INT32_MAX) return fail(VEDA_ERR_INVALID_ARG, "veda_select_blocks: too many rows");
-  select_kernel<<<static_cast<unsigned>(rows), kSelThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  select_kernel<<<static_cast<unsigned>((rows + kSelWarps - 1) / kSelWarps), kSelThreads, 0,
+                  reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return launched("select_kernel");
 }
 

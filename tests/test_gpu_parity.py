@@ -240,3 +240,14 @@ def test_device_check_flags_bad_lists_without_fault():
         V.check_device_status()
     assert e.value.status == 5
     V.check_device_status()       # the word was cleared
+
+
+@pytest.mark.parametrize("name,heads,rows", [
+    ("clip16x9_rho1_1", [7], [0, 250, 495]),          # 100% density: dense attention
+    ("clip16x9_rho1_2", [3], [1, 300]),
+    ("len_T62", [11], [0, 500, 991]),                 # 100k tokens, nT = 992
+])
+def test_sweep_extremes_sampled(name, heads, rows):
+    w = synth.get(name)
+    attn = [(0, 0, r) for r in rows]
+    _end_to_end(w, heads=heads, rows=rows, attn_rows=attn)
