@@ -7,17 +7,27 @@
 // function on partial blocks (here: key slots >= n_valid are masked).
 //
 // One persistent CTA per SM walks (batch, head, query tile) items in head-major order
-// (so the CTAs resident at one time share one head's K/V in L2). Roles:
-//   warp 4     TMA producer: Q tile, then K_j / V_j of the listed key tiles (128B swizzle)
-//   warp 5     MMA issuer (one thread): S = Q K^T into tensor memory (tcgen05, M=N=128,
-//              bf16 in, fp32 out), O += P V with P read from tensor memory
-//   warps 0-3  softmax + epilogue, one query row per thread (the 32x32b TMEM access
-//              shape gives each thread a whole row, so the row max and sum need no shuffle)
-// Tensor memory (512 columns): S0 | S1 | O | P0 | P1. Two S and P buffers let the MMA
-// compute S_{j+1} and P_{j-1} V_{j-1} while the softmax works on S_j. The running
-// maximum is only moved (and O rescaled in TMEM) when it grows by more than 2^8;
-// otherwise P is computed against the stale maximum, which is exact after the final
-// division by the row sum.
+// (so the CTAs resident at one time share one head's K/V in L2). A CTA works on two
+// query tiles at once ("slots" 0 and 1), so that while one slot's softmax runs the
+// tensor core works for the other:
+//   warpgroup 0 / 1   softmax + epilogue of slot 0 / 1, one query row per thread (the
+//                     32x32b TMEM access shape gives each thread a whole row, so the row
+//                     max and sum need no shuffle)
+//   warp 8            TMA producer: Q of each slot's item, then the K or V tile every MMA
+//                     op needs, in MMA order, through one 5-slot ring (128B swizzle)
+//   warp 9            MMA issuer (one thread, tcgen05.mma kind::f16, M = N = 128):
+//                     S_i = Q_i K^T (shared-memory operands, K-major) and
+//                     O_i += P_i V (P_i read from tensor memory, V MN-major)
+// Tensor memory: slot i owns columns [256 i, 256 i + 256): S_i in the first 128, O_i in
+// the next 128; P_i (bf16 pairs) is written over the first 64 columns of S_i once S_i
+// has been read. Per slot the MMA order is QK(0), PV(0), QK(1), PV(1), ...; tcgen05 MMAs
+// from one thread execute in issue order, so QK(j+1) overwrites S_i only after PV(j) has
+// read P_i. The two slots' streams are merged as QK0(0), QK1(0), PV0(0), QK0(1),
+// PV1(0), QK1(1), PV0(1), ...; the producer replays the same stream to fill the ring.
+// The running maximum is only moved (and O rescaled in place) when it grows by more
+// than 2^8; otherwise P uses the stale maximum, exact after the division by the row
+// sum. O_i is stable when S_i(j) is signalled: the commit that signals S_i(j) also
+// covers P_i(j-1) V.
 //
 // Every wait is bounded (veda_ptx.cuh): when one runs out the CTA raises a shared abort
 // flag, all roles leave their loops, in-flight copies and MMAs are drained with bounded
@@ -29,21 +39,24 @@
 namespace veda {
 namespace attn {
 
-constexpr int kThreads = 192;
-constexpr int kKStages = 3;
-constexpr int kVStages = 2;
-constexpr uint32_t kTileB = 32768;   // 128 x 128 bf16
-constexpr uint32_t kHalfB = 16384;   // 128 rows x 64 columns
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTileB;
-constexpr uint32_t kOffV = kOffK + kKStages * kTileB;
-constexpr uint32_t kSmemTiles = kOffV + kVStages * kTileB;   // 192 KB
-constexpr uint32_t kSmemBytes = kSmemTiles + 1024;           // + alignment slack
+constexpr int kThreads = 384;
+constexpr int kStages = 5;                 // K/V ring
+constexpr uint32_t kTileB = 32768;         // 128 x 128 bf16
+constexpr uint32_t kHalfB = 16384;         // 128 rows x 64 columns
+constexpr uint32_t kOffQ = 0;              // Q_0, Q_1
+constexpr uint32_t kOffRing = 2 * kTileB;
+constexpr uint32_t kSmemTiles = kOffRing + kStages * kTileB;   // 224 KB
+constexpr uint32_t kSmemBytes = kSmemTiles + 1024;             // + alignment slack
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;       // S_b at b*128, P_b at 384 + b*64
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);   // A, B K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);   // B (V) MN-major
 constexpr float kRescaleLog2 = 8.0f;
+// register split (setmaxnreg): two softmax warpgroups and one producer/MMA warpgroup;
+// the total equals the block's allocation at launch (384 threads x 168 registers)
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 224;
+constexpr int kControlRegs = 56;
+static_assert(2 * kSoftmaxRegs + kControlRegs <= 3 * kLaunchRegs, "register split exceeds the launch");
 
 struct Args {
   const int32_t* valid;      // [H][nT]
@@ -59,11 +72,10 @@ struct Args {
 };
 
 struct Bars {
-  uint64_t q_full, q_empty;
-  uint64_t k_full[kKStages], k_empty[kKStages];
-  uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[2], p_full[2], o_done[2];
-  uint64_t o_free, drain;
+  uint64_t full[kStages], empty[kStages];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full[2], p_full[2], o_done[2], o_free[2];
+  uint64_t drain;
   uint32_t tmem_base;
   int32_t abort;
 };
@@ -105,6 +117,99 @@ __device__ __forceinline__ bool warp_wait_abort(uint32_t bar, uint32_t parity, v
   return __all_sync(0xffffffffu, ok);
 }
 
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ------------------------------------------------------------------------------------
+// The merged MMA op stream of the two slots (replayed identically by producer and MMA).
+// Slot i takes the CTA's items m = i, i + 2, i + 4, ... (item u = blockIdx.x + m * grid)
+// that have at least one listed key tile.
+// ------------------------------------------------------------------------------------
+struct Op {
+  int32_t slot, j, n, nf;
+  int64_t u;
+  bool pv;         // P V (else Q K^T)
+  bool new_item;   // Q K^T of a slot's new item (needs its Q tile)
+  bool first_item; // the slot's first item (no earlier O to wait for)
+};
+
+struct Stream {
+  int64_t m[2];     // CTA-local item index of each slot's current item
+  int64_t u[2];
+  int32_t n[2], nf[2], j[2];
+  bool live[2], started[2];
+  int32_t slot_turn;   // slot whose unit comes next
+  int32_t pending_qk;  // after a slot's PV, its QK is emitted next (-1 if none)
+  int32_t init;        // initial QKs still to emit (2 .. 0)
+  int32_t items_done[2];
+
+  __device__ void seek(const Args& a, int s, int64_t from) {
+    live[s] = false;
+    for (int64_t mm = from;; mm += 2) {
+      const int64_t uu = blockIdx.x + mm * static_cast<int64_t>(gridDim.x);
+      if (uu >= a.items) return;
+      bool bad;
+      int32_t f;
+      const int32_t nn = item_blocks(a, uu, f, bad);
+      if (nn > 0) {
+        m[s] = mm; u[s] = uu; n[s] = nn; nf[s] = f; j[s] = 0; live[s] = true;
+        return;
+      }
+    }
+  }
+  __device__ void start(const Args& a) {
+    seek(a, 0, 0);
+    seek(a, 1, 1);
+    items_done[0] = items_done[1] = 0;
+    slot_turn = 0;
+    pending_qk = -1;
+    init = 0;
+  }
+  __device__ Op qk_op(int s, bool fresh) const {
+    Op o;
+    o.slot = s; o.j = j[s]; o.n = n[s]; o.nf = nf[s]; o.u = u[s]; o.pv = false;
+    o.new_item = fresh; o.first_item = items_done[s] == 0;
+    return o;
+  }
+  // Next op; false when both slots are done.
+  __device__ bool next(const Args& a, Op& o) {
+    if (init < 2) {                         // QK0(0), QK1(0)
+      while (init < 2) {
+        const int s = init++;
+        if (live[s]) { o = qk_op(s, true); return true; }
+      }
+    }
+    if (pending_qk >= 0) {                  // the QK that follows a slot's PV
+      const int s = pending_qk;
+      pending_qk = -1;
+      o = qk_op(s, j[s] == 0);
+      return true;
+    }
+    for (int t = 0; t < 2; ++t) {
+      const int s = (slot_turn + t) & 1;
+      if (!live[s]) continue;
+      slot_turn = s ^ 1;
+      o.slot = s; o.j = j[s]; o.n = n[s]; o.nf = nf[s]; o.u = u[s]; o.pv = true;
+      o.new_item = false; o.first_item = items_done[s] == 0;
+      if (j[s] + 1 < n[s]) {
+        ++j[s];
+      } else {
+        ++items_done[s];
+        seek(a, s, m[s] + 2);
+      }
+      if (live[s]) pending_qk = s;
+      return true;
+    }
+    return false;
+  }
+};
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const Args a) {
@@ -112,35 +217,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   __shared__ Bars bars;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
-  const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2;
   volatile int* abort = &bars.abort;
 
   if (tid == 0) {
-    mbar_init(smem_u32(&bars.q_full), 1);
-    mbar_init(smem_u32(&bars.q_empty), 1);
-    for (int i = 0; i < kKStages; ++i) {
-      mbar_init(smem_u32(&bars.k_full[i]), 1);
-      mbar_init(smem_u32(&bars.k_empty[i]), 1);
-    }
-    for (int i = 0; i < kVStages; ++i) {
-      mbar_init(smem_u32(&bars.v_full[i]), 1);
-      mbar_init(smem_u32(&bars.v_empty[i]), 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&bars.full[i]), 1);
+      mbar_init(smem_u32(&bars.empty[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars.q_full[i]), 1);
+      mbar_init(smem_u32(&bars.q_empty[i]), 1);
       mbar_init(smem_u32(&bars.s_full[i]), 1);
       mbar_init(smem_u32(&bars.p_full[i]), 4);
       mbar_init(smem_u32(&bars.o_done[i]), 1);
+      mbar_init(smem_u32(&bars.o_free[i]), 4);
     }
-    mbar_init(smem_u32(&bars.o_free), 4);
     mbar_init(smem_u32(&bars.drain), 1);
     bars.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(&bars.tmem_base), kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     prefetch_tensormap(&tmQ);
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
@@ -150,127 +251,108 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      uint32_t kc = 0, vc = 0, qc = 0;
-      bool stop = false;
-      for (int64_t u = blockIdx.x; u < a.items && !stop; u += gridDim.x) {
-        int32_t nf;
-        bool bad;
-        const int32_t n = item_blocks(a, u, nf, bad);
-        if (n == 0) continue;
-        const int64_t bh = u / a.nT;
-        if (qc > 0 && !mbar_wait(smem_u32(&bars.q_empty), (qc - 1) & 1, abort, 10)) break;
-        mbar_arrive_expect_tx(smem_u32(&bars.q_full), kTileB);
-        tma_load_2d(sb + kOffQ, &tmQ, smem_u32(&bars.q_full), 0, static_cast<int32_t>(u * 128));
-        tma_load_2d(sb + kOffQ + kHalfB, &tmQ, smem_u32(&bars.q_full), 64, static_cast<int32_t>(u * 128));
-        ++qc;
-        auto load_k = [&](int32_t j) -> bool {
-          const uint32_t st = kc % kKStages;
-          if (kc >= kKStages && !mbar_wait(smem_u32(&bars.k_empty[st]), (kc / kKStages - 1) & 1, abort, 11))
-            return false;
-          bool b2;
-          const int32_t idx = item_key(a, u, nf, j, b2);
-          if (b2) flag_status(ST_BAD_LIST);   // clamped to tile 0 by item_key
-          const int32_t row = static_cast<int32_t>((bh * a.nT + idx) * 128);
-          const uint32_t bar = smem_u32(&bars.k_full[st]);
-          mbar_arrive_expect_tx(bar, kTileB);
-          tma_load_2d(sb + kOffK + st * kTileB, &tmK, bar, 0, row);
-          tma_load_2d(sb + kOffK + st * kTileB + kHalfB, &tmK, bar, 64, row);
-          ++kc;
-          return true;
-        };
-        auto load_v = [&](int32_t j) -> bool {
-          const uint32_t st = vc % kVStages;
-          if (vc >= kVStages && !mbar_wait(smem_u32(&bars.v_empty[st]), (vc / kVStages - 1) & 1, abort, 12))
-            return false;
-          bool b2;
-          const int32_t idx = item_key(a, u, nf, j, b2);
-          const int32_t row = static_cast<int32_t>((bh * a.nT + idx) * 128);
-          const uint32_t bar = smem_u32(&bars.v_full[st]);
-          mbar_arrive_expect_tx(bar, kTileB);
-          tma_load_2d(sb + kOffV + st * kTileB, &tmV, bar, 0, row);
-          tma_load_2d(sb + kOffV + st * kTileB + kHalfB, &tmV, bar, 64, row);
-          ++vc;
-          return true;
-        };
-        for (int32_t j = 0; j < n && !stop; ++j) {
-          if (!load_k(j)) { stop = true; break; }
-          if (j >= 1 && !load_v(j - 1)) { stop = true; break; }
+  if (wg == 2) {
+    reg_dealloc<kControlRegs>();
+    if (warp == 8 && lane == 0) {
+      // ---------------------------------------------------------- TMA producer
+      Stream st;
+      st.start(a);
+      uint32_t lc = 0;           // ring loads issued
+      uint32_t qc[2] = {0, 0};   // Q loads issued per slot
+      Op o;
+      while (st.next(a, o)) {
+        const int s = o.slot;
+        if (o.new_item) {
+          if (qc[s] > 0 && !mbar_wait(smem_u32(&bars.q_empty[s]), (qc[s] - 1) & 1, abort, 10)) break;
+          const uint32_t qb = smem_u32(&bars.q_full[s]);
+          mbar_arrive_expect_tx(qb, kTileB);
+          tma_load_2d(sb + kOffQ + s * kTileB, &tmQ, qb, 0, static_cast<int32_t>(o.u * 128));
+          tma_load_2d(sb + kOffQ + s * kTileB + kHalfB, &tmQ, qb, 64, static_cast<int32_t>(o.u * 128));
+          ++qc[s];
         }
-        if (!stop && !load_v(n - 1)) stop = true;
+        const uint32_t stg = lc % kStages;
+        if (lc >= kStages && !mbar_wait(smem_u32(&bars.empty[stg]), (lc / kStages - 1) & 1, abort, 11)) break;
+        bool bad;
+        const int32_t idx = item_key(a, o.u, o.nf, o.j, bad);
+        if (bad) flag_status(ST_BAD_LIST);
+        const int32_t row = static_cast<int32_t>(((o.u / a.nT) * a.nT + idx) * 128);
+        const uint32_t fb = smem_u32(&bars.full[stg]);
+        const CUtensorMap* map = o.pv ? &tmV : &tmK;
+        mbar_arrive_expect_tx(fb, kTileB);
+        tma_load_2d(sb + kOffRing + stg * kTileB, map, fb, 0, row);
+        tma_load_2d(sb + kOffRing + stg * kTileB + kHalfB, map, fb, 64, row);
+        ++lc;
       }
       if (*abort) {
         // let the copies this thread issued land before the CTA exits
-        for (uint32_t i = kc > kKStages ? kc - kKStages : 0; i < kc; ++i)
-          mbar_wait(smem_u32(&bars.k_full[i % kKStages]), (i / kKStages) & 1, nullptr, 13);
-        for (uint32_t i = vc > kVStages ? vc - kVStages : 0; i < vc; ++i)
-          mbar_wait(smem_u32(&bars.v_full[i % kVStages]), (i / kVStages) & 1, nullptr, 14);
-        if (qc > 0) mbar_wait(smem_u32(&bars.q_full), (qc - 1) & 1, nullptr, 15);
+        for (uint32_t i = lc > kStages ? lc - kStages : 0; i < lc; ++i)
+          mbar_wait(smem_u32(&bars.full[i % kStages]), (i / kStages) & 1, nullptr, 13);
+        for (int s = 0; s < 2; ++s)
+          if (qc[s] > 0) mbar_wait(smem_u32(&bars.q_full[s]), (qc[s] - 1) & 1, nullptr, 14);
       }
-    }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t kc = 0, vc = 0, qc = 0, g = 0;
-      bool stop = false;
-      auto pv = [&](uint32_t gp, bool first) -> bool {
-        const uint32_t pb = gp & 1;
-        if (!mbar_wait(smem_u32(&bars.p_full[pb]), (gp >> 1) & 1, abort, 20)) return false;
-        const uint32_t vs = vc % kVStages;
-        if (!mbar_wait(smem_u32(&bars.v_full[vs]), (vc / kVStages) & 1, abort, 21)) return false;
-        if (first && qc >= 2 && !mbar_wait(smem_u32(&bars.o_free), (qc - 2) & 1, abort, 22)) return false;
+    } else if (warp == 9 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      Stream st;
+      st.start(a);
+      uint32_t lc = 0;                    // ring tiles consumed
+      uint32_t qc[2] = {0, 0};            // Q tiles consumed per slot
+      uint32_t pc[2] = {0, 0};            // P tiles consumed per slot
+      uint32_t oc[2] = {0, 0};            // items whose O was finished per slot
+      Op o;
+      while (st.next(a, o)) {
+        const int s = o.slot;
+        const uint32_t s_col = tmem + s * 256, o_col = s_col + 128;
+        if (!o.pv) {
+          if (o.new_item) {
+            if (!mbar_wait(smem_u32(&bars.q_full[s]), qc[s] & 1, abort, 20)) break;
+            ++qc[s];
+          }
+        } else {
+          if (!mbar_wait(smem_u32(&bars.p_full[s]), pc[s] & 1, abort, 21)) break;
+          ++pc[s];
+          // the first P V of an item overwrites O_i: the previous item's epilogue must be done
+          if (o.j == 0 && !o.first_item && !mbar_wait(smem_u32(&bars.o_free[s]), (oc[s] - 1) & 1, abort, 22))
+            break;
+        }
+        const uint32_t stg = lc % kStages;
+        if (!mbar_wait(smem_u32(&bars.full[stg]), (lc / kStages) & 1, abort, 23)) break;
         tc_fence_after();
-        const uint32_t vt = sb + kOffV + vs * kTileB;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + kColO, tmem + kColP + pb * 64 + kk * 8, desc_mnmajor(vt, kk), kIdescPV,
-                 (first && kk == 0) ? 0u : 1u);
-        tc_commit(smem_u32(&bars.o_done[pb]));
-        tc_commit(smem_u32(&bars.v_empty[vs]));
-        ++vc;
-        return true;
-      };
-      for (int64_t u = blockIdx.x; u < a.items && !stop; u += gridDim.x) {
-        int32_t nf;
-        bool bad;
-        const int32_t n = item_blocks(a, u, nf, bad);
-        if (n == 0) continue;
-        if (!mbar_wait(smem_u32(&bars.q_full), qc & 1, abort, 23)) break;
-        ++qc;
-        tc_fence_after();
-        for (int32_t j = 0; j < n; ++j) {
-          const uint32_t st = kc % kKStages;
-          if (!mbar_wait(smem_u32(&bars.k_full[st]), (kc / kKStages) & 1, abort, 24)) { stop = true; break; }
-          tc_fence_after();
-          const uint32_t kt = sb + kOffK + st * kTileB;
-          const uint32_t sbuf = g & 1;
+        const uint32_t tile = sb + kOffRing + stg * kTileB;
+        if (!o.pv) {
+          const uint32_t qt = sb + kOffQ + s * kTileB;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + kColS + sbuf * 128, desc_kmajor(sb + kOffQ, kk), desc_kmajor(kt, kk), kIdescQK,
-                   kk > 0 ? 1u : 0u);
-          tc_commit(smem_u32(&bars.s_full[sbuf]));
-          tc_commit(smem_u32(&bars.k_empty[st]));
-          ++kc;
-          if (j == n - 1) tc_commit(smem_u32(&bars.q_empty));
-          if (j >= 1 && !pv(g - 1, j == 1)) { stop = true; break; }
-          ++g;
+            mma_ss(s_col, desc_kmajor(qt, kk), desc_kmajor(tile, kk), kIdescQK, kk > 0 ? 1u : 0u);
+          tc_commit(smem_u32(&bars.s_full[s]));
+          if (o.j == o.n - 1) tc_commit(smem_u32(&bars.q_empty[s]));
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(o_col, s_col + kk * 8, desc_mnmajor(tile, kk), kIdescPV, (o.j == 0 && kk == 0) ? 0u : 1u);
+          if (o.j == o.n - 1) {
+            tc_commit(smem_u32(&bars.o_done[s]));
+            ++oc[s];
+          }
         }
-        if (stop) break;
-        if (!pv(g - 1, n == 1)) break;
+        tc_commit(smem_u32(&bars.empty[stg]));
+        ++lc;
       }
       // drain: every MMA issued so far completes before the tensor memory is freed
       tc_commit(smem_u32(&bars.drain));
       mbar_wait(smem_u32(&bars.drain), 0, nullptr, 25);
     }
   } else {
+    reg_alloc<kSoftmaxRegs>();
     // ------------------------------------------------------------ softmax + epilogue
-    const uint32_t row = tid;                                  // 0..127 = TMEM lane
-    const uint32_t lane_off = (warp * 32u) << 16;
-    uint32_t g = 0;
+    const int slot = static_cast<int>(wg);
+    const uint32_t row = tid & 127;                              // TMEM lane
+    const uint32_t lane_off = ((warp & 3) * 32u) << 16;
+    const uint32_t s_col = tmem + lane_off + slot * 256, o_col = s_col + 128;
+    uint32_t sc = 0, ic = 0;      // S tiles consumed, items finished (this slot)
     bool stop = false;
-    for (int64_t u = blockIdx.x; u < a.items && !stop; u += gridDim.x) {
+    for (int64_t mm = slot;; mm += 2) {
+      const int64_t u = blockIdx.x + mm * static_cast<int64_t>(gridDim.x);
+      if (u >= a.items || stop) break;
       int32_t nf;
       bool bad;
       const int32_t n = item_blocks(a, u, nf, bad);
@@ -287,18 +369,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       float m = -INFINITY, l = 0.f;
       bool list_bad = false;
       for (int32_t j = 0; j < n; ++j) {
-        const uint32_t sbuf = g & 1;
-        if (!warp_wait_abort(smem_u32(&bars.s_full[sbuf]), (g >> 1) & 1, abort, 30)) { stop = true; break; }
+        if (!warp_wait_abort(smem_u32(&bars.s_full[slot]), sc & 1, abort, 30)) { stop = true; break; }
+        ++sc;
         tc_fence_after();
         float s[128];
         {
-          // four 32-column loads in flight, one wait
           uint32_t r0[32], r1[32], r2[32], r3[32];
-          const uint32_t sa = tmem + lane_off + kColS + sbuf * 128;
-          tmem_ld32(sa, r0);
-          tmem_ld32(sa + 32, r1);
-          tmem_ld32(sa + 64, r2);
-          tmem_ld32(sa + 96, r3);
+          tmem_ld32(s_col, r0);
+          tmem_ld32(s_col + 32, r1);
+          tmem_ld32(s_col + 64, r2);
+          tmem_ld32(s_col + 96, r3);
           tmem_wait_ld();
           reg_fence32(r0); reg_fence32(r1); reg_fence32(r2); reg_fence32(r3);
 #pragma unroll
@@ -322,7 +402,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int i = 0; i < 128; ++i)
             if (i >= nv) s[i] = -INFINITY;
         }
-        // row max with eight independent chains (a single chain is 128 dependent steps)
         float mx8[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) mx8[c] = s[c];
@@ -336,28 +415,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         } else {
           const bool need = m_blk > m + kRescaleLog2;
           if (__any_sync(0xffffffffu, need)) {
-            // O must hold P V of every earlier block before it is rescaled
-            const uint32_t gp = g - 1;
-            if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 31)) { stop = true; break; }
-            tc_fence_after();
+            // O_i already holds P V of every earlier block (covered by the S commit)
             const float alpha = need ? ex2_approx(m - m_blk) : 1.0f;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               uint32_t r32[32];
-              tmem_ld32_sync(tmem + lane_off + kColO + c * 32, r32);
+              tmem_ld32_sync(o_col + c * 32, r32);
 #pragma unroll
               for (int i = 0; i < 32; ++i) r32[i] = __float_as_uint(__uint_as_float(r32[i]) * alpha);
-              tmem_st32(tmem + lane_off + kColO + c * 32, r32);
+              tmem_st32(o_col + c * 32, r32);
             }
             tmem_wait_st();
             if (need) { l *= alpha; m = m_blk; }
           }
-        }
-        // P_b is free once P_{g-2} V_{g-2} has completed
-        if (g >= 2) {
-          const uint32_t gp = g - 2;
-          if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 32)) { stop = true; break; }
-          tc_fence_after();
         }
         float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -371,25 +441,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           uint32_t p32[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) p32[i] = pack_bf16x2(s[c * 64 + 2 * i], s[c * 64 + 2 * i + 1]);
-          tmem_st32(tmem + lane_off + kColP + sbuf * 64 + c * 32, p32);
+          tmem_st32(s_col + c * 32, p32);   // P over the first 64 columns of S
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars.p_full[sbuf]));
-        ++g;
+        if (lane == 0) mbar_arrive(smem_u32(&bars.p_full[slot]));
       }
       if (stop) break;
       if (list_bad && row == 0) flag_status(ST_BAD_LIST);
       // epilogue: O / l -> bf16 rows, LSE
-      const uint32_t gl = g - 1;
-      if (!warp_wait_abort(smem_u32(&bars.o_done[gl & 1]), (gl >> 1) & 1, abort, 33)) break;
+      if (!warp_wait_abort(smem_u32(&bars.o_done[slot]), ic & 1, abort, 33)) break;
+      ++ic;
       tc_fence_after();
       const float inv_l = 1.0f / l;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t r32[32];
-        tmem_ld32_sync(tmem + lane_off + kColO + c * 32, r32);
+        tmem_ld32_sync(o_col + c * 32, r32);
         uint32_t packed[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -401,14 +470,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (a.lse) a.lse[grow] = (m + __log2f(l)) * 0.69314718055994531f;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars.o_free));
+      if (lane == 0) mbar_arrive(smem_u32(&bars.o_free[slot]));
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 9) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace attn

@@ -81,6 +81,15 @@ veda_status current_device(int& sms) {
       e = cudaFuncSetAttribute(x.f, cudaFuncAttributeMaxDynamicSharedMemorySize, x.bytes);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     }
+    // the attention kernel re-splits its registers between warpgroups (setmaxnreg); the
+    // split assumes the launch allocation it was built for, so refuse any other build
+    cudaFuncAttributes fa{};
+    if ((e = cudaFuncGetAttributes(&fa, attn::attn_fwd_kernel)) != cudaSuccess)
+      return cuda_fail(e, "cudaFuncGetAttributes");
+    if (fa.numRegs != attn::kLaunchRegs)
+      return fail(VEDA_ERR_UNSUPPORTED, "attention kernel built with " + std::to_string(fa.numRegs) +
+                                            " registers per thread; its register split needs " +
+                                            std::to_string(attn::kLaunchRegs));
     // persistent grids: as many CTAs as can be resident at once
     if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_copy, permute_kernel, kCopyThreads, 0)) != cudaSuccess ||
         (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_unpermute, unpermute_kernel, kCopyThreads, 0)) != cudaSuccess ||
@@ -366,6 +375,25 @@ veda_status veda_block_sparse_attn_fwd(const void* q, const void* k, const void*
   attn::attn_fwd_kernel<<<grid_for(a.items, sms, 1), attn::kThreads, attn::kSmemBytes,
                           reinterpret_cast<cudaStream_t>(stream)>>>(tq, tk, tv, a);
   return launched("attn_fwd_kernel");
+}
+
+// Self-test of the bounded waits: one thread waits on an mbarrier that nothing arrives
+// on; the wait gives up after `limit_ns`, records the timeout and the kernel returns.
+__global__ void wait_selftest_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  mbar_init(smem_u32(&bar), 1);
+  fence_mbar_init();
+  mbar_wait(smem_u32(&bar), 0, nullptr, 0xEE, limit_ns);
+}
+
+veda_status veda_selftest_wait_timeout(uint32_t limit_us, veda_stream_t stream) {
+  if (limit_us == 0 || limit_us > 1000000)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_selftest_wait_timeout: limit must be 1..1000000 us");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  wait_selftest_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_us) * 1000u);
+  return launched("wait_selftest_kernel");
 }
 
 veda_status veda_check_device_status(veda_stream_t stream, uint32_t* detail) {

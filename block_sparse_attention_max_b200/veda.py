@@ -28,6 +28,7 @@ EXPORTED = (
     "veda_block_scores_workspace_bytes", "veda_block_scores", "veda_block_scores_noalloc",
     "veda_select_blocks",
     "veda_block_sparse_attn_fwd", "veda_unpermute", "veda_check_device_status",
+    "veda_selftest_wait_timeout",
 )
 
 
@@ -70,6 +71,7 @@ _SIG = {
                                         _I, _I, _P]),
     "veda_unpermute": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "veda_check_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "veda_selftest_wait_timeout": (_I, [ctypes.c_uint32, _P]),
 }
 
 
@@ -322,6 +324,11 @@ def check_device_status(stream=None) -> int:
     st = lib().veda_check_device_status(_stream(stream), ctypes.byref(detail))
     _check("veda_check_device_status", st)
     return detail.value
+
+
+def selftest_wait_timeout(limit_us: int = 2000, stream=None) -> None:
+    """Launch the bounded-wait self-test (see include/veda.h); check the status afterwards."""
+    _check("veda_selftest_wait_timeout", lib().veda_selftest_wait_timeout(int(limit_us), _stream(stream)))
 
 
 # ---------------------------------------------------------------------------------------

@@ -273,6 +273,16 @@ VEDA_API veda_status veda_unpermute(const void* o_tiled, void* o, const int32_t*
                            int32_t N, int32_t H, int32_t D, int32_t Npad, veda_stream_t stream);
 
 /*
+ * Self-test of the library's failure detection (no counterpart on the pages). Launches
+ * one thread that waits on an mbarrier nothing will ever arrive on, through the same
+ * bounded-wait routine every kernel of the library uses, with a limit of `limit_us`
+ * microseconds (1 .. 1,000,000). The wait gives up, records a timeout in the status word
+ * and the kernel returns normally: the next veda_check_device_status() returns
+ * VEDA_ERR_TIMEOUT (site 0xEE in the detail bits) and the context stays usable.
+ */
+VEDA_API veda_status veda_selftest_wait_timeout(uint32_t limit_us, veda_stream_t stream);
+
+/*
  * Synchronise `stream`, then read and clear the current device's status word.
  * Returns VEDA_OK, VEDA_ERR_TIMEOUT, VEDA_ERR_DEVICE_CHECK or VEDA_ERR_CUDA.
  * detail (may be NULL) receives the raw status bits (see VEDA_STATUS_* in the

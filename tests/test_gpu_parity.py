@@ -251,3 +251,16 @@ def test_sweep_extremes_sampled(name, heads, rows):
     w = synth.get(name)
     attn = [(0, 0, r) for r in rows]
     _end_to_end(w, heads=heads, rows=rows, attn_rows=attn)
+
+
+def test_bounded_wait_runs_out_and_context_survives():
+    # failure detection without a fault: a wait on a barrier nothing arrives on gives up
+    # after 2 ms, the status word says VEDA_ERR_TIMEOUT, and the next call works
+    V = P.veda()
+    V.check_device_status()
+    V.selftest_wait_timeout(2000)
+    with pytest.raises(V.VedaError) as e:
+        V.check_device_status()
+    assert e.value.status == 4
+    V.check_device_status()
+    _stage_run(synth.TINY)
