@@ -71,8 +71,21 @@ struct Args {
   float scale_log2;          // softmax scale * log2(e)
 };
 
+// One word per ring slot, written by the producer before it arms the slot: what the MMA
+// issuer has to do with the tile.
+enum : uint32_t {
+  kOpPV = 1u << 0,        // P V (else Q K^T)
+  kOpNewItem = 1u << 1,   // Q K^T of a slot's new item: wait for its Q tile
+  kOpFirstBlk = 1u << 2,  // block 0 of the item (P V overwrites O)
+  kOpLastBlk = 1u << 3,   // last block of the item
+  kOpSlot1 = 1u << 4,     // slot 1 (else slot 0)
+  kOpFirstItem = 1u << 5, // the slot's first item (no earlier O to wait for)
+  kOpStop = 1u << 6,      // end of the stream (no tile)
+};
+
 struct Bars {
   uint64_t full[kStages], empty[kStages];
+  uint32_t op[kStages];
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[2], p_full[2], o_done[2], o_free[2];
   uint64_t drain;
@@ -106,15 +119,29 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int kk) {
   return smem_desc_sw128(tile + kk * 2048, kHalfB, 1024);
 }
 
-// Whole-warp bounded wait: lane 0 waits, the verdict is shared, and every lane then
-// observes the completed phase itself.
+// Whole-warp bounded wait: every lane polls the barrier and the warp leaves together
+// (a completed phase stays completed until the warp consumes it, so once one lane sees
+// it, all lanes do on their next poll). Fast path: one try_wait and one vote.
 __device__ __forceinline__ bool warp_wait_abort(uint32_t bar, uint32_t parity, volatile int* abort,
                                                 uint32_t site) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, site);
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  if (ok) ok = mbar_try_wait(bar, parity);
-  return __all_sync(0xffffffffu, ok);
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    if ((it & 31u) == 0) {
+      int give_up = 0;
+      if ((threadIdx.x & 31) == 0) {
+        if (*abort) {
+          give_up = 1;
+        } else if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          flag_status(ST_TIMEOUT | ((site & 0xffu) << ST_WAIT_SITE_SHIFT));
+          *abort = 1;
+          give_up = 1;
+        }
+      }
+      if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
+    }
+  }
 }
 
 template <int N>
@@ -278,10 +305,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int32_t row = static_cast<int32_t>(((o.u / a.nT) * a.nT + idx) * 128);
         const uint32_t fb = smem_u32(&bars.full[stg]);
         const CUtensorMap* map = o.pv ? &tmV : &tmK;
+        bars.op[stg] = (o.pv ? kOpPV : 0u) | (o.new_item ? kOpNewItem : 0u) | (o.j == 0 ? kOpFirstBlk : 0u) |
+                       (o.j == o.n - 1 ? kOpLastBlk : 0u) | (s ? kOpSlot1 : 0u) | (o.first_item ? kOpFirstItem : 0u);
         mbar_arrive_expect_tx(fb, kTileB);
         tma_load_2d(sb + kOffRing + stg * kTileB, map, fb, 0, row);
         tma_load_2d(sb + kOffRing + stg * kTileB + kHalfB, map, fb, 64, row);
         ++lc;
+      }
+      if (!*abort) {
+        // end of stream: one more ring slot carrying only the stop record
+        const uint32_t stg = lc % kStages;
+        if (lc < kStages || mbar_wait(smem_u32(&bars.empty[stg]), (lc / kStages - 1) & 1, abort, 12)) {
+          bars.op[stg] = kOpStop;
+          mbar_arrive(smem_u32(&bars.full[stg]));
+        }
       }
       if (*abort) {
         // let the copies this thread issued land before the CTA exits
@@ -292,50 +329,60 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
     } else if (warp == 9 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      Stream st;
-      st.start(a);
-      uint32_t lc = 0;                    // ring tiles consumed
-      uint32_t qc[2] = {0, 0};            // Q tiles consumed per slot
-      uint32_t pc[2] = {0, 0};            // P tiles consumed per slot
-      uint32_t oc[2] = {0, 0};            // items whose O was finished per slot
-      Op o;
-      while (st.next(a, o)) {
-        const int s = o.slot;
-        const uint32_t s_col = tmem + s * 256, o_col = s_col + 128;
-        if (!o.pv) {
-          if (o.new_item) {
-            if (!mbar_wait(smem_u32(&bars.q_full[s]), qc[s] & 1, abort, 20)) break;
-            ++qc[s];
-          }
-        } else {
-          if (!mbar_wait(smem_u32(&bars.p_full[s]), pc[s] & 1, abort, 21)) break;
-          ++pc[s];
-          // the first P V of an item overwrites O_i: the previous item's epilogue must be done
-          if (o.j == 0 && !o.first_item && !mbar_wait(smem_u32(&bars.o_free[s]), (oc[s] - 1) & 1, abort, 22))
-            break;
-        }
+      // Consumes the ring in order; each slot's op record says what to issue. No stream
+      // bookkeeping here: between two ops the tensor pipe only has ~1 MMA queued, so the
+      // issuer must get from one op's last MMA to the next op's first in a few dozen cycles.
+      // Descriptors of the tile bases; a k-step or another ring slot only moves the 14-bit
+      // start-address field (16-byte units), which never carries for addresses < 256 KB.
+      const uint64_t dQ = smem_desc_sw128(sb + kOffQ, 16, 1024);          // Q_0 (K-major)
+      const uint64_t dK = smem_desc_sw128(sb + kOffRing, 16, 1024);       // ring slot 0 as K
+      const uint64_t dV = smem_desc_sw128(sb + kOffRing, kHalfB, 1024);   // ring slot 0 as V
+      uint32_t qc0 = 0, qc1 = 0, pc0 = 0, pc1 = 0, oc0 = 0, oc1 = 0;
+      for (uint32_t lc = 0;; ++lc) {
         const uint32_t stg = lc % kStages;
         if (!mbar_wait(smem_u32(&bars.full[stg]), (lc / kStages) & 1, abort, 23)) break;
-        tc_fence_after();
-        const uint32_t tile = sb + kOffRing + stg * kTileB;
-        if (!o.pv) {
-          const uint32_t qt = sb + kOffQ + s * kTileB;
+        const uint32_t op = bars.op[stg];
+        if (op & kOpStop) break;
+        const uint32_t s = (op & kOpSlot1) ? 1u : 0u;
+        const uint32_t s_col = tmem + s * 256, o_col = s_col + 128;
+        const uint64_t ring_off = static_cast<uint64_t>(stg * (kTileB >> 4));
+        if (!(op & kOpPV)) {
+          if (op & kOpNewItem) {
+            uint32_t& qc = s ? qc1 : qc0;
+            if (!mbar_wait(smem_u32(&bars.q_full[s]), qc & 1, abort, 20)) break;
+            ++qc;
+          }
+          tc_fence_after();
+          const uint64_t a0 = dQ + static_cast<uint64_t>(s * (kTileB >> 4));
+          const uint64_t b0 = dK + ring_off;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(s_col, desc_kmajor(qt, kk), desc_kmajor(tile, kk), kIdescQK, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t koff = static_cast<uint64_t>((kk >> 2) * (kHalfB >> 4) + (kk & 3) * 2);
+            mma_ss(s_col, a0 + koff, b0 + koff, kIdescQK, kk > 0 ? 1u : 0u);
+          }
           tc_commit(smem_u32(&bars.s_full[s]));
-          if (o.j == o.n - 1) tc_commit(smem_u32(&bars.q_empty[s]));
+          if (op & kOpLastBlk) tc_commit(smem_u32(&bars.q_empty[s]));
         } else {
+          uint32_t& pc = s ? pc1 : pc0;
+          if (!mbar_wait(smem_u32(&bars.p_full[s]), pc & 1, abort, 21)) break;
+          ++pc;
+          // the first P V of an item overwrites O_i: the previous item's epilogue must be done
+          if ((op & kOpFirstBlk) && !(op & kOpFirstItem)) {
+            const uint32_t oc = s ? oc1 : oc0;
+            if (!mbar_wait(smem_u32(&bars.o_free[s]), (oc - 1) & 1, abort, 22)) break;
+          }
+          tc_fence_after();
+          const uint64_t b0 = dV + ring_off;
+          mma_ts(o_col, s_col, b0, kIdescPV, (op & kOpFirstBlk) ? 0u : 1u);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(o_col, s_col + kk * 8, desc_mnmajor(tile, kk), kIdescPV, (o.j == 0 && kk == 0) ? 0u : 1u);
-          if (o.j == o.n - 1) {
+          for (int kk = 1; kk < 8; ++kk)
+            mma_ts(o_col, s_col + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescPV, 1u);
+          if (op & kOpLastBlk) {
             tc_commit(smem_u32(&bars.o_done[s]));
-            ++oc[s];
+            if (s) ++oc1; else ++oc0;
           }
         }
         tc_commit(smem_u32(&bars.empty[stg]));
-        ++lc;
       }
       // drain: every MMA issued so far completes before the tensor memory is freed
       tc_commit(smem_u32(&bars.drain));
@@ -372,7 +419,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (!warp_wait_abort(smem_u32(&bars.s_full[slot]), sc & 1, abort, 30)) { stop = true; break; }
         ++sc;
         tc_fence_after();
-        float s[128];
+        uint32_t s[128];   // raw fp32 bits of this row of S
         {
           uint32_t r0[32], r1[32], r2[32], r3[32];
           tmem_ld32(s_col, r0);
@@ -383,10 +430,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           reg_fence32(r0); reg_fence32(r1); reg_fence32(r2); reg_fence32(r3);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            s[i] = __uint_as_float(r0[i]);
-            s[32 + i] = __uint_as_float(r1[i]);
-            s[64 + i] = __uint_as_float(r2[i]);
-            s[96 + i] = __uint_as_float(r3[i]);
+            s[i] = r0[i]; s[32 + i] = r1[i]; s[64 + i] = r2[i]; s[96 + i] = r3[i];
           }
         }
         int32_t nv = 128;
@@ -400,15 +444,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (nv < 128) {
 #pragma unroll
           for (int i = 0; i < 128; ++i)
-            if (i >= nv) s[i] = -INFINITY;
+            if (i >= nv) s[i] = 0xFF800000u;   // -inf
         }
+        // row max: eight independent chains of 3-input max
         float mx8[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) mx8[c] = s[c];
+        for (int c = 0; c < 8; ++c) mx8[c] = __uint_as_float(s[c]);
 #pragma unroll
-        for (int i = 8; i < 128; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int i = 8; i < 128; i += 2)
+          mx8[(i >> 1) & 7] = fmax3(mx8[(i >> 1) & 7], __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7]));
         const float m_blk = mx * a.scale_log2;
         if (j == 0) {
           m = m_blk;
@@ -417,30 +463,49 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if (__any_sync(0xffffffffu, need)) {
             // O_i already holds P V of every earlier block (covered by the S commit)
             const float alpha = need ? ex2_approx(m - m_blk) : 1.0f;
+            const uint64_t alpha2 = f2_pack(__float_as_uint(alpha), __float_as_uint(alpha));
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               uint32_t r32[32];
               tmem_ld32_sync(o_col + c * 32, r32);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) r32[i] = __float_as_uint(__uint_as_float(r32[i]) * alpha);
+              for (int i = 0; i < 16; ++i) {
+                const uint64_t v = f2_mul(f2_pack(r32[2 * i], r32[2 * i + 1]), alpha2);
+                float lo, hi;
+                f2_unpack(v, lo, hi);
+                r32[2 * i] = __float_as_uint(lo);
+                r32[2 * i + 1] = __float_as_uint(hi);
+              }
               tmem_st32(o_col + c * 32, r32);
             }
             tmem_wait_st();
             if (need) { l *= alpha; m = m_blk; }
           }
         }
-        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // p = 2^(s * scale_log2 - m): scale-and-subtract and the row sum in fp32 pairs
+        const uint64_t c2 = f2_pack(__float_as_uint(a.scale_log2), __float_as_uint(a.scale_log2));
+        const uint64_t nm2 = f2_pack(__float_as_uint(-m), __float_as_uint(-m));
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        uint32_t pk[64];
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          s[i] = ex2_approx(fmaf(s[i], a.scale_log2, -m));
-          rs8[i & 7] += s[i];
+        for (int i = 0; i < 64; ++i) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), c2, nm2), x0, x1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          acc[i & 3] = f2_add(acc[i & 3], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
+          pk[i] = pack_bf16x2(p0, p1);
         }
-        l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        {
+          float t0, t1, t2, t3, t4, t5, t6, t7;
+          f2_unpack(acc[0], t0, t1); f2_unpack(acc[1], t2, t3);
+          f2_unpack(acc[2], t4, t5); f2_unpack(acc[3], t6, t7);
+          l += ((t0 + t1) + (t2 + t3)) + ((t4 + t5) + (t6 + t7));
+        }
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t p32[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) p32[i] = pack_bf16x2(s[c * 64 + 2 * i], s[c * 64 + 2 * i + 1]);
+          for (int i = 0; i < 32; ++i) p32[i] = pk[c * 32 + i];
           tmem_st32(s_col + c * 32, p32);   // P over the first 64 columns of S
         }
         tmem_wait_st();
