@@ -113,6 +113,28 @@ class Clocks:
                 "samples": len(sm)}
 
 
+def _attn_traffic():
+    """DRAM bytes per attention launch at the 16:9 clip from the committed ncu summary, or
+    None when the kernel source has changed since the counters were taken."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "attn_fwd_clip16x9_h8.md")
+    src = os.path.join(ROOT, "block_sparse_attention_max_b200", "csrc", "k_attn.cuh")
+    if not (os.path.exists(prof) and os.path.exists(src)):
+        return None
+    fields = {}
+    for line in open(prof):
+        if ":" in line and line.split(":")[0].strip() in ("kernel_source_sha256", "dram_bytes_per_launch_clip16x9"):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if fields.get("kernel_source_sha256") != digest:
+        return None
+    try:
+        return int(fields["dram_bytes_per_launch_clip16x9"])
+    except (KeyError, ValueError):
+        return None
+
+
 def _visited_blocks(lists) -> int:
     return int(lists.full_cnt.sum().item() + lists.part_cnt.sum().item())
 
@@ -240,13 +262,7 @@ def run_veda(args):
     }
     for kname in list(hbm):
         hbm[kname.replace("_GBps", "_frac")] = hbm[kname] / peaks["hbm"]
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "attn_fwd_clip16x9_traffic.json")
-    if os.path.exists(prof):
-        try:
-            traffic = json.load(open(prof)).get("dram_bytes_per_launch")
-        except Exception:
-            traffic = None
+    traffic = _attn_traffic() if H == WORKLOAD.H else None
 
     line = {
         "metric": METRIC, "value": world * flop_step / (ms_step * 1e-3) / 1e12, "unit": UNIT,
@@ -319,14 +335,22 @@ def _cores():
 
 
 def cpu_baseline(seconds: float, inp):
-    # whole path on one head, attention on as many query tiles as fit the time budget
-    flop, dt = _oracle_sample(inp, [0], 16)
-    per_row = dt / 16
-    rows = int(max(16, min(WORKLOAD.nT, seconds / max(per_row, 1e-3))))
-    flop, dt = _oracle_sample(inp, [0], rows)
+    # whole path on heads 0.., attention on as many query tiles as fit the time budget
+    # (calibrated: fixed cost of the non-attention steps + cost per attention query tile)
+    _, t8 = _oracle_sample(inp, [0], 8)
+    _, t24 = _oracle_sample(inp, [0], 24)
+    per_row = max((t24 - t8) / 16, 1e-4)
+    fixed = max(t8 - 8 * per_row, 0.0)
+    heads = [0]
+    rows = int((seconds - fixed) / per_row)
+    while rows > WORKLOAD.nT * len(heads) and len(heads) < 4:
+        heads.append(len(heads))
+        rows = int((seconds - fixed * len(heads)) / per_row)
+    rows = max(16, min(WORKLOAD.nT, rows // len(heads)))
+    flop, dt = _oracle_sample(inp, heads, rows)
     return {"value": flop / dt / 1e12, "unit": UNIT, "cores": _cores(), "kind": "oracle",
-            "sample": f"fp64 oracle, all six steps on head 0 of 40, attention on {rows} of 496 "
-                      f"query tiles ({dt:.1f} s); value = visited-block FLOPs / CPU time"}
+            "sample": f"fp64 oracle, all six steps on {len(heads)} of 40 heads, attention on {rows} of 496 "
+                      f"query tiles per head ({dt:.1f} s); value = visited-block FLOPs / CPU time"}
 
 
 def run_reference(args):
@@ -370,8 +394,13 @@ def run_sweep(args):
     peaks = _peaks()
     cfgs = [synth.sweep_density(p, q) for p, q in synth.SWEEP_DENSITIES]
     cfgs += [synth.sweep_length(T) for T in synth.SWEEP_FRAMES]
+    cache = {}
     for w in cfgs:
-        inp = synth.make_inputs(w)
+        key = (w.grid, w.wid)
+        if key not in cache:                 # the density configs share one set of inputs
+            cache.clear()
+            cache[key] = synth.make_inputs(w)
+        inp = cache[key]
         maps = V.build_tile_map(w.grid, w.head_shapes, w.n_tail, inp.tile_order).to(dev)
         q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
         B, N, H, D = q.shape
@@ -393,7 +422,7 @@ def run_sweep(args):
         print(json.dumps({"sweep": w.name, "tokens": N, "nT": maps.nT, "density": f"{w.rho[0][0]}/{w.rho[0][1]}",
                           "visited_blocks": blocks, "attn_ms": ms, "attn_tflops": tf,
                           "frac_bf16_peak_burst": tf / peaks["bf16"]}), flush=True)
-        del bufs, q, k, v, inp
+        del bufs, q, k, v
         torch.cuda.empty_cache()
 
 
