@@ -13,17 +13,18 @@
 //   warpgroup 0 / 1   softmax + epilogue of slot 0 / 1, one query row per thread (the
 //                     32x32b TMEM access shape gives each thread a whole row, so the row
 //                     max and sum need no shuffle)
-//   warp 8            TMA producer: Q of each slot's item, then the K or V tile every MMA
-//                     op needs, in MMA order, through one 5-slot ring (128B swizzle)
-//   warp 9            MMA issuer (one thread, tcgen05.mma kind::f16, M = N = 128):
-//                     S_i = Q_i K^T (shared-memory operands, K-major) and
-//                     O_i += P_i V (P_i read from tensor memory, V MN-major)
+//   warps 8 / 11      TMA producer of slot 0 / 1: the slot's Q tile per item and its K_j,
+//                     V_j tiles into the slot's own buffers (128B swizzle)
+//   warps 9 / 10      MMA issuer of slot 0 / 1 (one thread each, tcgen05.mma kind::f16,
+//                     M = N = 128): S_i = Q_i K^T (shared-memory operands, K-major) and
+//                     O_i += P_i V (P_i read from tensor memory, V MN-major). With one
+//                     issuer per slot, a slot waiting for its softmax never holds up the
+//                     other slot's MMAs.
 // Tensor memory: slot i owns columns [256 i, 256 i + 256): S_i in the first 128, O_i in
 // the next 128; P_i (bf16 pairs) is written over the first 64 columns of S_i once S_i
 // has been read. Per slot the MMA order is QK(0), PV(0), QK(1), PV(1), ...; tcgen05 MMAs
 // from one thread execute in issue order, so QK(j+1) overwrites S_i only after PV(j) has
-// read P_i. The two slots' streams are merged as QK0(0), QK1(0), PV0(0), QK0(1),
-// PV1(0), QK1(1), PV0(1), ...; the producer replays the same stream to fill the ring.
+// read P_i, and QK(j+1) is issued right behind PV(j).
 // The running maximum is only moved (and O rescaled in place) when it grows by more
 // than 2^8; otherwise P uses the stale maximum, exact after the division by the row
 // sum. O_i is stable when S_i(j) is signalled: the commit that signals S_i(j) also
@@ -40,12 +41,14 @@ namespace veda {
 namespace attn {
 
 constexpr int kThreads = 384;
-constexpr int kStages = 5;                 // K/V ring
+constexpr int kKSt = 1;                    // K buffers per slot
+constexpr int kVSt = 1;                    // V buffers per slot
+constexpr int kRec = 8;                    // block records per slot (valid keys of block j)
 constexpr uint32_t kTileB = 32768;         // 128 x 128 bf16
 constexpr uint32_t kHalfB = 16384;         // 128 rows x 64 columns
-constexpr uint32_t kOffQ = 0;              // Q_0, Q_1
-constexpr uint32_t kOffRing = 2 * kTileB;
-constexpr uint32_t kSmemTiles = kOffRing + kStages * kTileB;   // 224 KB
+constexpr uint32_t kSlotB = (1 + kKSt + kVSt) * kTileB;        // Q, K ring, V ring of a slot
+constexpr uint32_t kOffK = kTileB, kOffV = kTileB * (1 + kKSt); // offsets within a slot
+constexpr uint32_t kSmemTiles = 2 * kSlotB;                    // 192 KB
 constexpr uint32_t kSmemBytes = kSmemTiles + 1024;             // + alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);   // A, B K-major
@@ -71,24 +74,34 @@ struct Args {
   float scale_log2;          // softmax scale * log2(e)
 };
 
-// One word per ring slot, written by the producer before it arms the slot: what the MMA
-// issuer has to do with the tile.
+// One word per K buffer, written by the slot's producer before it arms the buffer: what
+// the slot's issuer does with block j (Q K^T now, P V once the softmax is done).
 enum : uint32_t {
-  kOpPV = 1u << 0,        // P V (else Q K^T)
-  kOpNewItem = 1u << 1,   // Q K^T of a slot's new item: wait for its Q tile
-  kOpFirstBlk = 1u << 2,  // block 0 of the item (P V overwrites O)
-  kOpLastBlk = 1u << 3,   // last block of the item
-  kOpSlot1 = 1u << 4,     // slot 1 (else slot 0)
-  kOpFirstItem = 1u << 5, // the slot's first item (no earlier O to wait for)
-  kOpStop = 1u << 6,      // end of the stream (no tile)
+  kOpNewItem = 1u << 0,   // block 0 of an item: wait for its Q tile; P V overwrites O
+  kOpLastBlk = 1u << 1,   // last block of the item
+  kOpFirstItem = 1u << 2, // the slot's first item (no earlier O to wait for)
+  kOpStop = 1u << 3,      // end of the slot's stream (no tile)
+};
+
+struct SlotBars {
+  uint64_t k_full[kKSt], k_empty[kKSt], v_full[kVSt], v_empty[kVSt];
+  uint64_t q_full, q_empty, s_full, p_full, o_done, o_free, drain;
+  uint32_t k_op[kKSt];
+  // block records: the producer writes the number of valid key slots of the slot's block
+  // b into rec_nv[b % kRec] and arrives on rec_full[b % kRec]; it reuses an entry only
+  // after its K buffer came back, i.e. after the softmax finished block b - 2 >= b - kRec
+  uint64_t rec_full[kRec];
+  int32_t rec_nv[kRec];
 };
 
 struct Bars {
-  uint64_t full[kStages], empty[kStages];
-  uint32_t op[kStages];
-  uint64_t q_full[2], q_empty[2];
-  uint64_t s_full[2], p_full[2], o_done[2], o_free[2];
-  uint64_t drain;
+  SlotBars sl[2];
+  // turn taking of the two softmax warpgroups' exponential phases: group i waits on
+  // turn[i], and each of its warps arrives on turn[i ^ 1] when its exponentials are
+  // done; a group that has finished all its items raises finished[i] and arrives once
+  // more, after which the other group runs alone
+  uint64_t turn[2];
+  int32_t finished[2];
   uint32_t tmem_base;
   int32_t abort;
 };
@@ -107,16 +120,6 @@ __device__ __forceinline__ int32_t item_key(const Args& a, int64_t u, int32_t nf
   int32_t idx = j < nf ? a.full_idx[u * a.stride + j] : a.part_idx[u * a.stride + (j - nf)];
   bad = idx < 0 || idx >= a.nT;
   return bad ? 0 : idx;
-}
-
-// K-major operand (Q or K tile): k-step kk covers columns [16kk, 16kk+16).
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int kk) {
-  return smem_desc_sw128(tile + (kk >> 2) * kHalfB + (kk & 3) * 32, 16, 1024);
-}
-// MN-major operand (V tile as B of P V): k-step kk covers keys [16kk, 16kk+16);
-// the two 64-column halves are LBO = 16 KB apart, 8-key groups SBO = 1 KB apart.
-__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int kk) {
-  return smem_desc_sw128(tile + kk * 2048, kHalfB, 1024);
 }
 
 // Whole-warp bounded wait: every lane polls the barrier and the warp leaves together
@@ -144,6 +147,41 @@ __device__ __forceinline__ bool warp_wait_abort(uint32_t bar, uint32_t parity, v
   }
 }
 
+// Hides a value from the optimizer, so that per-k-step descriptors are formed next to
+// their MMA instead of being hoisted out of the loop into 24 live 64-bit registers.
+__device__ __forceinline__ uint64_t opaque(uint64_t x) {
+  uint64_t r;
+  asm volatile("mov.b64 %0, %1;" : "=l"(r) : "l"(x));
+  return r;
+}
+
+// Bounded wait for a softmax group's turn: the turn barrier's phase, or the other group
+// having finished all its work.
+__device__ __forceinline__ bool turn_wait(uint32_t bar, uint32_t parity, volatile int32_t* other_finished,
+                                          volatile int* abort, uint32_t site) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    int give_up = 0, done = 0;
+    if ((threadIdx.x & 31) == 0) {
+      done = *other_finished != 0;
+      if (!done && (it & 31u) == 0) {
+        if (*abort) {
+          give_up = 1;
+        } else if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          flag_status(ST_TIMEOUT | ((site & 0xffu) << ST_WAIT_SITE_SHIFT));
+          *abort = 1;
+          give_up = 1;
+        }
+      }
+    }
+    done = __shfl_sync(0xffffffffu, done, 0);
+    if (done) return true;
+    if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
+  }
+}
+
 template <int N>
 __device__ __forceinline__ void reg_alloc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
@@ -153,89 +191,10 @@ __device__ __forceinline__ void reg_dealloc() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// ------------------------------------------------------------------------------------
-// The merged MMA op stream of the two slots (replayed identically by producer and MMA).
-// Slot i takes the CTA's items m = i, i + 2, i + 4, ... (item u = blockIdx.x + m * grid)
-// that have at least one listed key tile.
-// ------------------------------------------------------------------------------------
-struct Op {
-  int32_t slot, j, n, nf;
-  int64_t u;
-  bool pv;         // P V (else Q K^T)
-  bool new_item;   // Q K^T of a slot's new item (needs its Q tile)
-  bool first_item; // the slot's first item (no earlier O to wait for)
-};
-
-struct Stream {
-  int64_t m[2];     // CTA-local item index of each slot's current item
-  int64_t u[2];
-  int32_t n[2], nf[2], j[2];
-  bool live[2], started[2];
-  int32_t slot_turn;   // slot whose unit comes next
-  int32_t pending_qk;  // after a slot's PV, its QK is emitted next (-1 if none)
-  int32_t init;        // initial QKs still to emit (2 .. 0)
-  int32_t items_done[2];
-
-  __device__ void seek(const Args& a, int s, int64_t from) {
-    live[s] = false;
-    for (int64_t mm = from;; mm += 2) {
-      const int64_t uu = blockIdx.x + mm * static_cast<int64_t>(gridDim.x);
-      if (uu >= a.items) return;
-      bool bad;
-      int32_t f;
-      const int32_t nn = item_blocks(a, uu, f, bad);
-      if (nn > 0) {
-        m[s] = mm; u[s] = uu; n[s] = nn; nf[s] = f; j[s] = 0; live[s] = true;
-        return;
-      }
-    }
-  }
-  __device__ void start(const Args& a) {
-    seek(a, 0, 0);
-    seek(a, 1, 1);
-    items_done[0] = items_done[1] = 0;
-    slot_turn = 0;
-    pending_qk = -1;
-    init = 0;
-  }
-  __device__ Op qk_op(int s, bool fresh) const {
-    Op o;
-    o.slot = s; o.j = j[s]; o.n = n[s]; o.nf = nf[s]; o.u = u[s]; o.pv = false;
-    o.new_item = fresh; o.first_item = items_done[s] == 0;
-    return o;
-  }
-  // Next op; false when both slots are done.
-  __device__ bool next(const Args& a, Op& o) {
-    if (init < 2) {                         // QK0(0), QK1(0)
-      while (init < 2) {
-        const int s = init++;
-        if (live[s]) { o = qk_op(s, true); return true; }
-      }
-    }
-    if (pending_qk >= 0) {                  // the QK that follows a slot's PV
-      const int s = pending_qk;
-      pending_qk = -1;
-      o = qk_op(s, j[s] == 0);
-      return true;
-    }
-    for (int t = 0; t < 2; ++t) {
-      const int s = (slot_turn + t) & 1;
-      if (!live[s]) continue;
-      slot_turn = s ^ 1;
-      o.slot = s; o.j = j[s]; o.n = n[s]; o.nf = nf[s]; o.u = u[s]; o.pv = true;
-      o.new_item = false; o.first_item = items_done[s] == 0;
-      if (j[s] + 1 < n[s]) {
-        ++j[s];
-      } else {
-        ++items_done[s];
-        seek(a, s, m[s] + 2);
-      }
-      if (live[s]) pending_qk = s;
-      return true;
-    }
-    return false;
-  }
-};
+// CTA-local item m of the persistent loop: slot i takes m = i, i + 2, i + 4, ...
+__device__ __forceinline__ int64_t cta_item(int64_t m) {
+  return blockIdx.x + m * static_cast<int64_t>(gridDim.x);
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -248,19 +207,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   volatile int* abort = &bars.abort;
 
   if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(smem_u32(&bars.full[i]), 1);
-      mbar_init(smem_u32(&bars.empty[i]), 1);
-    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bars.q_full[i]), 1);
-      mbar_init(smem_u32(&bars.q_empty[i]), 1);
-      mbar_init(smem_u32(&bars.s_full[i]), 1);
-      mbar_init(smem_u32(&bars.p_full[i]), 4);
-      mbar_init(smem_u32(&bars.o_done[i]), 1);
-      mbar_init(smem_u32(&bars.o_free[i]), 4);
+      SlotBars& b = bars.sl[i];
+      for (int k = 0; k < kKSt; ++k) {
+        mbar_init(smem_u32(&b.k_full[k]), 1);
+        mbar_init(smem_u32(&b.k_empty[k]), 1);
+      }
+      for (int k = 0; k < kVSt; ++k) {
+        mbar_init(smem_u32(&b.v_full[k]), 1);
+        mbar_init(smem_u32(&b.v_empty[k]), 1);
+      }
+      mbar_init(smem_u32(&b.q_full), 1);
+      mbar_init(smem_u32(&b.q_empty), 1);
+      mbar_init(smem_u32(&b.s_full), 1);
+      mbar_init(smem_u32(&b.p_full), 4);
+      mbar_init(smem_u32(&b.o_done), 1);
+      mbar_init(smem_u32(&b.o_free), 4);
+      mbar_init(smem_u32(&b.drain), 1);
+      for (int k = 0; k < kRec; ++k) mbar_init(smem_u32(&b.rec_full[k]), 1);
+      mbar_init(smem_u32(&bars.turn[i]), 4);
+      bars.finished[i] = 0;
     }
-    mbar_init(smem_u32(&bars.drain), 1);
     bars.abort = 0;
     fence_mbar_init();
   }
@@ -268,7 +235,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     tmem_alloc(smem_u32(&bars.tmem_base), kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if ((warp == 8 || warp == 11) && lane == 0) {
     prefetch_tensormap(&tmQ);
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
@@ -280,113 +247,133 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   if (wg == 2) {
     reg_dealloc<kControlRegs>();
-    if (warp == 8 && lane == 0) {
-      // ---------------------------------------------------------- TMA producer
-      Stream st;
-      st.start(a);
-      uint32_t lc = 0;           // ring loads issued
-      uint32_t qc[2] = {0, 0};   // Q loads issued per slot
-      Op o;
-      while (st.next(a, o)) {
-        const int s = o.slot;
-        if (o.new_item) {
-          if (qc[s] > 0 && !mbar_wait(smem_u32(&bars.q_empty[s]), (qc[s] - 1) & 1, abort, 10)) break;
-          const uint32_t qb = smem_u32(&bars.q_full[s]);
-          mbar_arrive_expect_tx(qb, kTileB);
-          tma_load_2d(sb + kOffQ + s * kTileB, &tmQ, qb, 0, static_cast<int32_t>(o.u * 128));
-          tma_load_2d(sb + kOffQ + s * kTileB + kHalfB, &tmQ, qb, 64, static_cast<int32_t>(o.u * 128));
-          ++qc[s];
-        }
-        const uint32_t stg = lc % kStages;
-        if (lc >= kStages && !mbar_wait(smem_u32(&bars.empty[stg]), (lc / kStages - 1) & 1, abort, 11)) break;
+    if ((warp == 8 || warp == 11) && lane == 0) {
+      // ---------------------------------------------------------- TMA producer of a slot
+      const int sl = warp == 8 ? 0 : 1;
+      SlotBars& b = bars.sl[sl];
+      const uint32_t base = sb + sl * kSlotB;
+      uint32_t kc = 0, vc = 0, qc = 0;
+      bool stop = false;
+      for (int64_t mm = sl; !stop; mm += 2) {
+        const int64_t u = cta_item(mm);
+        if (u >= a.items) break;
+        int32_t nf;
         bool bad;
-        const int32_t idx = item_key(a, o.u, o.nf, o.j, bad);
-        if (bad) flag_status(ST_BAD_LIST);
-        const int32_t row = static_cast<int32_t>(((o.u / a.nT) * a.nT + idx) * 128);
-        const uint32_t fb = smem_u32(&bars.full[stg]);
-        const CUtensorMap* map = o.pv ? &tmV : &tmK;
-        bars.op[stg] = (o.pv ? kOpPV : 0u) | (o.new_item ? kOpNewItem : 0u) | (o.j == 0 ? kOpFirstBlk : 0u) |
-                       (o.j == o.n - 1 ? kOpLastBlk : 0u) | (s ? kOpSlot1 : 0u) | (o.first_item ? kOpFirstItem : 0u);
-        mbar_arrive_expect_tx(fb, kTileB);
-        tma_load_2d(sb + kOffRing + stg * kTileB, map, fb, 0, row);
-        tma_load_2d(sb + kOffRing + stg * kTileB + kHalfB, map, fb, 64, row);
-        ++lc;
+        const int32_t n = item_blocks(a, u, nf, bad);
+        if (n == 0) continue;
+        if (qc > 0 && !mbar_wait(smem_u32(&b.q_empty), (qc - 1) & 1, abort, 10)) break;
+        mbar_arrive_expect_tx(smem_u32(&b.q_full), kTileB);
+        tma_load_2d(base, &tmQ, smem_u32(&b.q_full), 0, static_cast<int32_t>(u * 128));
+        tma_load_2d(base + kHalfB, &tmQ, smem_u32(&b.q_full), 64, static_cast<int32_t>(u * 128));
+        const int64_t head_row = (u / a.nT) * a.nT;
+        const int32_t* valid_h = a.valid + ((u / a.nT) % a.H) * a.nT;
+        for (int32_t j = 0; j < n; ++j) {
+          bool b2;
+          const int32_t idx = item_key(a, u, nf, j, b2);
+          if (b2) flag_status(ST_BAD_LIST);   // clamped to tile 0 by item_key
+          const int32_t row = static_cast<int32_t>((head_row + idx) * 128);
+          const uint32_t ks = kc % kKSt;
+          if (kc >= kKSt && !mbar_wait(smem_u32(&b.k_empty[ks]), (kc / kKSt - 1) & 1, abort, 11)) { stop = true; break; }
+          b.k_op[ks] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (qc == 0 ? kOpFirstItem : 0u);
+          const uint32_t kb = smem_u32(&b.k_full[ks]);
+          mbar_arrive_expect_tx(kb, kTileB);
+          tma_load_2d(base + kOffK + ks * kTileB, &tmK, kb, 0, row);
+          tma_load_2d(base + kOffK + ks * kTileB + kHalfB, &tmK, kb, 64, row);
+          // the block's record (entry kc % kRec was last read for block kc - kRec <= kc - 2)
+          int32_t nv = 128;
+          if (j >= nf) {
+            nv = valid_h[idx];
+            if (nv < 1 || nv > 128) {
+              flag_status(ST_BAD_LIST);
+              nv = nv < 1 ? 1 : 128;
+            }
+          }
+          b.rec_nv[kc % kRec] = nv;
+          mbar_arrive(smem_u32(&b.rec_full[kc % kRec]));
+          ++kc;
+          const uint32_t vs = vc % kVSt;
+          if (vc >= kVSt && !mbar_wait(smem_u32(&b.v_empty[vs]), (vc / kVSt - 1) & 1, abort, 12)) { stop = true; break; }
+          const uint32_t vb = smem_u32(&b.v_full[vs]);
+          mbar_arrive_expect_tx(vb, kTileB);
+          tma_load_2d(base + kOffV + vs * kTileB, &tmV, vb, 0, row);
+          tma_load_2d(base + kOffV + vs * kTileB + kHalfB, &tmV, vb, 64, row);
+          ++vc;
+        }
+        ++qc;
       }
       if (!*abort) {
-        // end of stream: one more ring slot carrying only the stop record
-        const uint32_t stg = lc % kStages;
-        if (lc < kStages || mbar_wait(smem_u32(&bars.empty[stg]), (lc / kStages - 1) & 1, abort, 12)) {
-          bars.op[stg] = kOpStop;
-          mbar_arrive(smem_u32(&bars.full[stg]));
+        // end of the slot's stream: one more K buffer carrying only the stop record
+        const uint32_t ks = kc % kKSt;
+        if (kc < kKSt || mbar_wait(smem_u32(&b.k_empty[ks]), (kc / kKSt - 1) & 1, abort, 16)) {
+          b.k_op[ks] = kOpStop;
+          mbar_arrive(smem_u32(&b.k_full[ks]));
         }
       }
       if (*abort) {
         // let the copies this thread issued land before the CTA exits
-        for (uint32_t i = lc > kStages ? lc - kStages : 0; i < lc; ++i)
-          mbar_wait(smem_u32(&bars.full[i % kStages]), (i / kStages) & 1, nullptr, 13);
-        for (int s = 0; s < 2; ++s)
-          if (qc[s] > 0) mbar_wait(smem_u32(&bars.q_full[s]), (qc[s] - 1) & 1, nullptr, 14);
+        for (uint32_t i = kc > kKSt ? kc - kKSt : 0; i < kc; ++i)
+          mbar_wait(smem_u32(&b.k_full[i % kKSt]), (i / kKSt) & 1, nullptr, 13);
+        for (uint32_t i = vc > kVSt ? vc - kVSt : 0; i < vc; ++i)
+          mbar_wait(smem_u32(&b.v_full[i % kVSt]), (i / kVSt) & 1, nullptr, 18);
+        if (qc > 0) mbar_wait(smem_u32(&b.q_full), (qc - 1) & 1, nullptr, 14);
       }
-    } else if (warp == 9 && lane == 0) {
-      // ---------------------------------------------------------- MMA issuer
-      // Consumes the ring in order; each slot's op record says what to issue. No stream
-      // bookkeeping here: between two ops the tensor pipe only has ~1 MMA queued, so the
-      // issuer must get from one op's last MMA to the next op's first in a few dozen cycles.
-      // Descriptors of the tile bases; a k-step or another ring slot only moves the 14-bit
-      // start-address field (16-byte units), which never carries for addresses < 256 KB.
-      const uint64_t dQ = smem_desc_sw128(sb + kOffQ, 16, 1024);          // Q_0 (K-major)
-      const uint64_t dK = smem_desc_sw128(sb + kOffRing, 16, 1024);       // ring slot 0 as K
-      const uint64_t dV = smem_desc_sw128(sb + kOffRing, kHalfB, 1024);   // ring slot 0 as V
-      uint32_t qc0 = 0, qc1 = 0, pc0 = 0, pc1 = 0, oc0 = 0, oc1 = 0;
-      for (uint32_t lc = 0;; ++lc) {
-        const uint32_t stg = lc % kStages;
-        if (!mbar_wait(smem_u32(&bars.full[stg]), (lc / kStages) & 1, abort, 23)) break;
-        const uint32_t op = bars.op[stg];
+    } else if ((warp == 9 || warp == 10) && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer of a slot
+      // Per block j: Q K^T into S_i as soon as K_j is in, then P V once the softmax has
+      // written P_i(j). Descriptors of the tile bases; a k-step or another buffer only moves
+      // the 14-bit start-address field (16-byte units), which never carries below 256 KB.
+      const int sl = warp - 9;
+      SlotBars& b = bars.sl[sl];
+      const uint32_t base = sb + sl * kSlotB;
+      const uint64_t dQ = smem_desc_sw128(base, 16, 1024);
+      const uint64_t dK = smem_desc_sw128(base + kOffK, 16, 1024);
+      const uint64_t dV = smem_desc_sw128(base + kOffV, kHalfB, 1024);
+      const uint32_t s_col = tmem + sl * 256, o_col = s_col + 128;
+      uint32_t qc = 0, pc = 0, oc = 0, vc = 0;
+      for (uint32_t kc = 0;; ++kc) {
+        const uint32_t ks = kc % kKSt;
+        if (!mbar_wait(smem_u32(&b.k_full[ks]), (kc / kKSt) & 1, abort, 23)) break;
+        const uint32_t op = b.k_op[ks];
         if (op & kOpStop) break;
-        const uint32_t s = (op & kOpSlot1) ? 1u : 0u;
-        const uint32_t s_col = tmem + s * 256, o_col = s_col + 128;
-        const uint64_t ring_off = static_cast<uint64_t>(stg * (kTileB >> 4));
-        if (!(op & kOpPV)) {
-          if (op & kOpNewItem) {
-            uint32_t& qc = s ? qc1 : qc0;
-            if (!mbar_wait(smem_u32(&bars.q_full[s]), qc & 1, abort, 20)) break;
-            ++qc;
-          }
-          tc_fence_after();
-          const uint64_t a0 = dQ + static_cast<uint64_t>(s * (kTileB >> 4));
-          const uint64_t b0 = dK + ring_off;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t koff = static_cast<uint64_t>((kk >> 2) * (kHalfB >> 4) + (kk & 3) * 2);
-            mma_ss(s_col, a0 + koff, b0 + koff, kIdescQK, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(smem_u32(&bars.s_full[s]));
-          if (op & kOpLastBlk) tc_commit(smem_u32(&bars.q_empty[s]));
-        } else {
-          uint32_t& pc = s ? pc1 : pc0;
-          if (!mbar_wait(smem_u32(&bars.p_full[s]), pc & 1, abort, 21)) break;
-          ++pc;
-          // the first P V of an item overwrites O_i: the previous item's epilogue must be done
-          if ((op & kOpFirstBlk) && !(op & kOpFirstItem)) {
-            const uint32_t oc = s ? oc1 : oc0;
-            if (!mbar_wait(smem_u32(&bars.o_free[s]), (oc - 1) & 1, abort, 22)) break;
-          }
-          tc_fence_after();
-          const uint64_t b0 = dV + ring_off;
-          mma_ts(o_col, s_col, b0, kIdescPV, (op & kOpFirstBlk) ? 0u : 1u);
-#pragma unroll
-          for (int kk = 1; kk < 8; ++kk)
-            mma_ts(o_col, s_col + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescPV, 1u);
-          if (op & kOpLastBlk) {
-            tc_commit(smem_u32(&bars.o_done[s]));
-            if (s) ++oc1; else ++oc0;
-          }
+        if (op & kOpNewItem) {
+          if (!mbar_wait(smem_u32(&b.q_full), qc & 1, abort, 20)) break;
+          ++qc;
         }
-        tc_commit(smem_u32(&bars.empty[stg]));
+        tc_fence_after();
+        const uint64_t a0 = opaque(dQ);
+        const uint64_t b0 = opaque(dK + static_cast<uint64_t>(ks * (kTileB >> 4)));
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t koff = static_cast<uint64_t>((kk >> 2) * (kHalfB >> 4) + (kk & 3) * 2);
+          mma_ss(s_col, a0 + koff, b0 + koff, kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&b.s_full));
+        if (op & kOpLastBlk) tc_commit(smem_u32(&b.q_empty));
+        tc_commit(smem_u32(&b.k_empty[ks]));
+        // P V of the same block
+        if (!mbar_wait(smem_u32(&b.p_full), pc & 1, abort, 21)) break;
+        ++pc;
+        const uint32_t vs = vc % kVSt;
+        if (!mbar_wait(smem_u32(&b.v_full[vs]), (vc / kVSt) & 1, abort, 24)) break;
+        // the first P V of an item overwrites O_i: the previous item's epilogue must be done
+        if ((op & kOpNewItem) && !(op & kOpFirstItem) && !mbar_wait(smem_u32(&b.o_free), (oc - 1) & 1, abort, 22))
+          break;
+        tc_fence_after();
+        const uint64_t v0 = opaque(dV + static_cast<uint64_t>(vs * (kTileB >> 4)));
+        mma_ts(o_col, s_col, v0, kIdescPV, (op & kOpNewItem) ? 0u : 1u);
+#pragma unroll
+        for (int kk = 1; kk < 8; ++kk)
+          mma_ts(o_col, s_col + kk * 8, v0 + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescPV, 1u);
+        tc_commit(smem_u32(&b.v_empty[vs]));
+        ++vc;
+        if (op & kOpLastBlk) {
+          tc_commit(smem_u32(&b.o_done));
+          ++oc;
+        }
       }
       // drain: every MMA issued so far completes before the tensor memory is freed
-      tc_commit(smem_u32(&bars.drain));
-      mbar_wait(smem_u32(&bars.drain), 0, nullptr, 25);
+      tc_commit(smem_u32(&b.drain));
+      mbar_wait(smem_u32(&b.drain), 0, nullptr, 25);
     }
   } else {
     reg_alloc<kSoftmaxRegs>();
@@ -395,10 +382,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t row = tid & 127;                              // TMEM lane
     const uint32_t lane_off = ((warp & 3) * 32u) << 16;
     const uint32_t s_col = tmem + lane_off + slot * 256, o_col = s_col + 128;
+    SlotBars& b = bars.sl[slot];
     uint32_t sc = 0, ic = 0;      // S tiles consumed, items finished (this slot)
+    uint32_t tc = 0;              // exponential turns taken
     bool stop = false;
+    volatile int32_t* other_finished = &bars.finished[slot ^ 1];
+    if (slot == 1) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars.turn[0]));   // group 0 goes first
+    }
     for (int64_t mm = slot;; mm += 2) {
-      const int64_t u = blockIdx.x + mm * static_cast<int64_t>(gridDim.x);
+      const int64_t u = cta_item(mm);
       if (u >= a.items || stop) break;
       int32_t nf;
       bool bad;
@@ -414,9 +408,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       const int32_t h = static_cast<int32_t>((u / a.nT) % a.H);
       float m = -INFINITY, l = 0.f;
-      bool list_bad = false;
       for (int32_t j = 0; j < n; ++j) {
-        if (!warp_wait_abort(smem_u32(&bars.s_full[slot]), sc & 1, abort, 30)) { stop = true; break; }
+        if (!warp_wait_abort(smem_u32(&b.rec_full[sc % kRec]), (sc / kRec) & 1, abort, 34)) { stop = true; break; }
+        int32_t nv = reinterpret_cast<volatile int32_t*>(b.rec_nv)[sc % kRec];
+        if (!warp_wait_abort(smem_u32(&b.s_full), sc & 1, abort, 30)) { stop = true; break; }
         ++sc;
         tc_fence_after();
         uint32_t s[128];   // raw fp32 bits of this row of S
@@ -432,14 +427,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int i = 0; i < 32; ++i) {
             s[i] = r0[i]; s[32 + i] = r1[i]; s[64 + i] = r2[i]; s[96 + i] = r3[i];
           }
-        }
-        int32_t nv = 128;
-        if (j >= nf) {
-          bool b2;
-          const int32_t idx = item_key(a, u, nf, j, b2);
-          list_bad |= b2;
-          nv = a.valid[static_cast<int64_t>(h) * a.nT + idx];
-          if (nv < 1 || nv > 128) { list_bad = true; nv = nv < 1 ? 1 : 128; }
         }
         if (nv < 128) {
 #pragma unroll
@@ -482,6 +469,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (need) { l *= alpha; m = m_blk; }
           }
         }
+        // this group's turn for the exponentials (the other group works on its load, max
+        // and P store meanwhile)
+        if (!turn_wait(smem_u32(&bars.turn[slot]), tc & 1, other_finished, abort, 35)) { stop = true; break; }
+        ++tc;
         // p = 2^(s * scale_log2 - m): scale-and-subtract and the row sum in fp32 pairs
         const uint64_t c2 = f2_pack(__float_as_uint(a.scale_log2), __float_as_uint(a.scale_log2));
         const uint64_t nm2 = f2_pack(__float_as_uint(-m), __float_as_uint(-m));
@@ -495,6 +486,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           acc[i & 3] = f2_add(acc[i & 3], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
           pk[i] = pack_bf16x2(p0, p1);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars.turn[slot ^ 1]));
         {
           float t0, t1, t2, t3, t4, t5, t6, t7;
           f2_unpack(acc[0], t0, t1); f2_unpack(acc[1], t2, t3);
@@ -511,12 +504,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars.p_full[slot]));
+        if (lane == 0) mbar_arrive(smem_u32(&b.p_full));
       }
       if (stop) break;
-      if (list_bad && row == 0) flag_status(ST_BAD_LIST);
       // epilogue: O / l -> bf16 rows, LSE
-      if (!warp_wait_abort(smem_u32(&bars.o_done[slot]), ic & 1, abort, 33)) break;
+      if (!warp_wait_abort(smem_u32(&b.o_done), ic & 1, abort, 33)) break;
       ++ic;
       tc_fence_after();
       const float inv_l = 1.0f / l;
@@ -535,7 +527,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (a.lse) a.lse[grow] = (m + __log2f(l)) * 0.69314718055994531f;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars.o_free[slot]));
+      if (lane == 0) mbar_arrive(smem_u32(&b.o_free));
+    }
+    // this group is done: the other one no longer waits for turns
+    __syncwarp();
+    if (lane == 0) {
+      reinterpret_cast<volatile int32_t*>(&bars.finished[slot])[0] = 1;
+      __threadfence_block();
+      mbar_arrive(smem_u32(&bars.turn[slot ^ 1]));
     }
   }
 
