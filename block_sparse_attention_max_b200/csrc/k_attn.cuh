@@ -7,28 +7,25 @@
 // function on partial blocks (here: key slots >= n_valid are masked).
 //
 // One persistent CTA per SM walks (batch, head, query tile) items in head-major order
-// (so the CTAs resident at one time share one head's K/V in L2). A CTA works on two
-// query tiles at once ("slots" 0 and 1), so that while one slot's softmax runs the
-// tensor core works for the other:
-//   warpgroup 0 / 1   softmax + epilogue of slot 0 / 1, one query row per thread (the
-//                     32x32b TMEM access shape gives each thread a whole row, so the row
-//                     max and sum need no shuffle)
-//   warps 8 / 11      TMA producer of slot 0 / 1: the slot's Q tile per item and its K_j,
-//                     V_j tiles into the slot's own buffers (128B swizzle)
-//   warps 9 / 10      MMA issuer of slot 0 / 1 (one thread each, tcgen05.mma kind::f16,
-//                     M = N = 128): S_i = Q_i K^T (shared-memory operands, K-major) and
-//                     O_i += P_i V (P_i read from tensor memory, V MN-major). With one
-//                     issuer per slot, a slot waiting for its softmax never holds up the
-//                     other slot's MMAs.
-// Tensor memory: slot i owns columns [256 i, 256 i + 256): S_i in the first 128, O_i in
-// the next 128; P_i (bf16 pairs) is written over the first 64 columns of S_i once S_i
-// has been read. Per slot the MMA order is QK(0), PV(0), QK(1), PV(1), ...; tcgen05 MMAs
-// from one thread execute in issue order, so QK(j+1) overwrites S_i only after PV(j) has
-// read P_i, and QK(j+1) is issued right behind PV(j).
-// The running maximum is only moved (and O rescaled in place) when it grows by more
-// than 2^8; otherwise P uses the stale maximum, exact after the division by the row
-// sum. O_i is stable when S_i(j) is signalled: the commit that signals S_i(j) also
-// covers P_i(j-1) V.
+// (so the CTAs resident at one time share one head's K/V in L2). Per CTA:
+//   warps 0..7   softmax: warp w owns the 16 query rows 32 (w % 4) + 16 (w / 4) + [0, 16) of
+//                the tile (TMEM lanes; a warp may address the 32-lane window of its w % 4).
+//                The 16x256b TMEM shape gives a thread two rows (r, r + 8) and 32 of the 128
+//                scores of each; a row's maximum is completed by two shuffles inside the
+//                thread quad that shares it, the row sum stays per thread until the epilogue.
+//                No warp waits for another warp's data, and all eight run one code path.
+//   warp 8       TMA producer of Q (per item) and K_j (kKSt-deep ring); it also writes a
+//                record per block (valid key slots) for the softmax
+//   warp 11      TMA producer of V_j (kVSt-deep ring), so that a V buffer still in use
+//                never holds back the next K load
+//   warp 9       Q K^T issuer (one thread): S_b = Q K_j^T, b = block parity, once every
+//                softmax warp has taken S(j-2) out of buffer b
+//   warp 10      P V issuer (one thread): O += P_b V_j, P_b read from tensor memory
+// Tensor memory (512 columns): S0 | S1 | O | P0 | P1. With two S buffers, each freed as
+// soon as the softmax holds it in registers, and P in buffers of its own, the tensor core
+// computes S(j+1) and P V(j-1) while the softmax works on block j. The running maximum is
+// only moved (and O rescaled in TMEM after P V(j-1) has landed) when it grows by more
+// than 2^8; otherwise P uses the stale maximum, exact after the division by the row sum.
 //
 // Every wait is bounded (veda_ptx.cuh): when one runs out the CTA raises a shared abort
 // flag, all roles leave their loops, in-flight copies and MMAs are drained with bounded
@@ -41,16 +38,20 @@ namespace veda {
 namespace attn {
 
 constexpr int kThreads = 384;
-constexpr int kKSt = 1;                    // K buffers per slot
-constexpr int kVSt = 1;                    // V buffers per slot
-constexpr int kRec = 8;                    // block records per slot (valid keys of block j)
+constexpr int kQSt = 2;                    // Q buffers (items)
+constexpr int kKSt = 3;                    // K ring (Q K^T issuer)
+constexpr int kVSt = 2;                    // V ring (P V issuer)
+constexpr int kRec = 8;                    // block records (valid key slots of block g)
+static_assert(kRec > kKSt + 2, "a block record is rewritten only after the softmax has read it");
 constexpr uint32_t kTileB = 32768;         // 128 x 128 bf16
 constexpr uint32_t kHalfB = 16384;         // 128 rows x 64 columns
-constexpr uint32_t kSlotB = (1 + kKSt + kVSt) * kTileB;        // Q, K ring, V ring of a slot
-constexpr uint32_t kOffK = kTileB, kOffV = kTileB * (1 + kKSt); // offsets within a slot
-constexpr uint32_t kSmemTiles = 2 * kSlotB;                    // 192 KB
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kQSt * kTileB;
+constexpr uint32_t kOffV = kOffK + kKSt * kTileB;
+constexpr uint32_t kSmemTiles = kOffV + kVSt * kTileB;         // 224 KB
 constexpr uint32_t kSmemBytes = kSmemTiles + 1024;             // + alignment slack
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;         // S_b at 128b, P_b at 384 + 64b
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);   // A, B K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);   // B (V) MN-major
 constexpr float kRescaleLog2 = 8.0f;
@@ -74,34 +75,23 @@ struct Args {
   float scale_log2;          // softmax scale * log2(e)
 };
 
-// One word per K buffer, written by the slot's producer before it arms the buffer: what
-// the slot's issuer does with block j (Q K^T now, P V once the softmax is done).
+// One word per K / V ring slot, written by its producer before it arms the slot.
 enum : uint32_t {
-  kOpNewItem = 1u << 0,   // block 0 of an item: wait for its Q tile; P V overwrites O
+  kOpNewItem = 1u << 0,   // block 0 of an item (Q K^T: wait for its Q tile; P V: O starts at 0)
   kOpLastBlk = 1u << 1,   // last block of the item
-  kOpFirstItem = 1u << 2, // the slot's first item (no earlier O to wait for)
-  kOpStop = 1u << 3,      // end of the slot's stream (no tile)
-};
-
-struct SlotBars {
-  uint64_t k_full[kKSt], k_empty[kKSt], v_full[kVSt], v_empty[kVSt];
-  uint64_t q_full, q_empty, s_full, p_full, o_done, o_free, drain;
-  uint32_t k_op[kKSt];
-  // block records: the producer writes the number of valid key slots of the slot's block
-  // b into rec_nv[b % kRec] and arrives on rec_full[b % kRec]; it reuses an entry only
-  // after its K buffer came back, i.e. after the softmax finished block b - 2 >= b - kRec
-  uint64_t rec_full[kRec];
-  int32_t rec_nv[kRec];
+  kOpFirstItem = 1u << 2, // the CTA's first item (no earlier O to wait for)
+  kOpStop = 1u << 3,      // end of the stream (no tile)
+  kOpQBufShift = 4,       // Q buffer of the item (bits 4..)
 };
 
 struct Bars {
-  SlotBars sl[2];
-  // turn taking of the two softmax warpgroups' exponential phases: group i waits on
-  // turn[i], and each of its warps arrives on turn[i ^ 1] when its exponentials are
-  // done; a group that has finished all its items raises finished[i] and arrives once
-  // more, after which the other group runs alone
-  uint64_t turn[2];
-  int32_t finished[2];
+  uint64_t q_full[kQSt], q_empty[kQSt];
+  uint64_t k_full[kKSt], k_empty[kKSt], v_full[kVSt], v_empty[kVSt];
+  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
+  uint64_t o_free, drain[2];
+  uint64_t rec_full[kRec];
+  uint32_t k_op[kKSt], v_op[kVSt];
+  int32_t rec_nv[kRec];
   uint32_t tmem_base;
   int32_t abort;
 };
@@ -148,38 +138,11 @@ __device__ __forceinline__ bool warp_wait_abort(uint32_t bar, uint32_t parity, v
 }
 
 // Hides a value from the optimizer, so that per-k-step descriptors are formed next to
-// their MMA instead of being hoisted out of the loop into 24 live 64-bit registers.
+// their MMA instead of being hoisted out of the loop into live 64-bit registers.
 __device__ __forceinline__ uint64_t opaque(uint64_t x) {
   uint64_t r;
   asm volatile("mov.b64 %0, %1;" : "=l"(r) : "l"(x));
   return r;
-}
-
-// Bounded wait for a softmax group's turn: the turn barrier's phase, or the other group
-// having finished all its work.
-__device__ __forceinline__ bool turn_wait(uint32_t bar, uint32_t parity, volatile int32_t* other_finished,
-                                          volatile int* abort, uint32_t site) {
-  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-    int give_up = 0, done = 0;
-    if ((threadIdx.x & 31) == 0) {
-      done = *other_finished != 0;
-      if (!done && (it & 31u) == 0) {
-        if (*abort) {
-          give_up = 1;
-        } else if (globaltimer_ns() - t0 > kWaitLimitNs) {
-          flag_status(ST_TIMEOUT | ((site & 0xffu) << ST_WAIT_SITE_SHIFT));
-          *abort = 1;
-          give_up = 1;
-        }
-      }
-    }
-    done = __shfl_sync(0xffffffffu, done, 0);
-    if (done) return true;
-    if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
-  }
 }
 
 template <int N>
@@ -191,9 +154,238 @@ __device__ __forceinline__ void reg_dealloc() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// CTA-local item m of the persistent loop: slot i takes m = i, i + 2, i + 4, ...
+// CTA-local item m of the persistent loop.
 __device__ __forceinline__ int64_t cta_item(int64_t m) {
   return blockIdx.x + m * static_cast<int64_t>(gridDim.x);
+}
+
+// ---------------------------------------------------------------- softmax
+// tcgen05 16-lane shapes. 16x256b: thread t of the warp holds, per 8-column group, the
+// column pair 2 (t % 4) + {0, 1} of rows t / 4 and t / 4 + 8 (relative to the lane base in
+// the address); .xN repeats that for N consecutive 8-column groups. 16x128b: thread t
+// holds column t % 4 of the same two rows per 4-column group.
+__device__ __forceinline__ void tmem_ld_16x256b_x16(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, "
+      "%35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, "
+      "%56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st_16x256b_x4(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_16x128b_x16(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+__device__ __forceinline__ float quad_max(float v) {
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+}
+__device__ __forceinline__ float quad_sum(float v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  return v + __shfl_xor_sync(0xffffffffu, v, 2);
+}
+
+// Softmax and epilogue of one warp's 16 rows for every item of the CTA. Thread (lane)
+// holds tile rows r0 = base + lane / 4 and r1 = r0 + 8 and, of every 8-column group k,
+// the columns 8k + 2c + {0, 1} (c = lane % 4): register 4k + e is row (e < 2 ? r0 : r1),
+// column 8k + 2c + (e & 1).
+__device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t tmem, uint32_t warp,
+                                             uint32_t lane) {
+  volatile int* abort = &bars.abort;
+  const uint32_t base = 32 * (warp & 3) + 16 * (warp >> 2);   // first TMEM lane (tile row)
+  const uint32_t lane_off = base << 16;
+  const uint32_t r0 = base + lane / 4, c = lane & 3;
+  uint32_t g = 0;
+  uint32_t items = 0;
+  for (int64_t mm = 0;; ++mm) {
+    const int64_t u = cta_item(mm);
+    if (u >= a.items) break;
+    int32_t nf;
+    bool bad;
+    const int32_t n = item_blocks(a, u, nf, bad);
+    __nv_bfloat16* orow0 = a.o + (u * 128 + r0) * 128;
+    __nv_bfloat16* orow1 = orow0 + 8 * 128;
+    if (n == 0) {
+      if (bad && lane == 0 && warp == 0) flag_status(ST_BAD_LIST);
+      uint4* z0 = reinterpret_cast<uint4*>(orow0 + c * 32);
+      uint4* z1 = reinterpret_cast<uint4*>(orow1 + c * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { z0[i] = make_uint4(0, 0, 0, 0); z1[i] = make_uint4(0, 0, 0, 0); }
+      if (a.lse && c == 0) { a.lse[u * 128 + r0] = -INFINITY; a.lse[u * 128 + r0 + 8] = -INFINITY; }
+      continue;
+    }
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    bool ok = true;
+    for (int32_t j = 0; j < n; ++j, ++g) {
+      const uint32_t sbuf = g & 1;
+      if (!warp_wait_abort(smem_u32(&bars.rec_full[g % kRec]), (g / kRec) & 1, abort, 36)) { ok = false; break; }
+      const int32_t nv = reinterpret_cast<volatile int32_t*>(bars.rec_nv)[g % kRec];
+      if (!warp_wait_abort(smem_u32(&bars.s_full[sbuf]), (g >> 1) & 1, abort, 30)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t s[64];
+      tmem_ld_16x256b_x16(tmem + lane_off + kColS + sbuf * 128, s);
+      tmem_wait_ld();
+      reg_fence(s);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars.s_free[sbuf]));
+      if (nv < 128) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (static_cast<int32_t>(8 * (i >> 2) + 2 * c + (i & 1)) >= nv) s[i] = 0xFF800000u;   // -inf
+      }
+      // row maxima: rows r0 (registers 4k, 4k+1) and r1 (4k+2, 4k+3), then the quad
+      float a4[4], b4[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        a4[q] = fmaxf(__uint_as_float(s[4 * q]), __uint_as_float(s[4 * q + 1]));
+        b4[q] = fmaxf(__uint_as_float(s[4 * q + 2]), __uint_as_float(s[4 * q + 3]));
+      }
+#pragma unroll
+      for (int k = 4; k < 16; ++k) {
+        a4[k & 3] = fmax3(a4[k & 3], __uint_as_float(s[4 * k]), __uint_as_float(s[4 * k + 1]));
+        b4[k & 3] = fmax3(b4[k & 3], __uint_as_float(s[4 * k + 2]), __uint_as_float(s[4 * k + 3]));
+      }
+      const float mb0 = quad_max(fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3]))) * a.scale_log2;
+      const float mb1 = quad_max(fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3]))) * a.scale_log2;
+      if (j == 0) {
+        m0 = mb0;
+        m1 = mb1;
+      } else {
+        const bool need0 = mb0 > m0 + kRescaleLog2, need1 = mb1 > m1 + kRescaleLog2;
+        if (__any_sync(0xffffffffu, need0 || need1)) {
+          // O must hold P V of every earlier block before it is rescaled
+          const uint32_t gp = g - 1;
+          if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 31)) { ok = false; break; }
+          tc_fence_after();
+          const float al0 = need0 ? ex2_approx(m0 - mb0) : 1.0f;
+          const float al1 = need1 ? ex2_approx(m1 - mb1) : 1.0f;
+          const uint64_t al0x2 = f2_pack(__float_as_uint(al0), __float_as_uint(al0));
+          const uint64_t al1x2 = f2_pack(__float_as_uint(al1), __float_as_uint(al1));
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t o16[16];
+            const uint32_t oa = tmem + lane_off + kColO + ch * 32;
+            tmem_ld_16x256b_x4(oa, o16);
+            tmem_wait_ld();
+            reg_fence(o16);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float x, y;
+              f2_unpack(f2_mul(f2_pack(o16[4 * q], o16[4 * q + 1]), al0x2), x, y);
+              o16[4 * q] = __float_as_uint(x); o16[4 * q + 1] = __float_as_uint(y);
+              f2_unpack(f2_mul(f2_pack(o16[4 * q + 2], o16[4 * q + 3]), al1x2), x, y);
+              o16[4 * q + 2] = __float_as_uint(x); o16[4 * q + 3] = __float_as_uint(y);
+            }
+            tmem_st_16x256b_x4(oa, o16);
+          }
+          tmem_wait_st();
+          if (need0) { l0 *= al0; m0 = mb0; }
+          if (need1) { l1 *= al1; m1 = mb1; }
+        }
+      }
+      // P = 2^(s * scale_log2 - m): P register 2k is row r0, 2k+1 row r1, column 4k + c
+      const uint64_t c2 = f2_pack(__float_as_uint(a.scale_log2), __float_as_uint(a.scale_log2));
+      const uint64_t nm0 = f2_pack(__float_as_uint(-m0), __float_as_uint(-m0));
+      const uint64_t nm1 = f2_pack(__float_as_uint(-m1), __float_as_uint(-m1));
+      uint64_t acc0[2] = {0ull, 0ull}, acc1[2] = {0ull, 0ull};
+      uint32_t pk[32];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        float x0, x1, y0, y1;
+        f2_unpack(f2_fma(f2_pack(s[4 * k], s[4 * k + 1]), c2, nm0), x0, x1);
+        f2_unpack(f2_fma(f2_pack(s[4 * k + 2], s[4 * k + 3]), c2, nm1), y0, y1);
+        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), q0 = ex2_approx(y0), q1 = ex2_approx(y1);
+        acc0[k & 1] = f2_add(acc0[k & 1], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
+        acc1[k & 1] = f2_add(acc1[k & 1], f2_pack(__float_as_uint(q0), __float_as_uint(q1)));
+        pk[2 * k] = pack_bf16x2(p0, p1);
+        pk[2 * k + 1] = pack_bf16x2(q0, q1);
+      }
+      {
+        float t0, t1, t2, t3;
+        f2_unpack(acc0[0], t0, t1); f2_unpack(acc0[1], t2, t3);
+        l0 += (t0 + t1) + (t2 + t3);
+        f2_unpack(acc1[0], t0, t1); f2_unpack(acc1[1], t2, t3);
+        l1 += (t0 + t1) + (t2 + t3);
+      }
+      // P buffer g & 1 is free once P V of block g - 2 has completed
+      if (g >= 2) {
+        const uint32_t gp = g - 2;
+        if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 32)) { ok = false; break; }
+        tc_fence_after();
+      }
+      tmem_st_16x128b_x16(tmem + lane_off + kColP + sbuf * 64, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars.p_full[sbuf]));
+    }
+    if (!ok) break;
+    // epilogue: row sums over the quad, O / l -> bf16, LSE
+    const float lt0 = quad_sum(l0), lt1 = quad_sum(l1);
+    const uint32_t gl = g - 1;
+    if (!warp_wait_abort(smem_u32(&bars.o_done[gl & 1]), (gl >> 1) & 1, abort, 33)) break;
+    tc_fence_after();
+    const float inv0 = 1.0f / lt0, inv1 = 1.0f / lt1;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+      uint32_t o16[16];
+      tmem_ld_16x256b_x4(tmem + lane_off + kColO + ch * 32, o16);
+      tmem_wait_ld();
+      reg_fence(o16);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int col = ch * 32 + 8 * q + 2 * static_cast<int>(c);
+        *reinterpret_cast<uint32_t*>(orow0 + col) =
+            pack_bf16x2(__uint_as_float(o16[4 * q]) * inv0, __uint_as_float(o16[4 * q + 1]) * inv0);
+        *reinterpret_cast<uint32_t*>(orow1 + col) =
+            pack_bf16x2(__uint_as_float(o16[4 * q + 2]) * inv1, __uint_as_float(o16[4 * q + 3]) * inv1);
+      }
+    }
+    if (a.lse && c == 0) {
+      a.lse[u * 128 + r0] = (m0 + __log2f(lt0)) * 0.69314718055994531f;
+      a.lse[u * 128 + r0 + 8] = (m1 + __log2f(lt1)) * 0.69314718055994531f;
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars.o_free));
+    ++items;
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -207,27 +399,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   volatile int* abort = &bars.abort;
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
-      SlotBars& b = bars.sl[i];
-      for (int k = 0; k < kKSt; ++k) {
-        mbar_init(smem_u32(&b.k_full[k]), 1);
-        mbar_init(smem_u32(&b.k_empty[k]), 1);
-      }
-      for (int k = 0; k < kVSt; ++k) {
-        mbar_init(smem_u32(&b.v_full[k]), 1);
-        mbar_init(smem_u32(&b.v_empty[k]), 1);
-      }
-      mbar_init(smem_u32(&b.q_full), 1);
-      mbar_init(smem_u32(&b.q_empty), 1);
-      mbar_init(smem_u32(&b.s_full), 1);
-      mbar_init(smem_u32(&b.p_full), 4);
-      mbar_init(smem_u32(&b.o_done), 1);
-      mbar_init(smem_u32(&b.o_free), 4);
-      mbar_init(smem_u32(&b.drain), 1);
-      for (int k = 0; k < kRec; ++k) mbar_init(smem_u32(&b.rec_full[k]), 1);
-      mbar_init(smem_u32(&bars.turn[i]), 4);
-      bars.finished[i] = 0;
+    for (int i = 0; i < kQSt; ++i) {
+      mbar_init(smem_u32(&bars.q_full[i]), 1);
+      mbar_init(smem_u32(&bars.q_empty[i]), 1);
     }
+    for (int i = 0; i < kKSt; ++i) {
+      mbar_init(smem_u32(&bars.k_full[i]), 1);
+      mbar_init(smem_u32(&bars.k_empty[i]), 1);
+    }
+    for (int i = 0; i < kVSt; ++i) {
+      mbar_init(smem_u32(&bars.v_full[i]), 1);
+      mbar_init(smem_u32(&bars.v_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bars.s_full[i]), 1);
+      mbar_init(smem_u32(&bars.s_free[i]), 8);
+      mbar_init(smem_u32(&bars.p_full[i]), 8);
+      mbar_init(smem_u32(&bars.o_done[i]), 1);
+      mbar_init(smem_u32(&bars.drain[i]), 1);
+    }
+    for (int i = 0; i < kRec; ++i) mbar_init(smem_u32(&bars.rec_full[i]), 1);
+    mbar_init(smem_u32(&bars.o_free), 8);
     bars.abort = 0;
     fence_mbar_init();
   }
@@ -247,24 +439,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   if (wg == 2) {
     reg_dealloc<kControlRegs>();
-    if ((warp == 8 || warp == 11) && lane == 0) {
-      // ---------------------------------------------------------- TMA producer of a slot
-      const int sl = warp == 8 ? 0 : 1;
-      SlotBars& b = bars.sl[sl];
-      const uint32_t base = sb + sl * kSlotB;
-      uint32_t kc = 0, vc = 0, qc = 0;
+    if (warp == 8 && lane == 0) {
+      // ---------------------------------------------------------- Q / K producer
+      uint32_t kc = 0, qc = 0;
       bool stop = false;
-      for (int64_t mm = sl; !stop; mm += 2) {
+      for (int64_t mm = 0; !stop; ++mm) {
         const int64_t u = cta_item(mm);
         if (u >= a.items) break;
         int32_t nf;
         bool bad;
         const int32_t n = item_blocks(a, u, nf, bad);
         if (n == 0) continue;
-        if (qc > 0 && !mbar_wait(smem_u32(&b.q_empty), (qc - 1) & 1, abort, 10)) break;
-        mbar_arrive_expect_tx(smem_u32(&b.q_full), kTileB);
-        tma_load_2d(base, &tmQ, smem_u32(&b.q_full), 0, static_cast<int32_t>(u * 128));
-        tma_load_2d(base + kHalfB, &tmQ, smem_u32(&b.q_full), 64, static_cast<int32_t>(u * 128));
+        const uint32_t qb = qc % kQSt;
+        if (qc >= kQSt && !mbar_wait(smem_u32(&bars.q_empty[qb]), (qc / kQSt - 1) & 1, abort, 10)) break;
+        const uint32_t qbar = smem_u32(&bars.q_full[qb]);
+        mbar_arrive_expect_tx(qbar, kTileB);
+        tma_load_2d(sb + kOffQ + qb * kTileB, &tmQ, qbar, 0, static_cast<int32_t>(u * 128));
+        tma_load_2d(sb + kOffQ + qb * kTileB + kHalfB, &tmQ, qbar, 64, static_cast<int32_t>(u * 128));
         const int64_t head_row = (u / a.nT) * a.nT;
         const int32_t* valid_h = a.valid + ((u / a.nT) % a.H) * a.nT;
         for (int32_t j = 0; j < n; ++j) {
@@ -273,13 +464,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if (b2) flag_status(ST_BAD_LIST);   // clamped to tile 0 by item_key
           const int32_t row = static_cast<int32_t>((head_row + idx) * 128);
           const uint32_t ks = kc % kKSt;
-          if (kc >= kKSt && !mbar_wait(smem_u32(&b.k_empty[ks]), (kc / kKSt - 1) & 1, abort, 11)) { stop = true; break; }
-          b.k_op[ks] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (qc == 0 ? kOpFirstItem : 0u);
-          const uint32_t kb = smem_u32(&b.k_full[ks]);
+          if (kc >= kKSt && !mbar_wait(smem_u32(&bars.k_empty[ks]), (kc / kKSt - 1) & 1, abort, 11)) { stop = true; break; }
+          bars.k_op[ks] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (qb << kOpQBufShift);
+          const uint32_t kb = smem_u32(&bars.k_full[ks]);
           mbar_arrive_expect_tx(kb, kTileB);
-          tma_load_2d(base + kOffK + ks * kTileB, &tmK, kb, 0, row);
-          tma_load_2d(base + kOffK + ks * kTileB + kHalfB, &tmK, kb, 64, row);
-          // the block's record (entry kc % kRec was last read for block kc - kRec <= kc - 2)
+          tma_load_2d(sb + kOffK + ks * kTileB, &tmK, kb, 0, row);
+          tma_load_2d(sb + kOffK + ks * kTileB + kHalfB, &tmK, kb, 64, row);
+          // block record (entry kc % kRec was last read for block kc - kRec, before the
+          // softmax freed S(kc - kRec) and so before K(kc - kRec + kKSt + 2) could load)
           int32_t nv = 128;
           if (j >= nf) {
             nv = valid_h[idx];
@@ -288,254 +480,133 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
               nv = nv < 1 ? 1 : 128;
             }
           }
-          b.rec_nv[kc % kRec] = nv;
-          mbar_arrive(smem_u32(&b.rec_full[kc % kRec]));
+          bars.rec_nv[kc % kRec] = nv;
+          mbar_arrive(smem_u32(&bars.rec_full[kc % kRec]));
           ++kc;
-          const uint32_t vs = vc % kVSt;
-          if (vc >= kVSt && !mbar_wait(smem_u32(&b.v_empty[vs]), (vc / kVSt - 1) & 1, abort, 12)) { stop = true; break; }
-          const uint32_t vb = smem_u32(&b.v_full[vs]);
-          mbar_arrive_expect_tx(vb, kTileB);
-          tma_load_2d(base + kOffV + vs * kTileB, &tmV, vb, 0, row);
-          tma_load_2d(base + kOffV + vs * kTileB + kHalfB, &tmV, vb, 64, row);
-          ++vc;
         }
         ++qc;
       }
       if (!*abort) {
-        // end of the slot's stream: one more K buffer carrying only the stop record
+        // end of stream: one more K slot carrying only the stop record
         const uint32_t ks = kc % kKSt;
-        if (kc < kKSt || mbar_wait(smem_u32(&b.k_empty[ks]), (kc / kKSt - 1) & 1, abort, 16)) {
-          b.k_op[ks] = kOpStop;
-          mbar_arrive(smem_u32(&b.k_full[ks]));
+        if (kc < kKSt || mbar_wait(smem_u32(&bars.k_empty[ks]), (kc / kKSt - 1) & 1, abort, 16)) {
+          bars.k_op[ks] = kOpStop;
+          mbar_arrive(smem_u32(&bars.k_full[ks]));
         }
       }
       if (*abort) {
         // let the copies this thread issued land before the CTA exits
         for (uint32_t i = kc > kKSt ? kc - kKSt : 0; i < kc; ++i)
-          mbar_wait(smem_u32(&b.k_full[i % kKSt]), (i / kKSt) & 1, nullptr, 13);
-        for (uint32_t i = vc > kVSt ? vc - kVSt : 0; i < vc; ++i)
-          mbar_wait(smem_u32(&b.v_full[i % kVSt]), (i / kVSt) & 1, nullptr, 18);
-        if (qc > 0) mbar_wait(smem_u32(&b.q_full), (qc - 1) & 1, nullptr, 14);
+          mbar_wait(smem_u32(&bars.k_full[i % kKSt]), (i / kKSt) & 1, nullptr, 13);
+        for (uint32_t i = qc > kQSt ? qc - kQSt : 0; i < qc; ++i)
+          mbar_wait(smem_u32(&bars.q_full[i % kQSt]), (i / kQSt) & 1, nullptr, 14);
       }
-    } else if ((warp == 9 || warp == 10) && lane == 0) {
-      // ---------------------------------------------------------- MMA issuer of a slot
-      // Per block j: Q K^T into S_i as soon as K_j is in, then P V once the softmax has
-      // written P_i(j). Descriptors of the tile bases; a k-step or another buffer only moves
-      // the 14-bit start-address field (16-byte units), which never carries below 256 KB.
-      const int sl = warp - 9;
-      SlotBars& b = bars.sl[sl];
-      const uint32_t base = sb + sl * kSlotB;
-      const uint64_t dQ = smem_desc_sw128(base, 16, 1024);
-      const uint64_t dK = smem_desc_sw128(base + kOffK, 16, 1024);
-      const uint64_t dV = smem_desc_sw128(base + kOffV, kHalfB, 1024);
-      const uint32_t s_col = tmem + sl * 256, o_col = s_col + 128;
-      uint32_t qc = 0, pc = 0, oc = 0, vc = 0;
-      for (uint32_t kc = 0;; ++kc) {
-        const uint32_t ks = kc % kKSt;
-        if (!mbar_wait(smem_u32(&b.k_full[ks]), (kc / kKSt) & 1, abort, 23)) break;
-        const uint32_t op = b.k_op[ks];
-        if (op & kOpStop) break;
-        if (op & kOpNewItem) {
-          if (!mbar_wait(smem_u32(&b.q_full), qc & 1, abort, 20)) break;
-          ++qc;
+    } else if (warp == 11 && lane == 0) {
+      // ---------------------------------------------------------- V producer
+      uint32_t vc = 0, items = 0;
+      bool stop = false;
+      for (int64_t mm = 0; !stop; ++mm) {
+        const int64_t u = cta_item(mm);
+        if (u >= a.items) break;
+        int32_t nf;
+        bool bad;
+        const int32_t n = item_blocks(a, u, nf, bad);
+        if (n == 0) continue;
+        const int64_t head_row = (u / a.nT) * a.nT;
+        for (int32_t j = 0; j < n; ++j) {
+          bool b2;
+          const int32_t idx = item_key(a, u, nf, j, b2);
+          const int32_t row = static_cast<int32_t>((head_row + idx) * 128);
+          const uint32_t vs = vc % kVSt;
+          if (vc >= kVSt && !mbar_wait(smem_u32(&bars.v_empty[vs]), (vc / kVSt - 1) & 1, abort, 12)) { stop = true; break; }
+          bars.v_op[vs] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (items == 0 ? kOpFirstItem : 0u);
+          const uint32_t vb = smem_u32(&bars.v_full[vs]);
+          mbar_arrive_expect_tx(vb, kTileB);
+          tma_load_2d(sb + kOffV + vs * kTileB, &tmV, vb, 0, row);
+          tma_load_2d(sb + kOffV + vs * kTileB + kHalfB, &tmV, vb, 64, row);
+          ++vc;
         }
+        ++items;
+      }
+      if (!*abort) {
+        const uint32_t vs = vc % kVSt;
+        if (vc < kVSt || mbar_wait(smem_u32(&bars.v_empty[vs]), (vc / kVSt - 1) & 1, abort, 17)) {
+          bars.v_op[vs] = kOpStop;
+          mbar_arrive(smem_u32(&bars.v_full[vs]));
+        }
+      }
+      if (*abort) {
+        for (uint32_t i = vc > kVSt ? vc - kVSt : 0; i < vc; ++i)
+          mbar_wait(smem_u32(&bars.v_full[i % kVSt]), (i / kVSt) & 1, nullptr, 18);
+      }
+    } else if (warp == 9 && lane == 0) {
+      // ---------------------------------------------------------- Q K^T issuer
+      // S buffer b = g & 1 is free once every softmax warp holds S(g - 2) in registers.
+      // Descriptors of the tile bases; a k-step or another ring slot only moves the 14-bit
+      // start-address field (16-byte units), which never carries for addresses < 256 KB.
+      const uint64_t dQ = smem_desc_sw128(sb + kOffQ, 16, 1024);
+      const uint64_t dK = smem_desc_sw128(sb + kOffK, 16, 1024);
+      uint32_t qn[kQSt];
+      for (int i = 0; i < kQSt; ++i) qn[i] = 0;   // Q tiles consumed per buffer
+      for (uint32_t g = 0;; ++g) {
+        const uint32_t ks = g % kKSt;
+        if (!mbar_wait(smem_u32(&bars.k_full[ks]), (g / kKSt) & 1, abort, 23)) break;
+        const uint32_t op = bars.k_op[ks];
+        if (op & kOpStop) break;
+        const uint32_t qb = op >> kOpQBufShift;
+        if (op & kOpNewItem) {
+          if (!mbar_wait(smem_u32(&bars.q_full[qb]), qn[qb] & 1, abort, 20)) break;
+          ++qn[qb];
+        }
+        const uint32_t sbuf = g & 1;
+        if (g >= 2 && !mbar_wait(smem_u32(&bars.s_free[sbuf]), ((g >> 1) - 1) & 1, abort, 26)) break;
         tc_fence_after();
-        const uint64_t a0 = opaque(dQ);
+        const uint64_t a0 = opaque(dQ + static_cast<uint64_t>(qb * (kTileB >> 4)));
         const uint64_t b0 = opaque(dK + static_cast<uint64_t>(ks * (kTileB >> 4)));
+        const uint32_t d = tmem + kColS + sbuf * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t koff = static_cast<uint64_t>((kk >> 2) * (kHalfB >> 4) + (kk & 3) * 2);
-          mma_ss(s_col, a0 + koff, b0 + koff, kIdescQK, kk > 0 ? 1u : 0u);
+          mma_ss(d, a0 + koff, b0 + koff, kIdescQK, kk > 0 ? 1u : 0u);
         }
-        tc_commit(smem_u32(&b.s_full));
-        if (op & kOpLastBlk) tc_commit(smem_u32(&b.q_empty));
-        tc_commit(smem_u32(&b.k_empty[ks]));
-        // P V of the same block
-        if (!mbar_wait(smem_u32(&b.p_full), pc & 1, abort, 21)) break;
-        ++pc;
-        const uint32_t vs = vc % kVSt;
-        if (!mbar_wait(smem_u32(&b.v_full[vs]), (vc / kVSt) & 1, abort, 24)) break;
-        // the first P V of an item overwrites O_i: the previous item's epilogue must be done
-        if ((op & kOpNewItem) && !(op & kOpFirstItem) && !mbar_wait(smem_u32(&b.o_free), (oc - 1) & 1, abort, 22))
+        tc_commit(smem_u32(&bars.s_full[sbuf]));
+        if (op & kOpLastBlk) tc_commit(smem_u32(&bars.q_empty[qb]));
+        tc_commit(smem_u32(&bars.k_empty[ks]));
+      }
+      tc_commit(smem_u32(&bars.drain[0]));
+      mbar_wait(smem_u32(&bars.drain[0]), 0, nullptr, 25);
+    } else if (warp == 10 && lane == 0) {
+      // ---------------------------------------------------------- P V issuer
+      const uint64_t dV = smem_desc_sw128(sb + kOffV, kHalfB, 1024);
+      uint32_t items_done = 0;
+      for (uint32_t g = 0;; ++g) {
+        const uint32_t vs = g % kVSt;
+        if (!mbar_wait(smem_u32(&bars.v_full[vs]), (g / kVSt) & 1, abort, 24)) break;
+        const uint32_t op = bars.v_op[vs];
+        if (op & kOpStop) break;
+        const uint32_t pb = g & 1;
+        if (!mbar_wait(smem_u32(&bars.p_full[pb]), (g >> 1) & 1, abort, 21)) break;
+        // the first P V of an item overwrites O: the previous item's epilogue must be done
+        if ((op & kOpNewItem) && !(op & kOpFirstItem) &&
+            !mbar_wait(smem_u32(&bars.o_free), (items_done - 1) & 1, abort, 22))
           break;
         tc_fence_after();
-        const uint64_t v0 = opaque(dV + static_cast<uint64_t>(vs * (kTileB >> 4)));
-        mma_ts(o_col, s_col, v0, kIdescPV, (op & kOpNewItem) ? 0u : 1u);
+        const uint64_t b0 = opaque(dV + static_cast<uint64_t>(vs * (kTileB >> 4)));
+        const uint32_t pa = tmem + kColP + pb * 64;
+        mma_ts(tmem + kColO, pa, b0, kIdescPV, (op & kOpNewItem) ? 0u : 1u);
 #pragma unroll
         for (int kk = 1; kk < 8; ++kk)
-          mma_ts(o_col, s_col + kk * 8, v0 + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescPV, 1u);
-        tc_commit(smem_u32(&b.v_empty[vs]));
-        ++vc;
-        if (op & kOpLastBlk) {
-          tc_commit(smem_u32(&b.o_done));
-          ++oc;
-        }
+          mma_ts(tmem + kColO, pa + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescPV, 1u);
+        tc_commit(smem_u32(&bars.o_done[pb]));
+        tc_commit(smem_u32(&bars.v_empty[vs]));
+        if (op & kOpLastBlk) ++items_done;
       }
-      // drain: every MMA issued so far completes before the tensor memory is freed
-      tc_commit(smem_u32(&b.drain));
-      mbar_wait(smem_u32(&b.drain), 0, nullptr, 25);
+      tc_commit(smem_u32(&bars.drain[1]));
+      mbar_wait(smem_u32(&bars.drain[1]), 0, nullptr, 27);
     }
   } else {
     reg_alloc<kSoftmaxRegs>();
-    // ------------------------------------------------------------ softmax + epilogue
-    const int slot = static_cast<int>(wg);
-    const uint32_t row = tid & 127;                              // TMEM lane
-    const uint32_t lane_off = ((warp & 3) * 32u) << 16;
-    const uint32_t s_col = tmem + lane_off + slot * 256, o_col = s_col + 128;
-    SlotBars& b = bars.sl[slot];
-    uint32_t sc = 0, ic = 0;      // S tiles consumed, items finished (this slot)
-    uint32_t tc = 0;              // exponential turns taken
-    bool stop = false;
-    volatile int32_t* other_finished = &bars.finished[slot ^ 1];
-    if (slot == 1) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars.turn[0]));   // group 0 goes first
-    }
-    for (int64_t mm = slot;; mm += 2) {
-      const int64_t u = cta_item(mm);
-      if (u >= a.items || stop) break;
-      int32_t nf;
-      bool bad;
-      const int32_t n = item_blocks(a, u, nf, bad);
-      const int64_t grow = u * 128 + row;
-      uint4* orow = reinterpret_cast<uint4*>(a.o + grow * 128);
-      if (n == 0) {
-        if (bad && row == 0) flag_status(ST_BAD_LIST);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) orow[c] = make_uint4(0, 0, 0, 0);
-        if (a.lse) a.lse[grow] = -INFINITY;
-        continue;
-      }
-      const int32_t h = static_cast<int32_t>((u / a.nT) % a.H);
-      float m = -INFINITY, l = 0.f;
-      for (int32_t j = 0; j < n; ++j) {
-        if (!warp_wait_abort(smem_u32(&b.rec_full[sc % kRec]), (sc / kRec) & 1, abort, 34)) { stop = true; break; }
-        int32_t nv = reinterpret_cast<volatile int32_t*>(b.rec_nv)[sc % kRec];
-        if (!warp_wait_abort(smem_u32(&b.s_full), sc & 1, abort, 30)) { stop = true; break; }
-        ++sc;
-        tc_fence_after();
-        uint32_t s[128];   // raw fp32 bits of this row of S
-        {
-          uint32_t r0[32], r1[32], r2[32], r3[32];
-          tmem_ld32(s_col, r0);
-          tmem_ld32(s_col + 32, r1);
-          tmem_ld32(s_col + 64, r2);
-          tmem_ld32(s_col + 96, r3);
-          tmem_wait_ld();
-          reg_fence32(r0); reg_fence32(r1); reg_fence32(r2); reg_fence32(r3);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            s[i] = r0[i]; s[32 + i] = r1[i]; s[64 + i] = r2[i]; s[96 + i] = r3[i];
-          }
-        }
-        if (nv < 128) {
-#pragma unroll
-          for (int i = 0; i < 128; ++i)
-            if (i >= nv) s[i] = 0xFF800000u;   // -inf
-        }
-        // row max: eight independent chains of 3-input max
-        float mx8[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mx8[c] = __uint_as_float(s[c]);
-#pragma unroll
-        for (int i = 8; i < 128; i += 2)
-          mx8[(i >> 1) & 7] = fmax3(mx8[(i >> 1) & 7], __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
-        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                               fmaxf(mx8[6], mx8[7]));
-        const float m_blk = mx * a.scale_log2;
-        if (j == 0) {
-          m = m_blk;
-        } else {
-          const bool need = m_blk > m + kRescaleLog2;
-          if (__any_sync(0xffffffffu, need)) {
-            // O_i already holds P V of every earlier block (covered by the S commit)
-            const float alpha = need ? ex2_approx(m - m_blk) : 1.0f;
-            const uint64_t alpha2 = f2_pack(__float_as_uint(alpha), __float_as_uint(alpha));
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t r32[32];
-              tmem_ld32_sync(o_col + c * 32, r32);
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const uint64_t v = f2_mul(f2_pack(r32[2 * i], r32[2 * i + 1]), alpha2);
-                float lo, hi;
-                f2_unpack(v, lo, hi);
-                r32[2 * i] = __float_as_uint(lo);
-                r32[2 * i + 1] = __float_as_uint(hi);
-              }
-              tmem_st32(o_col + c * 32, r32);
-            }
-            tmem_wait_st();
-            if (need) { l *= alpha; m = m_blk; }
-          }
-        }
-        // this group's turn for the exponentials (the other group works on its load, max
-        // and P store meanwhile)
-        if (!turn_wait(smem_u32(&bars.turn[slot]), tc & 1, other_finished, abort, 35)) { stop = true; break; }
-        ++tc;
-        // p = 2^(s * scale_log2 - m): scale-and-subtract and the row sum in fp32 pairs
-        const uint64_t c2 = f2_pack(__float_as_uint(a.scale_log2), __float_as_uint(a.scale_log2));
-        const uint64_t nm2 = f2_pack(__float_as_uint(-m), __float_as_uint(-m));
-        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-        uint32_t pk[64];
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), c2, nm2), x0, x1);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-          acc[i & 3] = f2_add(acc[i & 3], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bars.turn[slot ^ 1]));
-        {
-          float t0, t1, t2, t3, t4, t5, t6, t7;
-          f2_unpack(acc[0], t0, t1); f2_unpack(acc[1], t2, t3);
-          f2_unpack(acc[2], t4, t5); f2_unpack(acc[3], t6, t7);
-          l += ((t0 + t1) + (t2 + t3)) + ((t4 + t5) + (t6 + t7));
-        }
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t p32[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) p32[i] = pk[c * 32 + i];
-          tmem_st32(s_col + c * 32, p32);   // P over the first 64 columns of S
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&b.p_full));
-      }
-      if (stop) break;
-      // epilogue: O / l -> bf16 rows, LSE
-      if (!warp_wait_abort(smem_u32(&b.o_done), ic & 1, abort, 33)) break;
-      ++ic;
-      tc_fence_after();
-      const float inv_l = 1.0f / l;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r32[32];
-        tmem_ld32_sync(o_col + c * 32, r32);
-        uint32_t packed[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          packed[i] = pack_bf16x2(__uint_as_float(r32[2 * i]) * inv_l, __uint_as_float(r32[2 * i + 1]) * inv_l);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          orow[c * 4 + i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-      }
-      if (a.lse) a.lse[grow] = (m + __log2f(l)) * 0.69314718055994531f;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&b.o_free));
-    }
-    // this group is done: the other one no longer waits for turns
-    __syncwarp();
-    if (lane == 0) {
-      reinterpret_cast<volatile int32_t*>(&bars.finished[slot])[0] = 1;
-      __threadfence_block();
-      mbar_arrive(smem_u32(&bars.turn[slot ^ 1]));
-    }
+    softmax_role(a, bars, tmem, warp, lane);
   }
 
   tc_fence_before();
