@@ -265,77 +265,89 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars.s_free[sbuf]));
       if (nv < 128) {
+        // column 8k + 2c + e is a key slot < nv exactly for k < kv_e = ceil((nv - 2c - e) / 8)
+        const int32_t kv0 = (nv - 2 * static_cast<int32_t>(c) + 7) >> 3;
+        const int32_t kv1 = (nv - 2 * static_cast<int32_t>(c) + 6) >> 3;
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (static_cast<int32_t>(8 * (i >> 2) + 2 * c + (i & 1)) >= nv) s[i] = 0xFF800000u;   // -inf
-      }
-      // row maxima: rows r0 (registers 4k, 4k+1) and r1 (4k+2, 4k+3), then the quad
-      float a4[4], b4[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        a4[q] = fmaxf(__uint_as_float(s[4 * q]), __uint_as_float(s[4 * q + 1]));
-        b4[q] = fmaxf(__uint_as_float(s[4 * q + 2]), __uint_as_float(s[4 * q + 3]));
-      }
-#pragma unroll
-      for (int k = 4; k < 16; ++k) {
-        a4[k & 3] = fmax3(a4[k & 3], __uint_as_float(s[4 * k]), __uint_as_float(s[4 * k + 1]));
-        b4[k & 3] = fmax3(b4[k & 3], __uint_as_float(s[4 * k + 2]), __uint_as_float(s[4 * k + 3]));
-      }
-      const float mb0 = quad_max(fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3]))) * a.scale_log2;
-      const float mb1 = quad_max(fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3]))) * a.scale_log2;
-      if (j == 0) {
-        m0 = mb0;
-        m1 = mb1;
-      } else {
-        const bool need0 = mb0 > m0 + kRescaleLog2, need1 = mb1 > m1 + kRescaleLog2;
-        if (__any_sync(0xffffffffu, need0 || need1)) {
-          // O must hold P V of every earlier block before it is rescaled
-          const uint32_t gp = g - 1;
-          if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 31)) { ok = false; break; }
-          tc_fence_after();
-          const float al0 = need0 ? ex2_approx(m0 - mb0) : 1.0f;
-          const float al1 = need1 ? ex2_approx(m1 - mb1) : 1.0f;
-          const uint64_t al0x2 = f2_pack(__float_as_uint(al0), __float_as_uint(al0));
-          const uint64_t al1x2 = f2_pack(__float_as_uint(al1), __float_as_uint(al1));
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t o16[16];
-            const uint32_t oa = tmem + lane_off + kColO + ch * 32;
-            tmem_ld_16x256b_x4(oa, o16);
-            tmem_wait_ld();
-            reg_fence(o16);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float x, y;
-              f2_unpack(f2_mul(f2_pack(o16[4 * q], o16[4 * q + 1]), al0x2), x, y);
-              o16[4 * q] = __float_as_uint(x); o16[4 * q + 1] = __float_as_uint(y);
-              f2_unpack(f2_mul(f2_pack(o16[4 * q + 2], o16[4 * q + 3]), al1x2), x, y);
-              o16[4 * q + 2] = __float_as_uint(x); o16[4 * q + 3] = __float_as_uint(y);
-            }
-            tmem_st_16x256b_x4(oa, o16);
-          }
-          tmem_wait_st();
-          if (need0) { l0 *= al0; m0 = mb0; }
-          if (need1) { l1 *= al1; m1 = mb1; }
+        for (int k = 0; k < 16; ++k) {
+          if (k >= kv0) { s[4 * k] = 0xFF800000u; s[4 * k + 2] = 0xFF800000u; }   // -inf
+          if (k >= kv1) { s[4 * k + 1] = 0xFF800000u; s[4 * k + 3] = 0xFF800000u; }
         }
       }
-      // P = 2^(s * scale_log2 - m): P register 2k is row r0, 2k+1 row r1, column 4k + c
+      // Exponentials with the current running maximum m, computed together with the block's
+      // row maxima (one basic block, so the scheduler interleaves the MUFU and max chains).
+      // If a row's maximum grew by more than 2^8 (and always for block 0 of an item, whose
+      // reference is not known yet), the reference moves, O is rescaled and the pass is
+      // repeated; otherwise P uses the stale maximum, exact after the division by the row sum.
       const uint64_t c2 = f2_pack(__float_as_uint(a.scale_log2), __float_as_uint(a.scale_log2));
-      const uint64_t nm0 = f2_pack(__float_as_uint(-m0), __float_as_uint(-m0));
-      const uint64_t nm1 = f2_pack(__float_as_uint(-m1), __float_as_uint(-m1));
-      uint64_t acc0[2] = {0ull, 0ull}, acc1[2] = {0ull, 0ull};
+      uint64_t acc0[2], acc1[2];
       uint32_t pk[32];
+#pragma unroll 1
+      for (int pass = 0;; ++pass) {
+        const uint64_t nm0 = f2_pack(__float_as_uint(-m0), __float_as_uint(-m0));
+        const uint64_t nm1 = f2_pack(__float_as_uint(-m1), __float_as_uint(-m1));
+        acc0[0] = acc0[1] = acc1[0] = acc1[1] = 0ull;
+        float a4[4], b4[4];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        float x0, x1, y0, y1;
-        f2_unpack(f2_fma(f2_pack(s[4 * k], s[4 * k + 1]), c2, nm0), x0, x1);
-        f2_unpack(f2_fma(f2_pack(s[4 * k + 2], s[4 * k + 3]), c2, nm1), y0, y1);
-        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), q0 = ex2_approx(y0), q1 = ex2_approx(y1);
-        acc0[k & 1] = f2_add(acc0[k & 1], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
-        acc1[k & 1] = f2_add(acc1[k & 1], f2_pack(__float_as_uint(q0), __float_as_uint(q1)));
-        pk[2 * k] = pack_bf16x2(p0, p1);
-        pk[2 * k + 1] = pack_bf16x2(q0, q1);
+        for (int q = 0; q < 4; ++q) {
+          a4[q] = fmaxf(__uint_as_float(s[4 * q]), __uint_as_float(s[4 * q + 1]));
+          b4[q] = fmaxf(__uint_as_float(s[4 * q + 2]), __uint_as_float(s[4 * q + 3]));
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          if (k >= 4) {
+            a4[k & 3] = fmax3(a4[k & 3], __uint_as_float(s[4 * k]), __uint_as_float(s[4 * k + 1]));
+            b4[k & 3] = fmax3(b4[k & 3], __uint_as_float(s[4 * k + 2]), __uint_as_float(s[4 * k + 3]));
+          }
+          float x0, x1, y0, y1;
+          f2_unpack(f2_fma(f2_pack(s[4 * k], s[4 * k + 1]), c2, nm0), x0, x1);
+          f2_unpack(f2_fma(f2_pack(s[4 * k + 2], s[4 * k + 3]), c2, nm1), y0, y1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), q0 = ex2_approx(y0), q1 = ex2_approx(y1);
+          acc0[k & 1] = f2_add(acc0[k & 1], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
+          acc1[k & 1] = f2_add(acc1[k & 1], f2_pack(__float_as_uint(q0), __float_as_uint(q1)));
+          pk[2 * k] = pack_bf16x2(p0, p1);
+          pk[2 * k + 1] = pack_bf16x2(q0, q1);
+        }
+        const float mb0 = quad_max(fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3]))) * a.scale_log2;
+        const float mb1 = quad_max(fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3]))) * a.scale_log2;
+        const bool need0 = j == 0 || mb0 > m0 + kRescaleLog2;
+        const bool need1 = j == 0 || mb1 > m1 + kRescaleLog2;
+        if (pass == 1 || !__any_sync(0xffffffffu, need0 || need1)) break;
+        if (j == 0) {
+          m0 = mb0;   // block 0: O holds nothing yet
+          m1 = mb1;
+          continue;
+        }
+        // O must hold P V of every earlier block before it is rescaled
+        const uint32_t gp = g - 1;
+        if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 31)) { ok = false; break; }
+        tc_fence_after();
+        const float al0 = need0 ? ex2_approx(m0 - mb0) : 1.0f;
+        const float al1 = need1 ? ex2_approx(m1 - mb1) : 1.0f;
+        const uint64_t al0x2 = f2_pack(__float_as_uint(al0), __float_as_uint(al0));
+        const uint64_t al1x2 = f2_pack(__float_as_uint(al1), __float_as_uint(al1));
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t o16[16];
+          const uint32_t oa = tmem + lane_off + kColO + ch * 32;
+          tmem_ld_16x256b_x4(oa, o16);
+          tmem_wait_ld();
+          reg_fence(o16);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float x, y;
+            f2_unpack(f2_mul(f2_pack(o16[4 * q], o16[4 * q + 1]), al0x2), x, y);
+            o16[4 * q] = __float_as_uint(x); o16[4 * q + 1] = __float_as_uint(y);
+            f2_unpack(f2_mul(f2_pack(o16[4 * q + 2], o16[4 * q + 3]), al1x2), x, y);
+            o16[4 * q + 2] = __float_as_uint(x); o16[4 * q + 3] = __float_as_uint(y);
+          }
+          tmem_st_16x256b_x4(oa, o16);
+        }
+        tmem_wait_st();
+        if (need0) { l0 *= al0; m0 = mb0; }
+        if (need1) { l1 *= al1; m1 = mb1; }
       }
+      if (!ok) break;
       {
         float t0, t1, t2, t3;
         f2_unpack(acc0[0], t0, t1); f2_unpack(acc0[1], t2, t3);
