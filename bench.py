@@ -49,16 +49,36 @@ def _peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
 
 
-def _dist():
+def _dist(backend: str = "nccl"):
+    """One process per GPU, from the torchrun environment (RANK, LOCAL_RANK, WORLD_SIZE,
+    MASTER_ADDR/PORT). NCCL on GPUs; the CPU tests of this path use gloo. Short timeout, so
+    that ranks waiting for a lost peer end with an error."""
     if int(os.environ.get("WORLD_SIZE", "1")) > 1:
         import torch.distributed as dist
         from datetime import timedelta
         local = int(os.environ.get("LOCAL_RANK", "0"))
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timedelta(seconds=60))
         return dist, dist.get_rank(), dist.get_world_size()
     return None, 0, 1
+
+
+def _max_over_ranks(dist, x: float, device) -> float:
+    """The slowest rank's time (every rank gets it; identity without a process group)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _job_tflops(world: int, flop_per_rank_step: float, ms_step: float) -> float:
+    """Whole-job throughput: the work all replicas did over the slowest rank's step time."""
+    return world * flop_per_rank_step / (ms_step * 1e-3) / 1e12
 
 
 class Clocks:
@@ -139,6 +159,42 @@ def _visited_blocks(lists) -> int:
     return int(lists.full_cnt.sum().item() + lists.part_cnt.sum().item())
 
 
+def _valid_token_flop(lists, tile_valid: np.ndarray) -> float:
+    """Attention FLOP over valid query x valid key pairs of the visited blocks (4 D per pair)."""
+    fc, pc = lists.full_cnt.cpu().numpy(), lists.part_cnt.cpu().numpy()
+    fi, pi = lists.full_idx.cpu().numpy(), lists.part_idx.cpu().numpy()
+    B, H, nT = fc.shape
+    total = 0.0
+    for h in range(H):
+        v = tile_valid[h].astype(np.float64)
+        col = np.arange(fi.shape[-1])
+        for b in range(B):
+            fk = np.where(col[None, :] < fc[b, h][:, None], v[np.clip(fi[b, h], 0, nT - 1)], 0.0).sum(1)
+            pk = np.where(col[None, :] < pc[b, h][:, None], v[np.clip(pi[b, h], 0, nT - 1)], 0.0).sum(1)
+            total += float((v * (fk + pk)).sum())
+    return 4.0 * 128 * total
+
+
+def _random_device_lists(rng, lists, tile_valid: np.ndarray, dev):
+    """Fresh uniform random block lists with a forced diagonal and the same per-row budget as
+    `lists` (the 'new pattern per call' timing), split into full / partial tiles."""
+    from block_sparse_attention_max_b200 import veda as V
+    kcnt = (lists.full_cnt + lists.part_cnt).cpu().numpy()
+    B, H, nT = kcnt.shape
+    keys = rng.random((B, H, nT, nT), dtype=np.float32)
+    ar = np.arange(nT)
+    keys[:, :, ar, ar] = -1.0                                   # the diagonal ranks first
+    rank = np.argsort(np.argsort(keys, axis=-1), axis=-1)
+    sel = rank < kcnt[..., None]
+    full = sel & (tile_valid[None, :, None, :] == 128)
+    part = sel & ~full
+    stride = lists.stride
+    fi = np.argsort(~full, axis=-1, kind="stable")[..., :stride].astype(np.int32)   # ascending
+    pi = np.argsort(~part, axis=-1, kind="stable")[..., :stride].astype(np.int32)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+    return V.BlockLists(t(full.sum(-1).astype(np.int32)), t(fi), t(part.sum(-1).astype(np.int32)), t(pi), stride)
+
+
 def run_veda(args):
     from block_sparse_attention_max_b200 import veda as V
     dist, rank, world = _dist()
@@ -212,10 +268,7 @@ def run_veda(args):
     stage_names = ["permute_qkv", "pool_qk", "scores", "select", "attention", "unpermute"]
     stage_ms = {n: statistics.mean(m[i].elapsed_time(m[i + 1]) for m in all_marks)
                 for i, n in enumerate(stage_names)}
-    if dist:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = _max_over_ranks(dist, ms_total, dev)
     ms_step = ms_total / args.steps
 
     # end-to-end through the public API with host buffers (pinned), copies inside the region
@@ -243,17 +296,41 @@ def run_veda(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1) / e_steps
-    if dist:
-        t = torch.tensor([e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
+    e_ms = _max_over_ranks(dist, e0.elapsed_time(e1) / e_steps, dev)
     V.check_device_status()
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, wqh, wkh))
     d2h = oh.numel() * oh.element_size()
 
     attn_ms = stage_ms["attention"]
     attn_tflops = flop_step / (attn_ms * 1e-3) / 1e12
+
+    # secondary attention figures: valid-token and dense-equivalent rates of the same calls,
+    # and the same kernel on fresh uniform random lists (same budgets), one pattern per call
+    tile_valid = np.asarray(hmaps.tile_valid)
+    valid_flop = _valid_token_flop(bufs.lists, tile_valid)
+    rng = np.random.default_rng(7007)
+    patterns = [_random_device_lists(rng, bufs.lists, tile_valid, dev) for _ in range(4)]
+    rnd_blocks = statistics.mean(_visited_blocks(p) for p in patterns)
+    for p in patterns:
+        V.block_sparse_attn_fwd(bufs.q_t, bufs.k_t, bufs.v_t, maps, p, SCALE, bufs.o_t, bufs.lse)
+    rnd_times = []
+    for i in range(max(3, min(args.steps, 12))):
+        a0, a1 = event(), event()
+        a0.record(stream)
+        V.block_sparse_attn_fwd(bufs.q_t, bufs.k_t, bufs.v_t, maps, patterns[i % len(patterns)], SCALE,
+                                bufs.o_t, bufs.lse)
+        a1.record(stream)
+        a1.synchronize()
+        rnd_times.append(a0.elapsed_time(a1))
+    V.check_device_status()
+    rnd_ms = statistics.median(rnd_times)
+    attn_secondary = {
+        "valid_token_tflops": valid_flop / (attn_ms * 1e-3) / 1e12,
+        "dense_equivalent_tflops": 4.0 * D * N * N * H * B / (attn_ms * 1e-3) / 1e12,
+        "random_lists_ms": rnd_ms,
+        "random_lists_tflops": rnd_blocks * FLOP_PER_BLOCK / (rnd_ms * 1e-3) / 1e12,
+        "random_lists_note": "fresh uniform lists (forced diagonal, same per-row budgets), 4 patterns cycled",
+    }
     nbytes = N * H * D * 2
     hbm = {
         "permute_GBps": 3 * 2 * nbytes / (stage_ms["permute_qkv"] * 1e-3) / 1e9,
@@ -265,7 +342,7 @@ def run_veda(args):
     traffic = _attn_traffic() if H == WORKLOAD.H else None
 
     line = {
-        "metric": METRIC, "value": world * flop_step / (ms_step * 1e-3) / 1e12, "unit": UNIT,
+        "metric": METRIC, "value": _job_tflops(world, flop_step, ms_step), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded smoothed-field Q/K, N(0,1) V, random-init projections)",
@@ -274,13 +351,13 @@ def run_veda(args):
                    "parallelism": f"replicas x{world}", "visited_blocks": blocks,
                    "l2": f"inputs larger than L2 ({3 * N * H * D * 2 / 1e9:.2f} GB raster Q/K/V per step)"},
         "attn_ms_per_call": attn_ms, "attn_tflops": attn_tflops,
-        "attn_frac_bf16_peak": attn_tflops / peaks["bf16_sus"],
+        "attn_frac_bf16_peak": attn_tflops / peaks["bf16_sus"], "attn_secondary": attn_secondary,
         "stage_ms": stage_ms, "hbm_stages": hbm,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peaks["bf16_sus"],
                      "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_sus"], "traffic": traffic,
                      "kernel": "attn_fwd_kernel",
                      "peak_note": f"{peaks['source']} sustained dense bf16 (kernel timed inside a long step)"},
-        "e2e": {"value": world * flop_step / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+        "e2e": {"value": _job_tflops(world, flop_step, e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
