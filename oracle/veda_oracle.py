@@ -15,7 +15,7 @@ Sources (web pages, cited by title and section):
   "Key Features", sub-list "Veda sparse attention"; "NEWS" 2026/09/23).
 
 The pages give the steps in prose only; where they leave a step open the reading
-taken here is stated in the function's docstring (readings R1..R13). Everything
+taken here is stated in the function's docstring (readings R1..R19). Everything
 is computed in float64 from the bf16-rounded inputs (exact upcast).
 
 Steps, in the path's order:
@@ -27,6 +27,8 @@ Steps, in the path's order:
 5. ``budgets`` + ``select`` -- Bresenham budgets, forced diagonal, top-k lists
 6. ``attention``     -- softmax attention over the listed key tiles
 7. ``unpermute``     -- scatter back to raster order
+8. ``block_heat`` + ``mask_quality`` -- teacher block heat from dense attention, the
+   attention mass a mask keeps and its recall against the oracle mask
 
 plus ``dense_attention_raster``, an independent dense routine used as a pin.
 Parity status: every function here is pinned by a ``-m "not gpu"`` test
@@ -409,6 +411,84 @@ def dense_attention_raster(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: f
 def predictor_param_count(heads: int, blocks: int, D: int = 128) -> int:
     """Parameters of the per-head residual projections (reading R6): 2 * D * 3D per head per block."""
     return 2 * D * 3 * D * heads * blocks
+
+
+# ---------------------------------------------------------------------------------------
+# 8. block heat and mask quality (the predictor's teacher signal and its check)
+# ---------------------------------------------------------------------------------------
+
+def block_heat(q_tiled: np.ndarray, k_tiled: np.ndarray, n_valid: np.ndarray,
+               nT_per_head: Sequence[int], scale: float,
+               rows: Optional[Sequence[Tuple[int, int, int]]] = None) -> np.ndarray:
+    """Per-block attention mass of dense attention: the predictor's teacher signal.
+
+    [README] Key Features / Veda sparse attention: the predictor learns from "teacher
+    block heat from the dense LSE". Reading R18: heat[b, h, i, j] is the mean, over the
+    valid query slots q of tile i, of the sum over the valid key slots k of tile j of
+    exp(scale q.k - LSE_q), where LSE_q = log sum_k exp(scale q.k) over every valid key
+    of the head (dense attention). A valid row of heat therefore sums to 1 over j. Pad
+    query slots do not count; rows past a head's tile count stay 0.
+    q/k_tiled: [B, H, nT*128, D]; n_valid: [H, nT]. ``rows`` optionally restricts the
+    work to some (b, h, query tile) triples. Returns heat [B, H, nT, nT].
+    """
+    B, H, Npad, D = q_tiled.shape
+    nT = Npad // TILE
+    heat = np.zeros((B, H, nT, nT))
+    todo = rows if rows is not None else [(b, h, i) for b in range(B) for h in range(H)
+                                          for i in range(int(nT_per_head[h]))]
+    keys = {}
+    for (b, h, i) in todo:
+        n = int(nT_per_head[h])
+        if (b, h) not in keys:
+            idx = np.concatenate([np.arange(j * TILE, j * TILE + int(n_valid[h, j])) for j in range(n)])
+            owner = np.concatenate([np.full(int(n_valid[h, j]), j) for j in range(n)])
+            keys[(b, h)] = (k_tiled[b, h][idx], owner)
+        K, owner = keys[(b, h)]
+        nq = int(n_valid[h, i])
+        if nq == 0:
+            continue
+        Q = q_tiled[b, h, i * TILE: i * TILE + nq]
+        s = scale * (Q @ K.T)
+        m = s.max(axis=1, keepdims=True)
+        lse = m + np.log(np.exp(s - m).sum(axis=1, keepdims=True))
+        p = np.exp(s - lse)
+        heat[b, h, i, :n] = np.bincount(owner, weights=p.sum(axis=0) / nq, minlength=n)
+    return heat
+
+
+def mask_quality(heat: np.ndarray, n_valid: np.ndarray, nT_per_head: Sequence[int],
+                 pred: BlockLists, oracle: BlockLists):
+    """Attention mass a block mask keeps, and its block recall against the oracle mask.
+
+    [AGENTS] section 4: the predictor is checked by its recall against the oracle mask;
+    section 6: at a 10% keep ratio "even an oracle mask" keeps only about 0.63 of the
+    attention mass. Reading R19: the oracle mask is the selection step (same budgets,
+    forced diagonal, score order) run on heat as the score. The mass a mask keeps in row
+    (b, h, i) is the sum of heat[b, h, i, j] over its tiles j; the overall mass is the
+    mean over valid query slots (rows weighted by n_valid(i)). Block recall of a row is
+    |pred_i & oracle_i| / |oracle_i|; the overall recall is the mean over rows with a
+    non-empty oracle list.
+    Returns (mass_rows [B, H, nT], recall_rows [B, H, nT], mass, recall).
+    """
+    B, H, nT, _ = heat.shape
+    mass_rows = np.zeros((B, H, nT))
+    recall_rows = np.zeros((B, H, nT))
+    wsum = msum = 0.0
+    rsum, rcount = 0.0, 0
+    for b in range(B):
+        for h in range(H):
+            for i in range(int(nT_per_head[h])):
+                mine = set(np.concatenate([pred.full[b][h][i], pred.partial[b][h][i]]).tolist())
+                ref = set(np.concatenate([oracle.full[b][h][i], oracle.partial[b][h][i]]).tolist())
+                mass_rows[b, h, i] = sum(heat[b, h, i, j] for j in mine)
+                w = float(n_valid[h, i])
+                wsum += w
+                msum += w * mass_rows[b, h, i]
+                if ref:
+                    recall_rows[b, h, i] = len(mine & ref) / len(ref)
+                    rsum += recall_rows[b, h, i]
+                    rcount += 1
+    return mass_rows, recall_rows, (msum / wsum if wsum else 0.0), (rsum / rcount if rcount else 0.0)
 
 
 # ---------------------------------------------------------------------------------------
