@@ -92,6 +92,7 @@ struct Bars {
   uint64_t rec_full[kRec];
   uint32_t k_op[kKSt], v_op[kVSt];
   int32_t rec_nv[kRec];
+  int32_t rec_idx[kRec];
   uint32_t tmem_base;
   int32_t abort;
 };
@@ -400,6 +401,214 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
   }
 }
 
+// ---------------------------------------------------------------- control roles
+// One thread each. The Q / K producer and the Q K^T issuer are shared with the block-heat
+// kernel (k_heat.cuh), which runs the same Q K^T stream without P V.
+
+// TMA producer of Q (per item) and K_j (kKSt-deep ring), plus one record per block (valid
+// key slots and key tile index) for the softmax warps.
+__device__ __forceinline__ void role_qk_producer(const Args& a, Bars& bars, uint32_t sb, const CUtensorMap* tmQ,
+                                                 const CUtensorMap* tmK, volatile int* abort) {
+  uint32_t kc = 0, qc = 0;
+  bool stop = false;
+  for (int64_t mm = 0; !stop; ++mm) {
+    const int64_t u = cta_item(mm);
+    if (u >= a.items) break;
+    int32_t nf;
+    bool bad;
+    const int32_t n = item_blocks(a, u, nf, bad);
+    if (n == 0) continue;
+    const uint32_t qb = qc % kQSt;
+    if (qc >= kQSt && !mbar_wait(smem_u32(&bars.q_empty[qb]), (qc / kQSt - 1) & 1, abort, 10)) break;
+    const uint32_t qbar = smem_u32(&bars.q_full[qb]);
+    mbar_arrive_expect_tx(qbar, kTileB);
+    tma_load_2d(sb + kOffQ + qb * kTileB, tmQ, qbar, 0, static_cast<int32_t>(u * 128));
+    tma_load_2d(sb + kOffQ + qb * kTileB + kHalfB, tmQ, qbar, 64, static_cast<int32_t>(u * 128));
+    const int64_t head_row = (u / a.nT) * a.nT;
+    const int32_t* valid_h = a.valid + ((u / a.nT) % a.H) * a.nT;
+    for (int32_t j = 0; j < n; ++j) {
+      bool b2;
+      const int32_t idx = item_key(a, u, nf, j, b2);
+      if (b2) flag_status(ST_BAD_LIST);   // clamped to tile 0 by item_key
+      const int32_t row = static_cast<int32_t>((head_row + idx) * 128);
+      const uint32_t ks = kc % kKSt;
+      if (kc >= kKSt && !mbar_wait(smem_u32(&bars.k_empty[ks]), (kc / kKSt - 1) & 1, abort, 11)) { stop = true; break; }
+      bars.k_op[ks] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (qb << kOpQBufShift);
+      const uint32_t kb = smem_u32(&bars.k_full[ks]);
+      mbar_arrive_expect_tx(kb, kTileB);
+      tma_load_2d(sb + kOffK + ks * kTileB, tmK, kb, 0, row);
+      tma_load_2d(sb + kOffK + ks * kTileB + kHalfB, tmK, kb, 64, row);
+      // block record (entry kc % kRec was last read for block kc - kRec, before the
+      // softmax freed S(kc - kRec) and so before K(kc - kRec + kKSt + 2) could load)
+      int32_t nv = 128;
+      if (j >= nf) {
+        nv = valid_h[idx];
+        if (nv < 1 || nv > 128) {
+          flag_status(ST_BAD_LIST);
+          nv = nv < 1 ? 1 : 128;
+        }
+      }
+      bars.rec_nv[kc % kRec] = nv;
+      bars.rec_idx[kc % kRec] = idx;
+      mbar_arrive(smem_u32(&bars.rec_full[kc % kRec]));
+      ++kc;
+    }
+    ++qc;
+  }
+  if (!*abort) {
+    // end of stream: one more K slot carrying only the stop record
+    const uint32_t ks = kc % kKSt;
+    if (kc < kKSt || mbar_wait(smem_u32(&bars.k_empty[ks]), (kc / kKSt - 1) & 1, abort, 16)) {
+      bars.k_op[ks] = kOpStop;
+      mbar_arrive(smem_u32(&bars.k_full[ks]));
+    }
+  }
+  if (*abort) {
+    // let the copies this thread issued land before the CTA exits
+    for (uint32_t i = kc > kKSt ? kc - kKSt : 0; i < kc; ++i)
+      mbar_wait(smem_u32(&bars.k_full[i % kKSt]), (i / kKSt) & 1, nullptr, 13);
+    for (uint32_t i = qc > kQSt ? qc - kQSt : 0; i < qc; ++i)
+      mbar_wait(smem_u32(&bars.q_full[i % kQSt]), (i / kQSt) & 1, nullptr, 14);
+  }
+}
+
+// TMA producer of V_j (kVSt-deep ring).
+__device__ __forceinline__ void role_v_producer(const Args& a, Bars& bars, uint32_t sb, const CUtensorMap* tmV,
+                                                volatile int* abort) {
+  uint32_t vc = 0, items = 0;
+  bool stop = false;
+  for (int64_t mm = 0; !stop; ++mm) {
+    const int64_t u = cta_item(mm);
+    if (u >= a.items) break;
+    int32_t nf;
+    bool bad;
+    const int32_t n = item_blocks(a, u, nf, bad);
+    if (n == 0) continue;
+    const int64_t head_row = (u / a.nT) * a.nT;
+    for (int32_t j = 0; j < n; ++j) {
+      bool b2;
+      const int32_t idx = item_key(a, u, nf, j, b2);
+      const int32_t row = static_cast<int32_t>((head_row + idx) * 128);
+      const uint32_t vs = vc % kVSt;
+      if (vc >= kVSt && !mbar_wait(smem_u32(&bars.v_empty[vs]), (vc / kVSt - 1) & 1, abort, 12)) { stop = true; break; }
+      bars.v_op[vs] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (items == 0 ? kOpFirstItem : 0u);
+      const uint32_t vb = smem_u32(&bars.v_full[vs]);
+      mbar_arrive_expect_tx(vb, kTileB);
+      tma_load_2d(sb + kOffV + vs * kTileB, tmV, vb, 0, row);
+      tma_load_2d(sb + kOffV + vs * kTileB + kHalfB, tmV, vb, 64, row);
+      ++vc;
+    }
+    ++items;
+  }
+  if (!*abort) {
+    const uint32_t vs = vc % kVSt;
+    if (vc < kVSt || mbar_wait(smem_u32(&bars.v_empty[vs]), (vc / kVSt - 1) & 1, abort, 17)) {
+      bars.v_op[vs] = kOpStop;
+      mbar_arrive(smem_u32(&bars.v_full[vs]));
+    }
+  }
+  if (*abort) {
+    for (uint32_t i = vc > kVSt ? vc - kVSt : 0; i < vc; ++i)
+      mbar_wait(smem_u32(&bars.v_full[i % kVSt]), (i / kVSt) & 1, nullptr, 18);
+  }
+}
+
+// Q K^T issuer: S_b = Q K_j^T into TMEM buffer b = j & 1 once every softmax warp has taken
+// S(j - 2) out of it.
+__device__ __forceinline__ void role_qk_issuer(Bars& bars, uint32_t sb, uint32_t tmem, volatile int* abort) {
+  // S buffer b = g & 1 is free once every softmax warp holds S(g - 2) in registers.
+  // Descriptors of the tile bases; a k-step or another ring slot only moves the 14-bit
+  // start-address field (16-byte units), which never carries for addresses < 256 KB.
+  const uint64_t dQ = smem_desc_sw128(sb + kOffQ, 16, 1024);
+  const uint64_t dK = smem_desc_sw128(sb + kOffK, 16, 1024);
+  uint32_t qn[kQSt];
+  for (int i = 0; i < kQSt; ++i) qn[i] = 0;   // Q tiles consumed per buffer
+  for (uint32_t g = 0;; ++g) {
+    const uint32_t ks = g % kKSt;
+    if (!mbar_wait(smem_u32(&bars.k_full[ks]), (g / kKSt) & 1, abort, 23)) break;
+    const uint32_t op = bars.k_op[ks];
+    if (op & kOpStop) break;
+    const uint32_t qb = op >> kOpQBufShift;
+    if (op & kOpNewItem) {
+      if (!mbar_wait(smem_u32(&bars.q_full[qb]), qn[qb] & 1, abort, 20)) break;
+      ++qn[qb];
+    }
+    const uint32_t sbuf = g & 1;
+    if (g >= 2 && !mbar_wait(smem_u32(&bars.s_free[sbuf]), ((g >> 1) - 1) & 1, abort, 26)) break;
+    tc_fence_after();
+    const uint64_t a0 = opaque(dQ + static_cast<uint64_t>(qb * (kTileB >> 4)));
+    const uint64_t b0 = opaque(dK + static_cast<uint64_t>(ks * (kTileB >> 4)));
+    const uint32_t d = tmem + kColS + sbuf * 128;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint64_t koff = static_cast<uint64_t>((kk >> 2) * (kHalfB >> 4) + (kk & 3) * 2);
+      mma_ss(d, a0 + koff, b0 + koff, kIdescQK, kk > 0 ? 1u : 0u);
+    }
+    tc_commit(smem_u32(&bars.s_full[sbuf]));
+    if (op & kOpLastBlk) tc_commit(smem_u32(&bars.q_empty[qb]));
+    tc_commit(smem_u32(&bars.k_empty[ks]));
+  }
+  tc_commit(smem_u32(&bars.drain[0]));
+  mbar_wait(smem_u32(&bars.drain[0]), 0, nullptr, 25);
+}
+
+// P V issuer: O += P_b V_j with P_b read from TMEM.
+__device__ __forceinline__ void role_pv_issuer(Bars& bars, uint32_t sb, uint32_t tmem, volatile int* abort) {
+  const uint64_t dV = smem_desc_sw128(sb + kOffV, kHalfB, 1024);
+  uint32_t items_done = 0;
+  for (uint32_t g = 0;; ++g) {
+    const uint32_t vs = g % kVSt;
+    if (!mbar_wait(smem_u32(&bars.v_full[vs]), (g / kVSt) & 1, abort, 24)) break;
+    const uint32_t op = bars.v_op[vs];
+    if (op & kOpStop) break;
+    const uint32_t pb = g & 1;
+    if (!mbar_wait(smem_u32(&bars.p_full[pb]), (g >> 1) & 1, abort, 21)) break;
+    // the first P V of an item overwrites O: the previous item's epilogue must be done
+    if ((op & kOpNewItem) && !(op & kOpFirstItem) &&
+        !mbar_wait(smem_u32(&bars.o_free), (items_done - 1) & 1, abort, 22))
+      break;
+    tc_fence_after();
+    const uint64_t b0 = opaque(dV + static_cast<uint64_t>(vs * (kTileB >> 4)));
+    const uint32_t pa = tmem + kColP + pb * 64;
+    mma_ts(tmem + kColO, pa, b0, kIdescPV, (op & kOpNewItem) ? 0u : 1u);
+#pragma unroll
+    for (int kk = 1; kk < 8; ++kk)
+      mma_ts(tmem + kColO, pa + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescPV, 1u);
+    tc_commit(smem_u32(&bars.o_done[pb]));
+    tc_commit(smem_u32(&bars.v_empty[vs]));
+    if (op & kOpLastBlk) ++items_done;
+  }
+  tc_commit(smem_u32(&bars.drain[1]));
+  mbar_wait(smem_u32(&bars.drain[1]), 0, nullptr, 27);
+}
+
+// Barrier setup of a CTA (thread 0).
+__device__ __forceinline__ void init_bars(Bars& bars) {
+  for (int i = 0; i < kQSt; ++i) {
+    mbar_init(smem_u32(&bars.q_full[i]), 1);
+    mbar_init(smem_u32(&bars.q_empty[i]), 1);
+  }
+  for (int i = 0; i < kKSt; ++i) {
+    mbar_init(smem_u32(&bars.k_full[i]), 1);
+    mbar_init(smem_u32(&bars.k_empty[i]), 1);
+  }
+  for (int i = 0; i < kVSt; ++i) {
+    mbar_init(smem_u32(&bars.v_full[i]), 1);
+    mbar_init(smem_u32(&bars.v_empty[i]), 1);
+  }
+  for (int i = 0; i < 2; ++i) {
+    mbar_init(smem_u32(&bars.s_full[i]), 1);
+    mbar_init(smem_u32(&bars.s_free[i]), 8);
+    mbar_init(smem_u32(&bars.p_full[i]), 8);
+    mbar_init(smem_u32(&bars.o_done[i]), 1);
+    mbar_init(smem_u32(&bars.drain[i]), 1);
+  }
+  for (int i = 0; i < kRec; ++i) mbar_init(smem_u32(&bars.rec_full[i]), 1);
+  mbar_init(smem_u32(&bars.o_free), 8);
+  bars.abort = 0;
+  fence_mbar_init();
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const Args a) {
@@ -410,31 +619,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2;
   volatile int* abort = &bars.abort;
 
-  if (tid == 0) {
-    for (int i = 0; i < kQSt; ++i) {
-      mbar_init(smem_u32(&bars.q_full[i]), 1);
-      mbar_init(smem_u32(&bars.q_empty[i]), 1);
-    }
-    for (int i = 0; i < kKSt; ++i) {
-      mbar_init(smem_u32(&bars.k_full[i]), 1);
-      mbar_init(smem_u32(&bars.k_empty[i]), 1);
-    }
-    for (int i = 0; i < kVSt; ++i) {
-      mbar_init(smem_u32(&bars.v_full[i]), 1);
-      mbar_init(smem_u32(&bars.v_empty[i]), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bars.s_full[i]), 1);
-      mbar_init(smem_u32(&bars.s_free[i]), 8);
-      mbar_init(smem_u32(&bars.p_full[i]), 8);
-      mbar_init(smem_u32(&bars.o_done[i]), 1);
-      mbar_init(smem_u32(&bars.drain[i]), 1);
-    }
-    for (int i = 0; i < kRec; ++i) mbar_init(smem_u32(&bars.rec_full[i]), 1);
-    mbar_init(smem_u32(&bars.o_free), 8);
-    bars.abort = 0;
-    fence_mbar_init();
-  }
+  if (tid == 0) init_bars(bars);
   if (warp == 9) {
     tmem_alloc(smem_u32(&bars.tmem_base), kTmemCols);
     tmem_relinquish();
@@ -451,171 +636,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   if (wg == 2) {
     reg_dealloc<kControlRegs>();
-    if (warp == 8 && lane == 0) {
-      // ---------------------------------------------------------- Q / K producer
-      uint32_t kc = 0, qc = 0;
-      bool stop = false;
-      for (int64_t mm = 0; !stop; ++mm) {
-        const int64_t u = cta_item(mm);
-        if (u >= a.items) break;
-        int32_t nf;
-        bool bad;
-        const int32_t n = item_blocks(a, u, nf, bad);
-        if (n == 0) continue;
-        const uint32_t qb = qc % kQSt;
-        if (qc >= kQSt && !mbar_wait(smem_u32(&bars.q_empty[qb]), (qc / kQSt - 1) & 1, abort, 10)) break;
-        const uint32_t qbar = smem_u32(&bars.q_full[qb]);
-        mbar_arrive_expect_tx(qbar, kTileB);
-        tma_load_2d(sb + kOffQ + qb * kTileB, &tmQ, qbar, 0, static_cast<int32_t>(u * 128));
-        tma_load_2d(sb + kOffQ + qb * kTileB + kHalfB, &tmQ, qbar, 64, static_cast<int32_t>(u * 128));
-        const int64_t head_row = (u / a.nT) * a.nT;
-        const int32_t* valid_h = a.valid + ((u / a.nT) % a.H) * a.nT;
-        for (int32_t j = 0; j < n; ++j) {
-          bool b2;
-          const int32_t idx = item_key(a, u, nf, j, b2);
-          if (b2) flag_status(ST_BAD_LIST);   // clamped to tile 0 by item_key
-          const int32_t row = static_cast<int32_t>((head_row + idx) * 128);
-          const uint32_t ks = kc % kKSt;
-          if (kc >= kKSt && !mbar_wait(smem_u32(&bars.k_empty[ks]), (kc / kKSt - 1) & 1, abort, 11)) { stop = true; break; }
-          bars.k_op[ks] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (qb << kOpQBufShift);
-          const uint32_t kb = smem_u32(&bars.k_full[ks]);
-          mbar_arrive_expect_tx(kb, kTileB);
-          tma_load_2d(sb + kOffK + ks * kTileB, &tmK, kb, 0, row);
-          tma_load_2d(sb + kOffK + ks * kTileB + kHalfB, &tmK, kb, 64, row);
-          // block record (entry kc % kRec was last read for block kc - kRec, before the
-          // softmax freed S(kc - kRec) and so before K(kc - kRec + kKSt + 2) could load)
-          int32_t nv = 128;
-          if (j >= nf) {
-            nv = valid_h[idx];
-            if (nv < 1 || nv > 128) {
-              flag_status(ST_BAD_LIST);
-              nv = nv < 1 ? 1 : 128;
-            }
-          }
-          bars.rec_nv[kc % kRec] = nv;
-          mbar_arrive(smem_u32(&bars.rec_full[kc % kRec]));
-          ++kc;
-        }
-        ++qc;
-      }
-      if (!*abort) {
-        // end of stream: one more K slot carrying only the stop record
-        const uint32_t ks = kc % kKSt;
-        if (kc < kKSt || mbar_wait(smem_u32(&bars.k_empty[ks]), (kc / kKSt - 1) & 1, abort, 16)) {
-          bars.k_op[ks] = kOpStop;
-          mbar_arrive(smem_u32(&bars.k_full[ks]));
-        }
-      }
-      if (*abort) {
-        // let the copies this thread issued land before the CTA exits
-        for (uint32_t i = kc > kKSt ? kc - kKSt : 0; i < kc; ++i)
-          mbar_wait(smem_u32(&bars.k_full[i % kKSt]), (i / kKSt) & 1, nullptr, 13);
-        for (uint32_t i = qc > kQSt ? qc - kQSt : 0; i < qc; ++i)
-          mbar_wait(smem_u32(&bars.q_full[i % kQSt]), (i / kQSt) & 1, nullptr, 14);
-      }
-    } else if (warp == 11 && lane == 0) {
-      // ---------------------------------------------------------- V producer
-      uint32_t vc = 0, items = 0;
-      bool stop = false;
-      for (int64_t mm = 0; !stop; ++mm) {
-        const int64_t u = cta_item(mm);
-        if (u >= a.items) break;
-        int32_t nf;
-        bool bad;
-        const int32_t n = item_blocks(a, u, nf, bad);
-        if (n == 0) continue;
-        const int64_t head_row = (u / a.nT) * a.nT;
-        for (int32_t j = 0; j < n; ++j) {
-          bool b2;
-          const int32_t idx = item_key(a, u, nf, j, b2);
-          const int32_t row = static_cast<int32_t>((head_row + idx) * 128);
-          const uint32_t vs = vc % kVSt;
-          if (vc >= kVSt && !mbar_wait(smem_u32(&bars.v_empty[vs]), (vc / kVSt - 1) & 1, abort, 12)) { stop = true; break; }
-          bars.v_op[vs] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (items == 0 ? kOpFirstItem : 0u);
-          const uint32_t vb = smem_u32(&bars.v_full[vs]);
-          mbar_arrive_expect_tx(vb, kTileB);
-          tma_load_2d(sb + kOffV + vs * kTileB, &tmV, vb, 0, row);
-          tma_load_2d(sb + kOffV + vs * kTileB + kHalfB, &tmV, vb, 64, row);
-          ++vc;
-        }
-        ++items;
-      }
-      if (!*abort) {
-        const uint32_t vs = vc % kVSt;
-        if (vc < kVSt || mbar_wait(smem_u32(&bars.v_empty[vs]), (vc / kVSt - 1) & 1, abort, 17)) {
-          bars.v_op[vs] = kOpStop;
-          mbar_arrive(smem_u32(&bars.v_full[vs]));
-        }
-      }
-      if (*abort) {
-        for (uint32_t i = vc > kVSt ? vc - kVSt : 0; i < vc; ++i)
-          mbar_wait(smem_u32(&bars.v_full[i % kVSt]), (i / kVSt) & 1, nullptr, 18);
-      }
-    } else if (warp == 9 && lane == 0) {
-      // ---------------------------------------------------------- Q K^T issuer
-      // S buffer b = g & 1 is free once every softmax warp holds S(g - 2) in registers.
-      // Descriptors of the tile bases; a k-step or another ring slot only moves the 14-bit
-      // start-address field (16-byte units), which never carries for addresses < 256 KB.
-      const uint64_t dQ = smem_desc_sw128(sb + kOffQ, 16, 1024);
-      const uint64_t dK = smem_desc_sw128(sb + kOffK, 16, 1024);
-      uint32_t qn[kQSt];
-      for (int i = 0; i < kQSt; ++i) qn[i] = 0;   // Q tiles consumed per buffer
-      for (uint32_t g = 0;; ++g) {
-        const uint32_t ks = g % kKSt;
-        if (!mbar_wait(smem_u32(&bars.k_full[ks]), (g / kKSt) & 1, abort, 23)) break;
-        const uint32_t op = bars.k_op[ks];
-        if (op & kOpStop) break;
-        const uint32_t qb = op >> kOpQBufShift;
-        if (op & kOpNewItem) {
-          if (!mbar_wait(smem_u32(&bars.q_full[qb]), qn[qb] & 1, abort, 20)) break;
-          ++qn[qb];
-        }
-        const uint32_t sbuf = g & 1;
-        if (g >= 2 && !mbar_wait(smem_u32(&bars.s_free[sbuf]), ((g >> 1) - 1) & 1, abort, 26)) break;
-        tc_fence_after();
-        const uint64_t a0 = opaque(dQ + static_cast<uint64_t>(qb * (kTileB >> 4)));
-        const uint64_t b0 = opaque(dK + static_cast<uint64_t>(ks * (kTileB >> 4)));
-        const uint32_t d = tmem + kColS + sbuf * 128;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t koff = static_cast<uint64_t>((kk >> 2) * (kHalfB >> 4) + (kk & 3) * 2);
-          mma_ss(d, a0 + koff, b0 + koff, kIdescQK, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(smem_u32(&bars.s_full[sbuf]));
-        if (op & kOpLastBlk) tc_commit(smem_u32(&bars.q_empty[qb]));
-        tc_commit(smem_u32(&bars.k_empty[ks]));
-      }
-      tc_commit(smem_u32(&bars.drain[0]));
-      mbar_wait(smem_u32(&bars.drain[0]), 0, nullptr, 25);
-    } else if (warp == 10 && lane == 0) {
-      // ---------------------------------------------------------- P V issuer
-      const uint64_t dV = smem_desc_sw128(sb + kOffV, kHalfB, 1024);
-      uint32_t items_done = 0;
-      for (uint32_t g = 0;; ++g) {
-        const uint32_t vs = g % kVSt;
-        if (!mbar_wait(smem_u32(&bars.v_full[vs]), (g / kVSt) & 1, abort, 24)) break;
-        const uint32_t op = bars.v_op[vs];
-        if (op & kOpStop) break;
-        const uint32_t pb = g & 1;
-        if (!mbar_wait(smem_u32(&bars.p_full[pb]), (g >> 1) & 1, abort, 21)) break;
-        // the first P V of an item overwrites O: the previous item's epilogue must be done
-        if ((op & kOpNewItem) && !(op & kOpFirstItem) &&
-            !mbar_wait(smem_u32(&bars.o_free), (items_done - 1) & 1, abort, 22))
-          break;
-        tc_fence_after();
-        const uint64_t b0 = opaque(dV + static_cast<uint64_t>(vs * (kTileB >> 4)));
-        const uint32_t pa = tmem + kColP + pb * 64;
-        mma_ts(tmem + kColO, pa, b0, kIdescPV, (op & kOpNewItem) ? 0u : 1u);
-#pragma unroll
-        for (int kk = 1; kk < 8; ++kk)
-          mma_ts(tmem + kColO, pa + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescPV, 1u);
-        tc_commit(smem_u32(&bars.o_done[pb]));
-        tc_commit(smem_u32(&bars.v_empty[vs]));
-        if (op & kOpLastBlk) ++items_done;
-      }
-      tc_commit(smem_u32(&bars.drain[1]));
-      mbar_wait(smem_u32(&bars.drain[1]), 0, nullptr, 27);
-    }
+    if (warp == 8 && lane == 0)
+      role_qk_producer(a, bars, sb, &tmQ, &tmK, abort);
+    else if (warp == 11 && lane == 0)
+      role_v_producer(a, bars, sb, &tmV, abort);
+    else if (warp == 9 && lane == 0)
+      role_qk_issuer(bars, sb, tmem, abort);
+    else if (warp == 10 && lane == 0)
+      role_pv_issuer(bars, sb, tmem, abort);
   } else {
     reg_alloc<kSoftmaxRegs>();
     softmax_role(a, bars, tmem, warp, lane);

@@ -11,6 +11,7 @@
 
 #include "../../include/veda.h"
 #include "k_attn.cuh"
+#include "k_heat.cuh"
 #include "k_gather.cuh"
 #include "k_scores.cuh"
 #include "k_select.cuh"
@@ -76,6 +77,7 @@ veda_status current_device(int& sms) {
   if (!d.attrs_set) {
     struct { const void* f; int bytes; } attrs[] = {
         {reinterpret_cast<const void*>(attn::attn_fwd_kernel), static_cast<int>(attn::kSmemBytes)},
+        {reinterpret_cast<const void*>(heat::heat_kernel), static_cast<int>(attn::kSmemBytes)},
     };
     for (auto& x : attrs) {
       e = cudaFuncSetAttribute(x.f, cudaFuncAttributeMaxDynamicSharedMemorySize, x.bytes);
@@ -83,13 +85,16 @@ veda_status current_device(int& sms) {
     }
     // the attention kernel re-splits its registers between warpgroups (setmaxnreg); the
     // split assumes the launch allocation it was built for, so refuse any other build
-    cudaFuncAttributes fa{};
-    if ((e = cudaFuncGetAttributes(&fa, attn::attn_fwd_kernel)) != cudaSuccess)
-      return cuda_fail(e, "cudaFuncGetAttributes");
-    if (fa.numRegs != attn::kLaunchRegs)
-      return fail(VEDA_ERR_UNSUPPORTED, "attention kernel built with " + std::to_string(fa.numRegs) +
-                                            " registers per thread; its register split needs " +
-                                            std::to_string(attn::kLaunchRegs));
+    const void* split_kernels[] = {reinterpret_cast<const void*>(attn::attn_fwd_kernel),
+                                   reinterpret_cast<const void*>(heat::heat_kernel)};
+    for (const void* f : split_kernels) {
+      cudaFuncAttributes fa{};
+      if ((e = cudaFuncGetAttributes(&fa, f)) != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+      if (fa.numRegs != attn::kLaunchRegs)
+        return fail(VEDA_ERR_UNSUPPORTED, "attention/heat kernel built with " + std::to_string(fa.numRegs) +
+                                              " registers per thread; its register split needs " +
+                                              std::to_string(attn::kLaunchRegs));
+    }
     // persistent grids: as many CTAs as can be resident at once
     if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_copy, permute_kernel, kCopyThreads, 0)) != cudaSuccess ||
         (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_unpermute, unpermute_kernel, kCopyThreads, 0)) != cudaSuccess ||
@@ -375,6 +380,74 @@ veda_status veda_block_sparse_attn_fwd(const void* q, const void* k, const void*
   attn::attn_fwd_kernel<<<grid_for(a.items, sms, 1), attn::kThreads, attn::kSmemBytes,
                           reinterpret_cast<cudaStream_t>(stream)>>>(tq, tk, tv, a);
   return launched("attn_fwd_kernel");
+}
+
+veda_status veda_block_heat(const void* q, const void* k, const int32_t* tile_valid, const int32_t* full_cnt,
+                            const int32_t* full_idx, const int32_t* part_cnt, const int32_t* part_idx,
+                            int32_t list_stride, const float* lse, float softmax_scale, float* heat, int32_t B,
+                            int32_t H, int32_t nT, int32_t D, veda_stream_t stream) {
+  if (!q || !k || !tile_valid || !full_cnt || !full_idx || !part_cnt || !part_idx || !lse || !heat || B <= 0 ||
+      H <= 0 || nT <= 0 || list_stride <= 0)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_heat: bad pointer or size");
+  if (D != 128) return fail(VEDA_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_heat: softmax_scale must be positive and finite");
+  if (!aligned(q, 16) || !aligned(k, 16))
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_heat: Q/K must be 16-byte aligned");
+  const int64_t rows = static_cast<int64_t>(B) * H * nT * 128;
+  if (rows > INT32_MAX) return fail(VEDA_ERR_INVALID_ARG, "veda_block_heat: too many rows");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  if ((st = get_encoder()) != VEDA_OK) return st;
+  CUtensorMap tq, tk;
+  if ((st = encode_rows(tq, q, rows)) != VEDA_OK) return st;
+  if ((st = encode_rows(tk, k, rows)) != VEDA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t heat_bytes = static_cast<size_t>(B) * H * nT * nT * sizeof(float);
+  cudaError_t e = cudaMemsetAsync(heat, 0, heat_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(heat)");
+  heat::HeatArgs p{};
+  p.a.valid = tile_valid; p.a.full_cnt = full_cnt; p.a.full_idx = full_idx; p.a.part_cnt = part_cnt;
+  p.a.part_idx = part_idx; p.a.stride = list_stride; p.a.H = H; p.a.nT = nT;
+  p.a.items = static_cast<int64_t>(B) * H * nT;
+  p.lse = lse;
+  p.heat = heat;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  heat::heat_kernel<<<grid_for(p.a.items, sms, 1), attn::kThreads, attn::kSmemBytes, s>>>(tq, tk, p);
+  return launched("heat_kernel");
+}
+
+veda_status veda_mask_quality(const float* heat, const int32_t* tile_valid, const int32_t* nT_per_head,
+                              const int32_t* pred_full_cnt, const int32_t* pred_full_idx,
+                              const int32_t* pred_part_cnt, const int32_t* pred_part_idx, int32_t pred_stride,
+                              const int32_t* orc_full_cnt, const int32_t* orc_full_idx,
+                              const int32_t* orc_part_cnt, const int32_t* orc_part_idx, int32_t orc_stride,
+                              float* mass_rows, float* recall_rows, float* totals, int32_t B, int32_t H,
+                              int32_t nT, veda_stream_t stream) {
+  if (!heat || !tile_valid || !nT_per_head || !pred_full_cnt || !pred_full_idx || !pred_part_cnt ||
+      !pred_part_idx || !orc_full_cnt || !orc_full_idx || !orc_part_cnt || !orc_part_idx || !mass_rows ||
+      !recall_rows || !totals || B <= 0 || H <= 0 || nT <= 0 || pred_stride <= 0 || orc_stride <= 0)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_mask_quality: bad pointer or size");
+  if (nT > heat::kQualMaxTiles) return fail(VEDA_ERR_INVALID_ARG, "veda_mask_quality: nT exceeds VEDA_MAX_TILES");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(totals, 0, 4 * sizeof(float), s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(totals)");
+  heat::QualityArgs qa{};
+  qa.heat = heat; qa.valid = tile_valid; qa.nT_per_head = nT_per_head;
+  qa.pfc = pred_full_cnt; qa.pfi = pred_full_idx; qa.ppc = pred_part_cnt; qa.ppi = pred_part_idx;
+  qa.ofc = orc_full_cnt; qa.ofi = orc_full_idx; qa.opc = orc_part_cnt; qa.opi = orc_part_idx;
+  qa.pstride = pred_stride; qa.ostride = orc_stride;
+  qa.mass_rows = mass_rows; qa.recall_rows = recall_rows; qa.totals = totals;
+  qa.H = H; qa.nT = nT;
+  qa.rows = static_cast<int64_t>(B) * H * nT;
+  const int64_t blocks = (qa.rows + heat::kQualWarps - 1) / heat::kQualWarps;
+  if (blocks > INT32_MAX) return fail(VEDA_ERR_INVALID_ARG, "veda_mask_quality: too many rows");
+  heat::mask_quality_kernel<<<static_cast<unsigned>(blocks), 32 * heat::kQualWarps, 0, s>>>(qa);
+  return launched("mask_quality_kernel");
 }
 
 // Self-test of the bounded waits: one thread waits on an mbarrier that nothing arrives

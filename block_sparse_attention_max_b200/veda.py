@@ -27,8 +27,8 @@ EXPORTED = (
     "veda_build_tile_map", "veda_permute_tiles", "veda_tile_pool",
     "veda_block_scores_workspace_bytes", "veda_block_scores", "veda_block_scores_noalloc",
     "veda_select_blocks",
-    "veda_block_sparse_attn_fwd", "veda_unpermute", "veda_check_device_status",
-    "veda_selftest_wait_timeout",
+    "veda_block_sparse_attn_fwd", "veda_unpermute", "veda_block_heat", "veda_mask_quality",
+    "veda_check_device_status", "veda_selftest_wait_timeout",
 )
 
 
@@ -70,6 +70,9 @@ _SIG = {
     "veda_block_sparse_attn_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _F, _P, _P, _I, _I,
                                         _I, _I, _P]),
     "veda_unpermute": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "veda_block_heat": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _F, _P, _I, _I, _I, _I, _P]),
+    "veda_mask_quality": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _I, _P, _P, _P,
+                               _I, _I, _I, _P]),
     "veda_check_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "veda_selftest_wait_timeout": (_I, [ctypes.c_uint32, _P]),
 }
@@ -305,6 +308,61 @@ def block_sparse_attn_fwd(q_t: torch.Tensor, k_t: torch.Tensor, v_t: torch.Tenso
         _ptr(lists.full_idx), _ptr(lists.part_cnt), _ptr(lists.part_idx), lists.stride,
         float(scale), _ptr(out), _ptr(lse), B, H, nT, D, _stream(stream)))
     return out, lse
+
+
+def block_heat(q_t: torch.Tensor, k_t: torch.Tensor, maps: DeviceMaps, lists: BlockLists,
+               lse: torch.Tensor, scale: float, out: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """veda_block_heat: per-block attention mass against the given (dense) LSE."""
+    for t, n in ((q_t, "q"), (k_t, "k")):
+        _need(t, torch.bfloat16, n)
+    _need(lse, torch.float32, "lse")
+    B, H, Npad, D = q_t.shape
+    nT = Npad // 128
+    if out is None:
+        out = torch.empty((B, H, nT, nT), dtype=torch.float32, device=q_t.device)
+    _check("veda_block_heat", lib().veda_block_heat(
+        _ptr(q_t), _ptr(k_t), _ptr(maps.tile_valid), _ptr(lists.full_cnt), _ptr(lists.full_idx),
+        _ptr(lists.part_cnt), _ptr(lists.part_idx), lists.stride, _ptr(lse), float(scale),
+        _ptr(out), B, H, nT, D, _stream(stream)))
+    return out
+
+
+@dataclasses.dataclass
+class MaskQuality:
+    mass_rows: torch.Tensor     # [B, H, nT] heat kept per query tile
+    recall_rows: torch.Tensor   # [B, H, nT] |pred & oracle| / |oracle|
+    totals: torch.Tensor        # [4] see veda_mask_quality
+
+    @property
+    def mass(self) -> float:
+        """Attention mass the mask keeps, over valid query slots."""
+        t = self.totals.tolist()
+        return t[0] / t[1] if t[1] else 0.0
+
+    @property
+    def recall(self) -> float:
+        """Mean block recall against the oracle mask."""
+        t = self.totals.tolist()
+        return t[2] / t[3] if t[3] else 0.0
+
+
+def mask_quality(heat: torch.Tensor, maps: DeviceMaps, pred: BlockLists, oracle: BlockLists,
+                 stream=None) -> MaskQuality:
+    """veda_mask_quality: kept attention mass of `pred` and its recall against `oracle`."""
+    _need(heat, torch.float32, "heat")
+    B, H, nT, _ = heat.shape
+    dev = heat.device
+    q = MaskQuality(torch.empty((B, H, nT), dtype=torch.float32, device=dev),
+                    torch.empty((B, H, nT), dtype=torch.float32, device=dev),
+                    torch.empty(4, dtype=torch.float32, device=dev))
+    _check("veda_mask_quality", lib().veda_mask_quality(
+        _ptr(heat), _ptr(maps.tile_valid), _ptr(maps.nT_per_head), _ptr(pred.full_cnt),
+        _ptr(pred.full_idx), _ptr(pred.part_cnt), _ptr(pred.part_idx), pred.stride,
+        _ptr(oracle.full_cnt), _ptr(oracle.full_idx), _ptr(oracle.part_cnt), _ptr(oracle.part_idx),
+        oracle.stride, _ptr(q.mass_rows), _ptr(q.recall_rows), _ptr(q.totals), B, H, nT,
+        _stream(stream)))
+    return q
 
 
 def unpermute(o_t: torch.Tensor, maps: DeviceMaps, N: int, out: Optional[torch.Tensor] = None,

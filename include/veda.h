@@ -12,6 +12,12 @@
  *   5. veda_block_sparse_attn_fwd  attention over the listed key tiles only
  *   6. veda_unpermute              tiles -> raster order
  *
+ * and, for the predictor's teacher signal and its check ("Miowtion" README, Key Features;
+ * "Deploying this checkpoint", sections 4 and 6):
+ *
+ *   veda_block_heat                per-block attention mass of dense attention
+ *   veda_mask_quality              attention mass a mask keeps, recall against the oracle mask
+ *
  * Conventions shared by every call:
  *  - Ownership: the caller allocates and owns every buffer. Pointers named *_dev or
  *    documented as "device" must be device memory of the current CUDA device; the
@@ -271,6 +277,56 @@ VEDA_API veda_status veda_block_sparse_attn_fwd(const void* q, const void* k, co
  */
 VEDA_API veda_status veda_unpermute(const void* o_tiled, void* o, const int32_t* tile_map, int32_t B,
                            int32_t N, int32_t H, int32_t D, int32_t Npad, veda_stream_t stream);
+
+/*
+ * Teacher block heat (device). "Miowtion" README, Key Features / Veda sparse attention:
+ * the predictor is trained against teacher block heat from the dense LSE. For every
+ * (b, h, query tile i) and every key tile j listed for it:
+ *   heat[b][h][i][j] = (1 / n_i) * sum over valid query slots q of tile i
+ *                      of sum over valid key slots k of tile j of exp(scale * q.k - lse[q])
+ * with n_i = tile_valid[h][i]. With the lists of every key tile (step 4 at density 1/1)
+ * and the LSE of step 5 run on those lists (dense attention), each valid row of heat sums
+ * to 1.
+ *   q, k          [B][H][nT*128][128] bf16 (device, output of step 1), 16-byte aligned
+ *   tile_valid    [H][nT] int32 (device)
+ *   full_cnt/idx, part_cnt/idx  block lists as produced by step 4 (device)
+ *   lse           [B][H][nT*128] fp32 (device): natural-log LSE of the query rows
+ *   heat          [B][H][nT][nT] fp32 (device, out): overwritten; entries of blocks not
+ *                 listed are 0
+ * Out-of-range key indices or counts are flagged VEDA_ERR_DEVICE_CHECK.
+ */
+VEDA_API veda_status veda_block_heat(const void* q, const void* k, const int32_t* tile_valid,
+                            const int32_t* full_cnt, const int32_t* full_idx, const int32_t* part_cnt,
+                            const int32_t* part_idx, int32_t list_stride, const float* lse,
+                            float softmax_scale, float* heat, int32_t B, int32_t H, int32_t nT,
+                            int32_t D, veda_stream_t stream);
+
+/*
+ * Quality of a block mask against the oracle mask (device). "Deploying this checkpoint",
+ * section 4 (recall of the predictor against the oracle mask) and section 6 (the attention
+ * mass an oracle mask keeps at a 10% keep ratio). The oracle mask is step 4 run on heat as
+ * the score. For every row (b, h, i < nT_per_head[h]):
+ *   mass_rows[b][h][i]   = sum of heat[b][h][i][j] over the predicted tiles j
+ *   recall_rows[b][h][i] = |predicted & oracle| / |oracle| (0 when the oracle list is empty)
+ * and totals[0..3] receive sum(tile_valid * mass), sum(tile_valid), sum(recall) and the
+ * number of rows with a non-empty oracle list, so that the kept attention mass is
+ * totals[0] / totals[1] and the mean recall totals[2] / totals[3]. Rows i >= nT_per_head[h]
+ * get 0 and do not count.
+ *   heat          [B][H][nT][nT] fp32 (device)
+ *   tile_valid    [H][nT], nT_per_head [H] int32 (device)
+ *   pred_*, orc_* block lists (device) with strides pred_stride, orc_stride
+ *   mass_rows, recall_rows  [B][H][nT] fp32 (device, out); totals [4] fp32 (device, out,
+ *                 overwritten)
+ * Limits: nT <= VEDA_MAX_TILES. Bad counts or indices are flagged VEDA_ERR_DEVICE_CHECK.
+ */
+VEDA_API veda_status veda_mask_quality(const float* heat, const int32_t* tile_valid,
+                              const int32_t* nT_per_head, const int32_t* pred_full_cnt,
+                              const int32_t* pred_full_idx, const int32_t* pred_part_cnt,
+                              const int32_t* pred_part_idx, int32_t pred_stride,
+                              const int32_t* orc_full_cnt, const int32_t* orc_full_idx,
+                              const int32_t* orc_part_cnt, const int32_t* orc_part_idx,
+                              int32_t orc_stride, float* mass_rows, float* recall_rows, float* totals,
+                              int32_t B, int32_t H, int32_t nT, veda_stream_t stream);
 
 /*
  * Self-test of the library's failure detection (no counterpart on the pages). Launches

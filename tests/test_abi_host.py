@@ -83,6 +83,15 @@ def test_device_calls_validate_before_cuda(L):
                                         1, 1, 4, 128, None) == INVALID                 # bad scale
     assert L.veda_block_sparse_attn_fwd(8, 16, 16, 16, 16, 16, 16, 16, 4, 0.1, 16, None,
                                         1, 1, 4, 128, None) == INVALID                 # misaligned q
+    assert L.veda_block_heat(16, 16, 16, 16, 16, 16, 16, 4, None, 0.1, 16,
+                             1, 1, 4, 128, None) == INVALID                            # no LSE
+    assert L.veda_block_heat(16, 16, 16, 16, 16, 16, 16, 4, 16, 0.1, 16,
+                             1, 1, 4, 64, None) == UNSUPPORTED                         # head_dim 64
+    assert L.veda_block_heat(16, 24, 16, 16, 16, 16, 16, 4, 16, 0.1, 16,
+                             1, 1, 4, 128, None) == INVALID                            # misaligned k
+    args = [16] * 7 + [4] + [16] * 4 + [4] + [16] * 3
+    assert L.veda_mask_quality(*args, 1, 1, 4096, None) == INVALID                     # nT too large
+    assert L.veda_mask_quality(*args[:-1], None, 1, 1, 4, None) == INVALID             # no totals
     assert veda.block_scores_workspace_bytes(1, 2, 4) == 2 * 2 * 4 * 128 * 4
 
 
