@@ -461,6 +461,67 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_heat(args):
+    """Teacher block heat and mask quality on the 16:9 clip (not the contract line): the
+    predicted path, every key tile listed (density 1/1), dense attention for the LSE, block
+    heat over all blocks (timed), the oracle mask selected on the heat, and the attention mass
+    kept by the predicted and by the oracle mask plus the predicted mask's recall. The heat
+    kernel does one MUFU ex2 per score, so its roofline is the MUFU rate: 16 ex2 per cycle
+    per SM x 148 SMs x the maximum SM clock."""
+    from block_sparse_attention_max_b200 import veda as V
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = workload(args)
+    inp = synth.make_inputs(w)
+    maps = V.build_tile_map(w.grid, w.head_shapes, w.n_tail, inp.tile_order).to(dev)
+    q, k, v, wq, wk = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.wq, inp.wk))
+    bufs = V.sparse_attention(q, k, v, wq, wk, maps, w.rho, SCALE)
+    B, H, Npad, D = bufs.q_t.shape
+    nT = Npad // 128
+    dense = V.select_blocks(torch.zeros((B, H, nT, nT), dtype=torch.float32, device=dev), maps,
+                            [(1, 1)] * len(w.rho))
+    blocks = _visited_blocks(dense)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n):
+        for _ in range(args.warmup):
+            fn()
+        times = []
+        for _ in range(n):
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            fn()
+            a1.record(stream)
+            a1.synchronize()
+            times.append(a0.elapsed_time(a1))
+        return statistics.median(times)
+
+    o_d = torch.empty_like(bufs.q_t)
+    lse = torch.empty((B, H, Npad), dtype=torch.float32, device=dev)
+    heat = torch.empty((B, H, nT, nT), dtype=torch.float32, device=dev)
+    n = max(3, min(args.steps, 10))
+    dense_ms = timed(lambda: V.block_sparse_attn_fwd(bufs.q_t, bufs.k_t, bufs.v_t, maps, dense, SCALE, o_d, lse), n)
+    heat_ms = timed(lambda: V.block_heat(bufs.q_t, bufs.k_t, maps, dense, lse, SCALE, out=heat), n)
+    orc = V.select_blocks(heat, maps, w.rho)
+    q_pred = V.mask_quality(heat, maps, bufs.lists, orc)
+    q_orc = V.mask_quality(heat, maps, orc, orc)
+    V.check_device_status()
+    ex2 = blocks * 128 * 128
+    peak_ex2 = 16 * 148 * 1.965e9
+    line = {
+        "heat": f"clip16x9: B=1 H={H} grid 31x30x54 (50220 tokens) tile (1,8,16), nT={nT}, all blocks",
+        "blocks": blocks, "dense_attn_ms": dense_ms,
+        "dense_attn_tflops": blocks * FLOP_PER_BLOCK / (dense_ms * 1e-3) / 1e12,
+        "heat_ms": heat_ms,
+        "heat_roofline": {"bound": "alu", "achieved": ex2 / (heat_ms * 1e-3) / 1e12, "unit": "T ex2/s",
+                          "peak": peak_ex2 / 1e12, "frac": ex2 / (heat_ms * 1e-3) / peak_ex2,
+                          "peak_note": "MUFU: 16 ex2 per cycle per SM x 148 SMs x 1965 MHz (maximum SM clock)"},
+        "heat_qk_tflops": blocks * 2 * 128 ** 3 / (heat_ms * 1e-3) / 1e12,
+        "predicted_mask_mass": q_pred.mass, "oracle_mask_mass": q_orc.mass, "predicted_recall": q_pred.recall,
+        "density": f"{w.rho[0][0]}/{w.rho[0][1]}",
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_sweep(args):
     """Density and length sweep of the attention step (not the contract line): for each
     configuration, permute/pool/score/select once, then time the attention call alone
@@ -512,6 +573,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=24)
+    ap.add_argument("--heat", action="store_true",
+                    help="teacher block heat and mask quality on the clip (one JSON line)")
     ap.add_argument("--sweep", action="store_true",
                     help="density / length sweep of the attention step (one JSON line per config)")
     ap.add_argument("--heads", type=int, default=WORKLOAD.H,
@@ -523,6 +586,8 @@ def main():
         run_reference(args)
     elif args.sweep:
         run_sweep(args)
+    elif args.heat:
+        run_heat(args)
     else:
         run_veda(args)
 
