@@ -15,7 +15,7 @@ Sources (web pages, cited by title and section):
   "Key Features", sub-list "Veda sparse attention"; "NEWS" 2026/09/23).
 
 The pages give the steps in prose only; where they leave a step open the reading
-taken here is stated in the function's docstring (readings R1..R19). Everything
+taken here is stated in the function's docstring (readings R1..R21). Everything
 is computed in float64 from the bf16-rounded inputs (exact upcast).
 
 Steps, in the path's order:
@@ -27,6 +27,7 @@ Steps, in the path's order:
 5. ``budgets`` + ``select`` -- Bresenham budgets, forced diagonal, top-k lists
 6. ``attention``     -- softmax attention over the listed key tiles
 7. ``unpermute``     -- scatter back to raster order
+7b. ``transpose_lists`` + ``attention_backward`` -- gradients over the same lists
 8. ``block_heat`` + ``mask_quality`` -- teacher block heat from dense attention, the
    attention mass a mask keeps and its recall against the oracle mask
 
@@ -411,6 +412,67 @@ def dense_attention_raster(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: f
 def predictor_param_count(heads: int, blocks: int, D: int = 128) -> int:
     """Parameters of the per-head residual projections (reading R6): 2 * D * 3D per head per block."""
     return 2 * D * 3 * D * heads * blocks
+
+
+# ---------------------------------------------------------------------------------------
+# 7b. attention backward over the same block lists
+# ---------------------------------------------------------------------------------------
+
+def transpose_lists(lists: BlockLists, nT_per_head: Sequence[int], nT: int):
+    """Query tiles of every key tile: T[b][h][j] = ascending i with j listed for query tile i.
+
+    [README] Key Features / Veda sparse attention: the block-sparse integration carries
+    "transposed backward lists" -- the backward walks, for each key tile, the query tiles
+    that attended to it. Reading R20: full and partial lists together; key tiles past a
+    head's tile count get empty lists.
+    """
+    B = len(lists.full)
+    H = len(lists.full[0])
+    out = [[[[] for _ in range(nT)] for _ in range(H)] for _ in range(B)]
+    for b in range(B):
+        for h in range(H):
+            for i in range(int(nT_per_head[h])):
+                for j in np.concatenate([lists.full[b][h][i], lists.partial[b][h][i]]):
+                    out[b][h][int(j)].append(i)
+    return [[[np.array(sorted(t), np.int64) for t in hh] for hh in bb] for bb in out]
+
+
+def attention_backward(q_tiled: np.ndarray, k_tiled: np.ndarray, v_tiled: np.ndarray, n_valid: np.ndarray,
+                       lists: BlockLists, scale: float, o_tiled: np.ndarray, lse: np.ndarray,
+                       do_tiled: np.ndarray):
+    """Gradients of the block-sparse attention forward with respect to Q, K and V.
+
+    The backward of step 6 for an output gradient dO, over exactly the forward's keys
+    (the valid slots of the listed tiles). Per query row q: P = exp(scale q.k - LSE_q),
+    D_q = dO_q . O_q, dP = dO_q . v, dS = P (dP - D_q); then dQ_q = scale sum_k dS k,
+    dK_k += scale sum_q dS q and dV_k += sum_q P dO_q. Reading R21: pad query slots are
+    treated like the forward treats them (computed, with whatever dO they are given); pad
+    key slots receive no gradient; rows with no listed key tile give dQ = 0.
+    q/k/v/o/do_tiled: [B, H, nT*128, D]; lse: [B, H, nT*128] (the forward's).
+    Returns dq, dk, dv [B, H, nT*128, D].
+    """
+    B, H, Npad, D = q_tiled.shape
+    nT = Npad // TILE
+    dq = np.zeros((B, H, Npad, D))
+    dk = np.zeros((B, H, Npad, D))
+    dv = np.zeros((B, H, Npad, D))
+    for b in range(B):
+        for h in range(H):
+            for r in range(nT):
+                keys = np.sort(np.concatenate([lists.full[b][h][r], lists.partial[b][h][r]]))
+                if len(keys) == 0:
+                    continue
+                idx = np.concatenate([np.arange(j * TILE, j * TILE + int(n_valid[h, j])) for j in keys])
+                sl = slice(r * TILE, (r + 1) * TILE)
+                Q, dO, O = q_tiled[b, h, sl], do_tiled[b, h, sl], o_tiled[b, h, sl]
+                K, V = k_tiled[b, h, idx], v_tiled[b, h, idx]
+                P = np.exp(scale * (Q @ K.T) - lse[b, h, sl][:, None])
+                Dq = (dO * O).sum(axis=1, keepdims=True)
+                dS = P * (dO @ V.T - Dq)
+                dq[b, h, sl] = scale * (dS @ K)
+                dk[b, h, idx] += scale * (dS.T @ Q)
+                dv[b, h, idx] += P.T @ dO
+    return dq, dk, dv
 
 
 # ---------------------------------------------------------------------------------------
