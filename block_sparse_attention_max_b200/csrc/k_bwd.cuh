@@ -1,0 +1,552 @@
+// k_bwd.cuh -- backward of the block-sparse attention forward over the same block lists.
+//
+// "Miowtion" README, Key Features / Veda sparse attention: the block-sparse integration
+// carries "transposed backward lists". For an output gradient dO, per query row q over the
+// forward's keys: P = exp(scale q.k - LSE_q), D_q = dO_q . O_q, dS = P (dO_q . v - D_q),
+// dQ_q = scale sum_k dS k, dK_k += scale sum_q dS q, dV_k += sum_q P dO_q.
+//
+// Three launches:
+//   delta_kernel           D = rowsum(dO * O) per query row (HBM stream)
+//   transpose_lists_kernel query tiles of every key tile (one warp per key tile)
+//   bwd_kernel<kModeDQ>    one query tile per CTA item, over its forward list: S = Q K_j^T,
+//                          dP = dO V_j^T, dS in TMEM, dQ += dS K_j
+//   bwd_kernel<kModeDKDV>  one key tile per CTA item, over its transposed list:
+//                          S^T = K Q_i^T, dP^T = V dO_i^T, P^T and dS^T in TMEM,
+//                          dV += P^T dO_i, dK += dS^T Q_i
+// Both modes share the structure: per item two "fixed" tiles (Q, dO or K, V), per block two
+// "streamed" tiles (K_j, V_j or Q_i, dO_i) in a 2-slot ring; the two score-like MMAs are
+// fixed x streamed^T (shared-memory operands, K-major); the accumulating MMAs read their A
+// operand (dS, P^T, dS^T as bf16) from tensor memory and the streamed tile as an MN-major B
+// operand. Tensor memory: S | dP | acc0 | acc1 (128 columns each). The eight softmax warps
+// use the forward's 16-lane layout (16 rows per warp, rows r0 and r0 + 8 per thread).
+// This version is single-buffered: a block's S/dP MMAs follow the previous block's
+// accumulating MMAs in issue order (so they overwrite S/dP only after those read them).
+#pragma once
+
+#include "k_attn.cuh"
+
+namespace veda {
+namespace bwd {
+
+using attn::kThreads;
+using attn::kTileB;
+using attn::kHalfB;
+
+constexpr int kModeDQ = 0;
+constexpr int kModeDKDV = 1;
+constexpr int kStrSt = 2;                       // streamed ring slots
+constexpr uint32_t kStatB = 1024;               // LSE + D rows of a streamed query tile (dK/dV)
+constexpr uint32_t kSlotB = 2 * kTileB + kStatB;
+constexpr uint32_t kOffFix = 0;                 // two fixed tiles
+constexpr uint32_t kOffStr = 2 * kTileB;        // ring of streamed slots
+constexpr uint32_t kSmemTiles = kOffStr + kStrSt * kSlotB;     // 194 KB
+constexpr uint32_t kSmemBytes = kSmemTiles + 1024;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColDP = 128, kColA0 = 256, kColA1 = 384;
+constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);   // A, B K-major
+constexpr uint32_t kIdescTS = idesc_bf16_f32(128, 128, 0, 1);   // B MN-major
+constexpr int kRec = 8;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct Args {
+  const int32_t* valid;         // [H][nT]
+  // lists of the item: the forward's (dQ: full + partial) or the transposed ones (dK/dV:
+  // full only, part_cnt == nullptr)
+  const int32_t* full_cnt;
+  const int32_t* full_idx;
+  const int32_t* part_cnt;
+  const int32_t* part_idx;
+  int32_t stride;
+  const float* lse;             // [B*H*nT*128] natural-log LSE of the forward
+  const float* delta;           // [B*H*nT*128] D = rowsum(dO * O)
+  __nv_bfloat16* out0;          // dQ (dQ mode) or dV (dK/dV mode) [B*H*nT*128][128]
+  __nv_bfloat16* out1;          // dK (dK/dV mode)
+  int32_t H, nT;
+  int64_t items;                // B*H*nT
+  float scale;                  // softmax scale
+};
+
+struct Bars {
+  uint64_t fix_full, fix_empty, str_full[kStrSt], str_empty[kStrSt];
+  uint64_t s_full, p_full, o_done, o_free, drain;
+  uint64_t rec_full[kRec];
+  int32_t rec_nv[kRec];
+  uint32_t str_op[kStrSt];
+  uint32_t tmem_base;
+  int32_t abort;
+};
+
+enum : uint32_t { kOpNewItem = 1u, kOpLastBlk = 2u, kOpFirstItem = 4u, kOpStop = 8u };
+
+__device__ __forceinline__ int32_t list_len(const Args& a, int64_t u, int32_t& nf, bool& bad) {
+  nf = a.full_cnt[u];
+  const int32_t np = a.part_cnt ? a.part_cnt[u] : 0;
+  bad = nf < 0 || np < 0 || nf > a.stride || np > a.stride || nf + np > a.nT;
+  if (bad) { nf = 0; return 0; }
+  return nf + np;
+}
+__device__ __forceinline__ int32_t list_at(const Args& a, int64_t u, int32_t nf, int32_t j, bool& bad) {
+  const int32_t idx = j < nf ? a.full_idx[u * a.stride + j] : a.part_idx[u * a.stride + (j - nf)];
+  bad = idx < 0 || idx >= a.nT;
+  return bad ? 0 : idx;
+}
+
+// ---------------------------------------------------------------- producer (one thread)
+template <int MODE>
+__device__ __forceinline__ void role_producer(const Args& a, Bars& bars, uint32_t sb, const CUtensorMap* tmF0,
+                                              const CUtensorMap* tmF1, const CUtensorMap* tmS0,
+                                              const CUtensorMap* tmS1, volatile int* abort) {
+  uint32_t sc = 0, fc = 0;
+  bool stop = false;
+  for (int64_t mm = 0; !stop; ++mm) {
+    const int64_t u = attn::cta_item(mm);
+    if (u >= a.items) break;
+    int32_t nf;
+    bool bad;
+    const int32_t n = list_len(a, u, nf, bad);
+    if (n == 0) continue;
+    if (fc > 0 && !mbar_wait(smem_u32(&bars.fix_empty), (fc - 1) & 1, abort, 40)) break;
+    const uint32_t fb = smem_u32(&bars.fix_full);
+    mbar_arrive_expect_tx(fb, 2 * kTileB);
+    const int32_t frow = static_cast<int32_t>(u * 128);
+    tma_load_2d(sb + kOffFix, tmF0, fb, 0, frow);
+    tma_load_2d(sb + kOffFix + kHalfB, tmF0, fb, 64, frow);
+    tma_load_2d(sb + kOffFix + kTileB, tmF1, fb, 0, frow);
+    tma_load_2d(sb + kOffFix + kTileB + kHalfB, tmF1, fb, 64, frow);
+    const int64_t head_row = (u / a.nT) * a.nT;
+    const int32_t* valid_h = a.valid + ((u / a.nT) % a.H) * a.nT;
+    for (int32_t j = 0; j < n; ++j) {
+      bool b2;
+      const int32_t idx = list_at(a, u, nf, j, b2);
+      if (b2) flag_status(ST_BAD_LIST);
+      const int64_t t = head_row + idx;                 // streamed tile (b, h, idx)
+      const int32_t srow = static_cast<int32_t>(t * 128);
+      const uint32_t ss = sc % kStrSt;
+      if (sc >= kStrSt && !mbar_wait(smem_u32(&bars.str_empty[ss]), (sc / kStrSt - 1) & 1, abort, 41)) {
+        stop = true;
+        break;
+      }
+      bars.str_op[ss] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (fc == 0 ? kOpFirstItem : 0u);
+      const uint32_t slot = sb + kOffStr + ss * kSlotB;
+      const uint32_t sbar = smem_u32(&bars.str_full[ss]);
+      mbar_arrive_expect_tx(sbar, 2 * kTileB + (MODE == kModeDKDV ? kStatB : 0u));
+      tma_load_2d(slot, tmS0, sbar, 0, srow);
+      tma_load_2d(slot + kHalfB, tmS0, sbar, 64, srow);
+      tma_load_2d(slot + kTileB, tmS1, sbar, 0, srow);
+      tma_load_2d(slot + kTileB + kHalfB, tmS1, sbar, 64, srow);
+      if (MODE == kModeDKDV) {
+        // the streamed query tile's LSE and D rows (512 B each, 16-byte aligned)
+        bulk_g2s(slot + 2 * kTileB, a.lse + t * 128, 512, sbar);
+        bulk_g2s(slot + 2 * kTileB + 512, a.delta + t * 128, 512, sbar);
+      }
+      if (MODE == kModeDQ) {
+        // block record for the softmax: valid key slots of the streamed key tile (entry
+        // sc % kRec was last read for block sc - kRec, long before slot sc - kStrSt came back)
+        int32_t nv = valid_h[idx];
+        if (nv < 0 || nv > 128) {
+          flag_status(ST_BAD_LIST);
+          nv = nv < 0 ? 0 : 128;
+        }
+        bars.rec_nv[sc % kRec] = nv;
+        mbar_arrive(smem_u32(&bars.rec_full[sc % kRec]));
+      }
+      ++sc;
+    }
+    ++fc;
+  }
+  if (!*abort) {
+    const uint32_t ss = sc % kStrSt;
+    if (sc < kStrSt || mbar_wait(smem_u32(&bars.str_empty[ss]), (sc / kStrSt - 1) & 1, abort, 42)) {
+      bars.str_op[ss] = kOpStop;
+      mbar_arrive(smem_u32(&bars.str_full[ss]));
+    }
+  }
+  if (*abort) {
+    for (uint32_t i = sc > kStrSt ? sc - kStrSt : 0; i < sc; ++i)
+      mbar_wait(smem_u32(&bars.str_full[i % kStrSt]), (i / kStrSt) & 1, nullptr, 43);
+    if (fc > 0) mbar_wait(smem_u32(&bars.fix_full), (fc - 1) & 1, nullptr, 44);
+  }
+}
+
+// ---------------------------------------------------------------- MMA issuer (one thread)
+template <int MODE>
+__device__ __forceinline__ void role_issuer(Bars& bars, uint32_t sb, uint32_t tmem, volatile int* abort) {
+  const uint64_t dF = smem_desc_sw128(sb + kOffFix, 16, 1024);          // fixed tiles, K-major
+  const uint64_t dS = smem_desc_sw128(sb + kOffStr, 16, 1024);          // streamed tiles, K-major
+  const uint64_t dSm = smem_desc_sw128(sb + kOffStr, kHalfB, 1024);     // streamed tiles, MN-major
+  uint32_t fn = 0, items = 0;
+  for (uint32_t g = 0;; ++g) {
+    const uint32_t ss = g % kStrSt;
+    if (!mbar_wait(smem_u32(&bars.str_full[ss]), (g / kStrSt) & 1, abort, 45)) break;
+    const uint32_t op = bars.str_op[ss];
+    if (op & kOpStop) break;
+    if (op & kOpNewItem) {
+      if (!mbar_wait(smem_u32(&bars.fix_full), fn & 1, abort, 46)) break;
+      ++fn;
+    }
+    tc_fence_after();
+    const uint64_t slot_off = static_cast<uint64_t>(ss * (kSlotB >> 4));
+    // S-like = F0 x S0^T, dP-like = F1 x S1^T
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const uint64_t a0 = attn::opaque(dF + static_cast<uint64_t>(t * (kTileB >> 4)));
+      const uint64_t b0 = attn::opaque(dS + slot_off + static_cast<uint64_t>(t * (kTileB >> 4)));
+      const uint32_t d = tmem + (t == 0 ? kColS : kColDP);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t koff = static_cast<uint64_t>((kk >> 2) * (kHalfB >> 4) + (kk & 3) * 2);
+        mma_ss(d, a0 + koff, b0 + koff, kIdescSS, kk > 0 ? 1u : 0u);
+      }
+    }
+    tc_commit(smem_u32(&bars.s_full));
+    if (!mbar_wait(smem_u32(&bars.p_full), g & 1, abort, 47)) break;
+    // the first accumulation of an item overwrites acc: the previous epilogue must be done
+    if ((op & kOpNewItem) && !(op & kOpFirstItem) && !mbar_wait(smem_u32(&bars.o_free), (items - 1) & 1, abort, 48))
+      break;
+    tc_fence_after();
+    const uint32_t acc_first = (op & kOpNewItem) ? 0u : 1u;
+    if (MODE == kModeDQ) {
+      // dQ += dS (over S, bf16) x K_j (streamed tile 0, MN-major)
+      const uint64_t b0 = attn::opaque(dSm + slot_off);
+      const uint32_t pa = tmem + kColS;
+      mma_ts(tmem + kColA0, pa, b0, kIdescTS, acc_first);
+#pragma unroll
+      for (int kk = 1; kk < 8; ++kk)
+        mma_ts(tmem + kColA0, pa + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescTS, 1u);
+    } else {
+      // dV += P^T (over S) x dO_i (streamed tile 1); dK += dS^T (over dP) x Q_i (streamed tile 0)
+      const uint64_t bq = attn::opaque(dSm + slot_off);
+      const uint64_t bo = attn::opaque(dSm + slot_off + static_cast<uint64_t>(kTileB >> 4));
+      mma_ts(tmem + kColA0, tmem + kColS, bo, kIdescTS, acc_first);
+#pragma unroll
+      for (int kk = 1; kk < 8; ++kk)
+        mma_ts(tmem + kColA0, tmem + kColS + kk * 8, bo + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescTS, 1u);
+      mma_ts(tmem + kColA1, tmem + kColDP, bq, kIdescTS, acc_first);
+#pragma unroll
+      for (int kk = 1; kk < 8; ++kk)
+        mma_ts(tmem + kColA1, tmem + kColDP + kk * 8, bq + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescTS, 1u);
+    }
+    tc_commit(smem_u32(&bars.str_empty[ss]));
+    if (op & kOpLastBlk) {
+      tc_commit(smem_u32(&bars.fix_empty));
+      tc_commit(smem_u32(&bars.o_done));
+      ++items;
+    }
+  }
+  tc_commit(smem_u32(&bars.drain));
+  mbar_wait(smem_u32(&bars.drain), 0, nullptr, 49);
+}
+
+// ---------------------------------------------------------------- softmax warps
+// Thread: tile rows r0 = base + lane / 4 and r0 + 8; of every 8-column group k the columns
+// 8k + 2c + {0, 1} (register 4k + e: row e < 2 ? r0 : r1, column 8k + 2c + (e & 1)).
+// dQ mode: rows are queries (their LSE / D from global), columns keys (>= n_valid masked).
+// dK/dV mode: rows are keys (>= n_valid masked), columns queries (LSE / D from the slot).
+template <int MODE>
+__device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t sb, uint32_t tmem, uint32_t warp,
+                                             uint32_t lane) {
+  using namespace attn;
+  volatile int* abort = &bars.abort;
+  const uint32_t base = 32 * (warp & 3) + 16 * (warp >> 2);
+  const uint32_t lane_off = base << 16;
+  const uint32_t r0 = base + lane / 4, c = lane & 3;
+  const float sl2 = a.scale * kLog2e;
+  const uint64_t c2 = f2_pack(__float_as_uint(sl2), __float_as_uint(sl2));
+  uint32_t g = 0, items = 0;
+  for (int64_t mm = 0;; ++mm) {
+    const int64_t u = cta_item(mm);
+    if (u >= a.items) break;
+    int32_t nf;
+    bool bad;
+    const int32_t n = list_len(a, u, nf, bad);
+    __nv_bfloat16* o0r0 = a.out0 + (u * 128 + r0) * 128;
+    __nv_bfloat16* o0r1 = o0r0 + 8 * 128;
+    __nv_bfloat16* o1r0 = MODE == kModeDKDV ? a.out1 + (u * 128 + r0) * 128 : nullptr;
+    __nv_bfloat16* o1r1 = MODE == kModeDKDV ? o1r0 + 8 * 128 : nullptr;
+    if (n == 0) {
+      if (bad && lane == 0 && warp == 0) flag_status(ST_BAD_LIST);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        reinterpret_cast<uint4*>(o0r0 + c * 32)[i] = make_uint4(0, 0, 0, 0);
+        reinterpret_cast<uint4*>(o0r1 + c * 32)[i] = make_uint4(0, 0, 0, 0);
+        if (MODE == kModeDKDV) {
+          reinterpret_cast<uint4*>(o1r0 + c * 32)[i] = make_uint4(0, 0, 0, 0);
+          reinterpret_cast<uint4*>(o1r1 + c * 32)[i] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      continue;
+    }
+    // per-item row statistics (dQ mode) or key-row validity (dK/dV mode)
+    uint64_t nl0 = 0, nl1 = 0;   // -LSE log2e of rows r0, r1 (dQ)
+    float d0 = 0.f, d1 = 0.f;    // D of rows r0, r1 (dQ)
+    bool row0_ok = true, row1_ok = true;
+    if (MODE == kModeDQ) {
+      const float l0 = -a.lse[u * 128 + r0] * kLog2e, l1 = -a.lse[u * 128 + r0 + 8] * kLog2e;
+      nl0 = f2_pack(__float_as_uint(l0), __float_as_uint(l0));
+      nl1 = f2_pack(__float_as_uint(l1), __float_as_uint(l1));
+      d0 = a.delta[u * 128 + r0];
+      d1 = a.delta[u * 128 + r0 + 8];
+    } else {
+      const int32_t h = static_cast<int32_t>((u / a.nT) % a.H), j = static_cast<int32_t>(u % a.nT);
+      const int32_t nvk = a.valid[static_cast<int64_t>(h) * a.nT + j];
+      row0_ok = static_cast<int32_t>(r0) < nvk;
+      row1_ok = static_cast<int32_t>(r0 + 8) < nvk;
+    }
+    bool ok = true;
+    for (int32_t jj = 0; jj < n; ++jj, ++g) {
+      int32_t nv = 128;
+      if (MODE == kModeDQ) {
+        if (!warp_wait_abort(smem_u32(&bars.rec_full[g % kRec]), (g / kRec) & 1, abort, 50)) { ok = false; break; }
+        nv = reinterpret_cast<volatile int32_t*>(bars.rec_nv)[g % kRec];
+      }
+      if (MODE == kModeDKDV) {
+        // the LSE / D rows were written into the slot by the copy engine: observe the slot's
+        // own barrier (already complete) before reading them
+        const uint32_t ss = g % kStrSt;
+        if (!warp_wait_abort(smem_u32(&bars.str_full[ss]), (g / kStrSt) & 1, abort, 53)) { ok = false; break; }
+      }
+      if (!warp_wait_abort(smem_u32(&bars.s_full), g & 1, abort, 51)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t s[64], dp[64];
+      tmem_ld_16x256b_x16(tmem + lane_off + kColS, s);
+      tmem_ld_16x256b_x16(tmem + lane_off + kColDP, dp);
+      tmem_wait_ld();
+      reg_fence(s);
+      reg_fence(dp);
+      if (MODE == kModeDQ && nv < 128) {
+        const int32_t kv0 = (nv - 2 * static_cast<int32_t>(c) + 7) >> 3;
+        const int32_t kv1 = (nv - 2 * static_cast<int32_t>(c) + 6) >> 3;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          if (k >= kv0) { s[4 * k] = 0xFF800000u; s[4 * k + 2] = 0xFF800000u; }   // -inf
+          if (k >= kv1) { s[4 * k + 1] = 0xFF800000u; s[4 * k + 3] = 0xFF800000u; }
+        }
+      }
+      const uint32_t stat = sb + kOffStr + (g % kStrSt) * kSlotB + 2 * kTileB;   // dK/dV: LSE, D
+      uint32_t pk[32];
+      // P (in place of s), and for dK/dV P^T packed over S
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        uint64_t na, nb;
+        if (MODE == kModeDQ) {
+          na = nl0;
+          nb = nl1;
+        } else {
+          // columns are queries: their -LSE log2e, the same for both rows
+          float2 l2;
+          asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(l2.x), "=f"(l2.y)
+                       : "r"(stat + (8 * k + 2 * c) * 4));
+          na = f2_pack(__float_as_uint(-l2.x * kLog2e), __float_as_uint(-l2.y * kLog2e));
+          nb = na;
+        }
+        float x0, x1, y0, y1;
+        f2_unpack(f2_fma(f2_pack(s[4 * k], s[4 * k + 1]), c2, na), x0, x1);
+        f2_unpack(f2_fma(f2_pack(s[4 * k + 2], s[4 * k + 3]), c2, nb), y0, y1);
+        float p0 = ex2_approx(x0), p1 = ex2_approx(x1), q0 = ex2_approx(y0), q1 = ex2_approx(y1);
+        if (MODE == kModeDKDV) {
+          if (!row0_ok) { p0 = 0.f; p1 = 0.f; }
+          if (!row1_ok) { q0 = 0.f; q1 = 0.f; }
+          pk[2 * k] = pack_bf16x2(p0, p1);
+          pk[2 * k + 1] = pack_bf16x2(q0, q1);
+        }
+        s[4 * k] = __float_as_uint(p0); s[4 * k + 1] = __float_as_uint(p1);
+        s[4 * k + 2] = __float_as_uint(q0); s[4 * k + 3] = __float_as_uint(q1);
+      }
+      if (MODE == kModeDKDV) tmem_st_16x128b_x16(tmem + lane_off + kColS, pk);
+      // dS = P (dP - D), packed over S (dQ) or over dP (dK/dV)
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        float da0, da1, db0, db1;
+        if (MODE == kModeDQ) {
+          da0 = da1 = d0;
+          db0 = db1 = d1;
+        } else {
+          float2 dd;
+          asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(dd.x), "=f"(dd.y)
+                       : "r"(stat + 512 + (8 * k + 2 * c) * 4));
+          da0 = db0 = dd.x;
+          da1 = db1 = dd.y;
+        }
+        const float e0 = __uint_as_float(s[4 * k]) * (__uint_as_float(dp[4 * k]) - da0);
+        const float e1 = __uint_as_float(s[4 * k + 1]) * (__uint_as_float(dp[4 * k + 1]) - da1);
+        const float f0 = __uint_as_float(s[4 * k + 2]) * (__uint_as_float(dp[4 * k + 2]) - db0);
+        const float f1 = __uint_as_float(s[4 * k + 3]) * (__uint_as_float(dp[4 * k + 3]) - db1);
+        pk[2 * k] = pack_bf16x2(e0, e1);
+        pk[2 * k + 1] = pack_bf16x2(f0, f1);
+      }
+      tmem_st_16x128b_x16(tmem + lane_off + (MODE == kModeDQ ? kColS : kColDP), pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars.p_full));
+    }
+    if (!ok) break;
+    // epilogue: acc0 (dQ or dV), acc1 (dK) -> bf16 rows; dQ and dK carry the softmax scale
+    if (!warp_wait_abort(smem_u32(&bars.o_done), items & 1, abort, 52)) break;
+    tc_fence_after();
+#pragma unroll 1
+    for (int t = 0; t < (MODE == kModeDKDV ? 2 : 1); ++t) {
+      const float mul = (MODE == kModeDQ || t == 1) ? a.scale : 1.0f;
+      __nv_bfloat16* rA = t == 0 ? o0r0 : o1r0;
+      __nv_bfloat16* rB = t == 0 ? o0r1 : o1r1;
+      const bool zA = MODE == kModeDKDV && !row0_ok, zB = MODE == kModeDKDV && !row1_ok;   // pad key rows
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t o16[16];
+        tmem_ld_16x256b_x4(tmem + lane_off + (t == 0 ? kColA0 : kColA1) + ch * 32, o16);
+        tmem_wait_ld();
+        reg_fence(o16);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int col = ch * 32 + 8 * q + 2 * static_cast<int>(c);
+          *reinterpret_cast<uint32_t*>(rA + col) =
+              zA ? 0u : pack_bf16x2(__uint_as_float(o16[4 * q]) * mul, __uint_as_float(o16[4 * q + 1]) * mul);
+          *reinterpret_cast<uint32_t*>(rB + col) =
+              zB ? 0u : pack_bf16x2(__uint_as_float(o16[4 * q + 2]) * mul, __uint_as_float(o16[4 * q + 3]) * mul);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars.o_free));
+    ++items;
+  }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_kernel(const __grid_constant__ CUtensorMap tmF0, const __grid_constant__ CUtensorMap tmF1,
+           const __grid_constant__ CUtensorMap tmS0, const __grid_constant__ CUtensorMap tmS1, const Args a) {
+  using namespace attn;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ Bars bars;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2;
+  volatile int* abort = &bars.abort;
+  if (tid == 0) {
+    mbar_init(smem_u32(&bars.fix_full), 1);
+    mbar_init(smem_u32(&bars.fix_empty), 1);
+    for (int i = 0; i < kStrSt; ++i) {
+      mbar_init(smem_u32(&bars.str_full[i]), 1);
+      mbar_init(smem_u32(&bars.str_empty[i]), 1);
+    }
+    mbar_init(smem_u32(&bars.s_full), 1);
+    mbar_init(smem_u32(&bars.p_full), 8);
+    mbar_init(smem_u32(&bars.o_done), 1);
+    mbar_init(smem_u32(&bars.o_free), 8);
+    mbar_init(smem_u32(&bars.drain), 1);
+    for (int i = 0; i < kRec; ++i) mbar_init(smem_u32(&bars.rec_full[i]), 1);
+    bars.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(&bars.tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tensormap(&tmF0);
+    prefetch_tensormap(&tmF1);
+    prefetch_tensormap(&tmS0);
+    prefetch_tensormap(&tmS1);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+  if (wg == 2) {
+    reg_dealloc<kControlRegs>();
+    if (warp == 8 && lane == 0)
+      role_producer<MODE>(a, bars, sb, &tmF0, &tmF1, &tmS0, &tmS1, abort);
+    else if (warp == 9 && lane == 0)
+      role_issuer<MODE>(bars, sb, tmem, abort);
+  } else {
+    reg_alloc<kSoftmaxRegs>();
+    softmax_role<MODE>(a, bars, sb, tmem, warp, lane);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------- D = rowsum(dO * O)
+// 16 threads per 256-byte row (16 bytes each), a warp two rows per step.
+__global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ dout,
+                                                    const __nv_bfloat16* __restrict__ o, float* __restrict__ delta,
+                                                    int64_t rows) {
+  const uint32_t c = threadIdx.x & 15;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * (blockDim.x / 16);
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 16) + (threadIdx.x >> 4); r < rows; r += stride) {
+    const uint4 x = *reinterpret_cast<const uint4*>(dout + r * 128 + c * 8);
+    const uint4 y = *reinterpret_cast<const uint4*>(o + r * 128 + c * 8);
+    const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&x);
+    const __nv_bfloat162* yp = reinterpret_cast<const __nv_bfloat162*>(&y);
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 a2 = __bfloat1622float2(xp[i]), b2 = __bfloat1622float2(yp[i]);
+      acc = fmaf(a2.x, b2.x, acc);
+      acc = fmaf(a2.y, b2.y, acc);
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (c == 0) delta[r] = acc;
+  }
+}
+
+// ---------------------------------------------------------------- transposed lists
+// One warp per (b, h, key tile j): for the head's query tiles i in order, a lane tests
+// whether j is in row i's ascending full or partial list (binary search); ballot compaction
+// writes the hits in ascending i.
+__device__ __forceinline__ bool sorted_has(const int32_t* p, int32_t n, int32_t x) {
+  int32_t lo = 0, hi = n;
+  while (lo < hi) {
+    const int32_t mid = (lo + hi) >> 1;
+    if (p[mid] < x) lo = mid + 1; else hi = mid;
+  }
+  return lo < n && p[lo] == x;
+}
+
+__global__ void __launch_bounds__(128) transpose_lists_kernel(const int32_t* full_cnt, const int32_t* full_idx,
+                                                              const int32_t* part_cnt, const int32_t* part_idx,
+                                                              int32_t stride, const int32_t* nT_per_head,
+                                                              int32_t* t_cnt, int32_t* t_idx, int32_t t_stride,
+                                                              int32_t H, int32_t nT, int64_t rows) {
+  const uint32_t lane = threadIdx.x & 31;
+  const int64_t u = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  if (u >= rows) return;
+  const int32_t j = static_cast<int32_t>(u % nT), h = static_cast<int32_t>((u / nT) % H);
+  int32_t nth = nT_per_head[h];
+  if (nth < 0 || nth > nT) {
+    if (lane == 0) flag_status(ST_BAD_LIST);
+    nth = 0;
+  }
+  const int64_t row0 = u - j;   // (b, h, 0)
+  int32_t cnt = 0;
+  uint32_t lt;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt));
+  for (int32_t i0 = 0; i0 < (j < nth ? nth : 0); i0 += 32) {
+    const int32_t i = i0 + static_cast<int32_t>(lane);
+    bool hit = false;
+    if (i < nth) {
+      const int64_t r = row0 + i;
+      int32_t nf = full_cnt[r], np = part_cnt[r];
+      if (nf < 0 || np < 0 || nf > stride || np > stride) { flag_status(ST_BAD_LIST); nf = 0; np = 0; }
+      hit = sorted_has(full_idx + r * stride, nf, j) || sorted_has(part_idx + r * stride, np, j);
+    }
+    const uint32_t bal = __ballot_sync(0xffffffffu, hit);
+    if (hit) {
+      const int32_t pos = cnt + __popc(bal & lt);
+      if (pos < t_stride) t_idx[u * t_stride + pos] = i;
+    }
+    cnt += __popc(bal);
+  }
+  if (lane == 0) {
+    if (cnt > t_stride) flag_status(ST_LIST_OVERFLOW);
+    t_cnt[u] = cnt < t_stride ? cnt : t_stride;
+  }
+}
+
+}  // namespace bwd
+}  // namespace veda

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -12,6 +13,7 @@
 #include "../../include/veda.h"
 #include "k_attn.cuh"
 #include "k_heat.cuh"
+#include "k_bwd.cuh"
 #include "k_gather.cuh"
 #include "k_scores.cuh"
 #include "k_select.cuh"
@@ -78,6 +80,8 @@ veda_status current_device(int& sms) {
     struct { const void* f; int bytes; } attrs[] = {
         {reinterpret_cast<const void*>(attn::attn_fwd_kernel), static_cast<int>(attn::kSmemBytes)},
         {reinterpret_cast<const void*>(heat::heat_kernel), static_cast<int>(attn::kSmemBytes)},
+        {reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDQ>), static_cast<int>(bwd::kSmemBytes)},
+        {reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDKDV>), static_cast<int>(bwd::kSmemBytes)},
     };
     for (auto& x : attrs) {
       e = cudaFuncSetAttribute(x.f, cudaFuncAttributeMaxDynamicSharedMemorySize, x.bytes);
@@ -86,7 +90,9 @@ veda_status current_device(int& sms) {
     // the attention kernel re-splits its registers between warpgroups (setmaxnreg); the
     // split assumes the launch allocation it was built for, so refuse any other build
     const void* split_kernels[] = {reinterpret_cast<const void*>(attn::attn_fwd_kernel),
-                                   reinterpret_cast<const void*>(heat::heat_kernel)};
+                                   reinterpret_cast<const void*>(heat::heat_kernel),
+                                   reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDQ>),
+                                   reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDKDV>)};
     for (const void* f : split_kernels) {
       cudaFuncAttributes fa{};
       if ((e = cudaFuncGetAttributes(&fa, f)) != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
@@ -448,6 +454,85 @@ veda_status veda_mask_quality(const float* heat, const int32_t* tile_valid, cons
   if (blocks > INT32_MAX) return fail(VEDA_ERR_INVALID_ARG, "veda_mask_quality: too many rows");
   heat::mask_quality_kernel<<<static_cast<unsigned>(blocks), 32 * heat::kQualWarps, 0, s>>>(qa);
   return launched("mask_quality_kernel");
+}
+
+veda_status veda_transpose_lists(const int32_t* full_cnt, const int32_t* full_idx, const int32_t* part_cnt,
+                                 const int32_t* part_idx, int32_t list_stride, const int32_t* nT_per_head,
+                                 int32_t* t_cnt, int32_t* t_idx, int32_t t_stride, int32_t B, int32_t H, int32_t nT,
+                                 veda_stream_t stream) {
+  if (!full_cnt || !full_idx || !part_cnt || !part_idx || !nT_per_head || !t_cnt || !t_idx || B <= 0 || H <= 0 ||
+      nT <= 0 || list_stride <= 0 || t_stride <= 0)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_transpose_lists: bad pointer or size");
+  if (t_stride < nT && t_stride < list_stride)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_transpose_lists: t_stride must be >= nT");
+  const int64_t rows = static_cast<int64_t>(B) * H * nT;
+  const int64_t blocks = (rows + 3) / 4;
+  if (blocks > INT32_MAX) return fail(VEDA_ERR_INVALID_ARG, "veda_transpose_lists: too many rows");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  bwd::transpose_lists_kernel<<<static_cast<unsigned>(blocks), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      full_cnt, full_idx, part_cnt, part_idx, list_stride, nT_per_head, t_cnt, t_idx, t_stride, H, nT, rows);
+  return launched("transpose_lists_kernel");
+}
+
+veda_status veda_block_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                       const float* lse, const int32_t* tile_valid, const int32_t* full_cnt,
+                                       const int32_t* full_idx, const int32_t* part_cnt, const int32_t* part_idx,
+                                       int32_t list_stride, const int32_t* t_cnt, const int32_t* t_idx,
+                                       int32_t t_stride, float softmax_scale, void* dq, void* dk, void* dv,
+                                       float* delta, int32_t B, int32_t H, int32_t nT, int32_t D,
+                                       veda_stream_t stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !tile_valid || !full_cnt || !full_idx || !part_cnt || !part_idx ||
+      !t_cnt || !t_idx || !dq || !dk || !dv || !delta || B <= 0 || H <= 0 || nT <= 0 || list_stride <= 0 ||
+      t_stride <= 0)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_sparse_attn_bwd: bad pointer or size");
+  if (D != 128) return fail(VEDA_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_sparse_attn_bwd: softmax_scale must be positive and finite");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 16) || !aligned(delta, 16))
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_sparse_attn_bwd: tensors must be 16-byte aligned");
+  const int64_t rows = static_cast<int64_t>(B) * H * nT * 128;
+  if (rows > INT32_MAX) return fail(VEDA_ERR_INVALID_ARG, "veda_block_sparse_attn_bwd: too many rows");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  if ((st = get_encoder()) != VEDA_OK) return st;
+  CUtensorMap tq, tk, tv, tdo;
+  if ((st = encode_rows(tq, q, rows)) != VEDA_OK) return st;
+  if ((st = encode_rows(tk, k, rows)) != VEDA_OK) return st;
+  if ((st = encode_rows(tv, v, rows)) != VEDA_OK) return st;
+  if ((st = encode_rows(tdo, dout, rows)) != VEDA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // D = rowsum(dO * O)
+  const int64_t dblocks = std::min<int64_t>((rows + 15) / 16, static_cast<int64_t>(sms) * 16);
+  bwd::delta_kernel<<<static_cast<unsigned>(dblocks), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(o), delta, rows);
+  if ((st = launched("delta_kernel")) != VEDA_OK) return st;
+  bwd::Args a{};
+  a.valid = tile_valid;
+  a.lse = lse;
+  a.delta = delta;
+  a.H = H;
+  a.nT = nT;
+  a.items = static_cast<int64_t>(B) * H * nT;
+  a.scale = softmax_scale;
+  // dQ: query tiles over the forward lists (fixed Q, dO; streamed K, V)
+  a.full_cnt = full_cnt; a.full_idx = full_idx; a.part_cnt = part_cnt; a.part_idx = part_idx;
+  a.stride = list_stride;
+  a.out0 = static_cast<__nv_bfloat16*>(dq);
+  a.out1 = nullptr;
+  const unsigned grid = grid_for(a.items, sms, 1);
+  bwd::bwd_kernel<bwd::kModeDQ><<<grid, bwd::kThreads, bwd::kSmemBytes, s>>>(tq, tdo, tk, tv, a);
+  if ((st = launched("bwd_kernel<dQ>")) != VEDA_OK) return st;
+  // dK, dV: key tiles over the transposed lists (fixed K, V; streamed Q, dO)
+  a.full_cnt = t_cnt; a.full_idx = t_idx; a.part_cnt = nullptr; a.part_idx = nullptr;
+  a.stride = t_stride;
+  a.out0 = static_cast<__nv_bfloat16*>(dv);
+  a.out1 = static_cast<__nv_bfloat16*>(dk);
+  bwd::bwd_kernel<bwd::kModeDKDV><<<grid, bwd::kThreads, bwd::kSmemBytes, s>>>(tk, tv, tq, tdo, a);
+  return launched("bwd_kernel<dK,dV>");
 }
 
 // Self-test of the bounded waits: one thread waits on an mbarrier that nothing arrives

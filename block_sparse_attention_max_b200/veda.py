@@ -27,7 +27,8 @@ EXPORTED = (
     "veda_build_tile_map", "veda_permute_tiles", "veda_tile_pool",
     "veda_block_scores_workspace_bytes", "veda_block_scores", "veda_block_scores_noalloc",
     "veda_select_blocks",
-    "veda_block_sparse_attn_fwd", "veda_unpermute", "veda_block_heat", "veda_mask_quality",
+    "veda_block_sparse_attn_fwd", "veda_unpermute", "veda_transpose_lists",
+    "veda_block_sparse_attn_bwd", "veda_block_heat", "veda_mask_quality",
     "veda_check_device_status", "veda_selftest_wait_timeout",
 )
 
@@ -70,6 +71,9 @@ _SIG = {
     "veda_block_sparse_attn_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _F, _P, _P, _I, _I,
                                         _I, _I, _P]),
     "veda_unpermute": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "veda_transpose_lists": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "veda_block_sparse_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I,
+                                        _F, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "veda_block_heat": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _F, _P, _I, _I, _I, _I, _P]),
     "veda_mask_quality": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _I, _P, _P, _P,
                                _I, _I, _I, _P]),
@@ -308,6 +312,45 @@ def block_sparse_attn_fwd(q_t: torch.Tensor, k_t: torch.Tensor, v_t: torch.Tenso
         _ptr(lists.full_idx), _ptr(lists.part_cnt), _ptr(lists.part_idx), lists.stride,
         float(scale), _ptr(out), _ptr(lse), B, H, nT, D, _stream(stream)))
     return out, lse
+
+
+@dataclasses.dataclass
+class TransposedLists:
+    cnt: torch.Tensor    # [B, H, nT] int32: query tiles per key tile
+    idx: torch.Tensor    # [B, H, nT, stride] int32, ascending
+    stride: int
+
+
+def transpose_lists(lists: BlockLists, maps: DeviceMaps, stream=None) -> TransposedLists:
+    """veda_transpose_lists: the query tiles of every key tile (the backward's lists)."""
+    B, H, nT = lists.full_cnt.shape
+    dev = lists.full_cnt.device
+    t = TransposedLists(torch.empty((B, H, nT), dtype=torch.int32, device=dev),
+                        torch.zeros((B, H, nT, nT), dtype=torch.int32, device=dev), nT)
+    _check("veda_transpose_lists", lib().veda_transpose_lists(
+        _ptr(lists.full_cnt), _ptr(lists.full_idx), _ptr(lists.part_cnt), _ptr(lists.part_idx),
+        lists.stride, _ptr(maps.nT_per_head), _ptr(t.cnt), _ptr(t.idx), t.stride, B, H, nT,
+        _stream(stream)))
+    return t
+
+
+def block_sparse_attn_bwd(q_t: torch.Tensor, k_t: torch.Tensor, v_t: torch.Tensor, o_t: torch.Tensor,
+                          do_t: torch.Tensor, lse: torch.Tensor, maps: DeviceMaps, lists: BlockLists,
+                          tlists: TransposedLists, scale: float, stream=None):
+    """veda_block_sparse_attn_bwd: dQ, dK, dV (tile order, bf16) over the forward's lists."""
+    for t, n in ((q_t, "q"), (k_t, "k"), (v_t, "v"), (o_t, "o"), (do_t, "dout")):
+        _need(t, torch.bfloat16, n)
+    _need(lse, torch.float32, "lse")
+    B, H, Npad, D = q_t.shape
+    nT = Npad // 128
+    dq, dk, dv = torch.empty_like(q_t), torch.empty_like(k_t), torch.empty_like(v_t)
+    delta = torch.empty((B, H, Npad), dtype=torch.float32, device=q_t.device)
+    _check("veda_block_sparse_attn_bwd", lib().veda_block_sparse_attn_bwd(
+        _ptr(q_t), _ptr(k_t), _ptr(v_t), _ptr(o_t), _ptr(do_t), _ptr(lse), _ptr(maps.tile_valid),
+        _ptr(lists.full_cnt), _ptr(lists.full_idx), _ptr(lists.part_cnt), _ptr(lists.part_idx),
+        lists.stride, _ptr(tlists.cnt), _ptr(tlists.idx), tlists.stride, float(scale), _ptr(dq),
+        _ptr(dk), _ptr(dv), _ptr(delta), B, H, nT, D, _stream(stream)))
+    return dq, dk, dv
 
 
 def block_heat(q_t: torch.Tensor, k_t: torch.Tensor, maps: DeviceMaps, lists: BlockLists,

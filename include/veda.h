@@ -12,9 +12,11 @@
  *   5. veda_block_sparse_attn_fwd  attention over the listed key tiles only
  *   6. veda_unpermute              tiles -> raster order
  *
- * and, for the predictor's teacher signal and its check ("Miowtion" README, Key Features;
- * "Deploying this checkpoint", sections 4 and 6):
+ * and, for training and for the predictor's teacher signal and its check ("Miowtion" README,
+ * Key Features; "Deploying this checkpoint", sections 4 and 6):
  *
+ *   veda_transpose_lists           query tiles of every key tile (the backward's lists)
+ *   veda_block_sparse_attn_bwd     dQ, dK, dV over the same block lists
  *   veda_block_heat                per-block attention mass of dense attention
  *   veda_mask_quality              attention mass a mask keeps, recall against the oracle mask
  *
@@ -277,6 +279,51 @@ VEDA_API veda_status veda_block_sparse_attn_fwd(const void* q, const void* k, co
  */
 VEDA_API veda_status veda_unpermute(const void* o_tiled, void* o, const int32_t* tile_map, int32_t B,
                            int32_t N, int32_t H, int32_t D, int32_t Npad, veda_stream_t stream);
+
+/*
+ * Transposed block lists for the backward (device). "Miowtion" README, Key Features / Veda
+ * sparse attention ("transposed backward lists"): for every (b, h, key tile j), the query
+ * tiles i < nT_per_head[h] whose full or partial list (as produced by step 4) holds j, in
+ * ascending order.
+ *   full_cnt/idx, part_cnt/idx  forward lists (device), ascending per row, stride list_stride
+ *   nT_per_head   [H] int32 (device)
+ *   t_cnt         [B][H][nT] int32 (device, out); key tiles j >= nT_per_head[h] get 0
+ *   t_idx         [B][H][nT][t_stride] int32 (device, out); t_stride >= nT
+ * Bad counts are flagged VEDA_ERR_DEVICE_CHECK.
+ */
+VEDA_API veda_status veda_transpose_lists(const int32_t* full_cnt, const int32_t* full_idx,
+                                 const int32_t* part_cnt, const int32_t* part_idx,
+                                 int32_t list_stride, const int32_t* nT_per_head, int32_t* t_cnt,
+                                 int32_t* t_idx, int32_t t_stride, int32_t B, int32_t H, int32_t nT,
+                                 veda_stream_t stream);
+
+/*
+ * Backward of step 5 over the same block lists (device). For an output gradient dO, over
+ * exactly the keys the forward visited, per query row q: P = exp(scale q.k - LSE_q),
+ * D_q = dO_q . O_q, dS = P (dO_q . v - D_q); then
+ *   dQ_q = scale * sum_k dS k,   dK_k = scale * sum_q dS q,   dV_k = sum_q P dO_q.
+ * Pad query slots are treated as the forward treats them; pad key slots (slot >=
+ * tile_valid) receive 0; query tiles with no listed key tile get dQ = 0 and key tiles
+ * listed by no query tile get dK = dV = 0.
+ *   q, k, v, o    [B][H][nT*128][128] bf16 (device): the forward's inputs and output
+ *   dout          [B][H][nT*128][128] bf16 (device): dO in tile order (step 1 applied to
+ *                 the raster gradient: pad slots 0)
+ *   lse           [B][H][nT*128] fp32 (device): the forward's LSE
+ *   tile_valid    [H][nT] int32 (device)
+ *   full_cnt/idx, part_cnt/idx  the forward's lists; t_cnt/t_idx from veda_transpose_lists
+ *   dq, dk, dv    [B][H][nT*128][128] bf16 (device, out)
+ *   delta         [B][H][nT*128] fp32 (device): scratch, receives D
+ * All tensors 16-byte aligned. Out-of-range indices or counts are flagged
+ * VEDA_ERR_DEVICE_CHECK.
+ */
+VEDA_API veda_status veda_block_sparse_attn_bwd(const void* q, const void* k, const void* v,
+                                       const void* o, const void* dout, const float* lse,
+                                       const int32_t* tile_valid, const int32_t* full_cnt,
+                                       const int32_t* full_idx, const int32_t* part_cnt,
+                                       const int32_t* part_idx, int32_t list_stride,
+                                       const int32_t* t_cnt, const int32_t* t_idx, int32_t t_stride,
+                                       float softmax_scale, void* dq, void* dk, void* dv, float* delta,
+                                       int32_t B, int32_t H, int32_t nT, int32_t D, veda_stream_t stream);
 
 /*
  * Teacher block heat (device). "Miowtion" README, Key Features / Veda sparse attention:
