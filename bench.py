@@ -522,6 +522,51 @@ def run_heat(args):
     print(json.dumps(line), flush=True)
 
 
+def run_bwd(args):
+    """Backward of the attention step on the 16:9 clip (not the contract line): the predicted
+    path and forward, then the transposed lists and the backward (D, dQ, dK/dV) for a seeded
+    output gradient, timed with CUDA events per stage. Algorithmic work: 2.5x the forward's
+    4*128^3 FLOP per visited block (five 128^3 GEMMs); executed work: 14*128^3 (S and dP are
+    recomputed in both kernels)."""
+    from block_sparse_attention_max_b200 import veda as V
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = _peaks()
+    w = workload(args)
+    inp = synth.make_inputs(w)
+    maps = V.build_tile_map(w.grid, w.head_shapes, w.n_tail, inp.tile_order).to(dev)
+    q, k, v, wq, wk = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.wq, inp.wk))
+    bufs = V.sparse_attention(q, k, v, wq, wk, maps, w.rho, SCALE)
+    gen = torch.Generator().manual_seed(1000 * w.wid + 8)
+    do_t = V.permute_tiles(torch.randn(inp.q.shape, generator=gen).to(torch.bfloat16).to(dev), maps)
+    blocks = _visited_blocks(bufs.lists)
+    stream = torch.cuda.current_stream()
+    t_ms, b_ms = [], []
+    for i in range(args.warmup + max(3, min(args.steps, 10))):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        tl = V.transpose_lists(bufs.lists, maps)
+        e[1].record(stream)
+        V.block_sparse_attn_bwd(bufs.q_t, bufs.k_t, bufs.v_t, bufs.o_t, do_t, bufs.lse, maps, bufs.lists, tl, SCALE)
+        e[2].record(stream)
+        e[2].synchronize()
+        if i >= args.warmup:
+            t_ms.append(e[0].elapsed_time(e[1]))
+            b_ms.append(e[1].elapsed_time(e[2]))
+    V.check_device_status()
+    bms = statistics.median(b_ms)
+    alg = blocks * 10 * 128 ** 3
+    exe = blocks * 14 * 128 ** 3
+    line = {
+        "bwd": f"clip16x9: B=1 H={w.H} grid 31x30x54 (50220 tokens) tile (1,8,16), nT={w.nT}, density 1/10",
+        "blocks": blocks, "transpose_lists_ms": statistics.median(t_ms), "bwd_ms": bms,
+        "bwd_tflops_algorithmic": alg / (bms * 1e-3) / 1e12,
+        "bwd_roofline": {"bound": "tensor", "achieved": exe / (bms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                         "peak": peaks["bf16_sus"], "frac": exe / (bms * 1e-3) / 1e12 / peaks["bf16_sus"],
+                         "note": "executed MMA work (14*128^3 per block) against the measured sustained bf16 peak"},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_sweep(args):
     """Density and length sweep of the attention step (not the contract line): for each
     configuration, permute/pool/score/select once, then time the attention call alone
@@ -573,6 +618,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=24)
+    ap.add_argument("--bwd", action="store_true",
+                    help="backward of the attention step on the clip (one JSON line)")
     ap.add_argument("--heat", action="store_true",
                     help="teacher block heat and mask quality on the clip (one JSON line)")
     ap.add_argument("--sweep", action="store_true",
@@ -588,6 +635,8 @@ def main():
         run_sweep(args)
     elif args.heat:
         run_heat(args)
+    elif args.bwd:
+        run_bwd(args)
     else:
         run_veda(args)
 
