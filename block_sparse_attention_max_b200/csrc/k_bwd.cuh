@@ -46,6 +46,7 @@ constexpr uint32_t kColS = 0, kColDP = 128, kColA0 = 256, kColA1 = 384;
 constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);   // A, B K-major
 constexpr uint32_t kIdescTS = idesc_bf16_f32(128, 128, 0, 1);   // B MN-major
 constexpr int kRec = 8;
+constexpr int kItemRec = 4;                     // item records (dynamic work queue)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Args {
@@ -64,6 +65,7 @@ struct Args {
   int32_t H, nT;
   int64_t items;                // B*H*nT
   float scale;                  // softmax scale
+  int32_t* next_item;           // work-queue counter, zeroed before the launch
 };
 
 struct Bars {
@@ -71,6 +73,11 @@ struct Bars {
   uint64_t s_full, p_full, o_done, o_free, drain;
   uint64_t rec_full[kRec];
   int32_t rec_nv[kRec];
+  // items are taken from a global counter by the producer (transposed lists are very
+  // uneven: a popular key tile is listed by hundreds of query tiles) and handed to the
+  // softmax warps through these records (-1 = no more work)
+  uint64_t item_full[kItemRec], item_free[kItemRec];
+  int32_t item_u[kItemRec];
   uint32_t str_op[kStrSt];
   uint32_t tmem_base;
   int32_t abort;
@@ -98,8 +105,12 @@ __device__ __forceinline__ void role_producer(const Args& a, Bars& bars, uint32_
                                               const CUtensorMap* tmS1, volatile int* abort) {
   uint32_t sc = 0, fc = 0;
   bool stop = false;
-  for (int64_t mm = 0; !stop; ++mm) {
-    const int64_t u = attn::cta_item(mm);
+  for (uint32_t ic = 0; !stop; ++ic) {
+    const uint32_t is = ic % kItemRec;
+    if (ic >= kItemRec && !mbar_wait(smem_u32(&bars.item_free[is]), (ic / kItemRec - 1) & 1, abort, 54)) break;
+    const int64_t u = atomicAdd(a.next_item, 1);
+    bars.item_u[is] = u < a.items ? static_cast<int32_t>(u) : -1;
+    mbar_arrive(smem_u32(&bars.item_full[is]));
     if (u >= a.items) break;
     int32_t nf;
     bool bad;
@@ -253,9 +264,14 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
   const float sl2 = a.scale * kLog2e;
   const uint64_t c2 = f2_pack(__float_as_uint(sl2), __float_as_uint(sl2));
   uint32_t g = 0, items = 0;
-  for (int64_t mm = 0;; ++mm) {
-    const int64_t u = cta_item(mm);
-    if (u >= a.items) break;
+  for (uint32_t ic = 0;; ++ic) {
+    const uint32_t is = ic % kItemRec;
+    if (!warp_wait_abort(smem_u32(&bars.item_full[is]), (ic / kItemRec) & 1, abort, 55)) break;
+    const int32_t ui = reinterpret_cast<volatile int32_t*>(bars.item_u)[is];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars.item_free[is]));
+    if (ui < 0) break;
+    const int64_t u = ui;
     int32_t nf;
     bool bad;
     const int32_t n = list_len(a, u, nf, bad);
@@ -437,6 +453,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmF0, const __grid_constant__ CUt
     mbar_init(smem_u32(&bars.o_free), 8);
     mbar_init(smem_u32(&bars.drain), 1);
     for (int i = 0; i < kRec; ++i) mbar_init(smem_u32(&bars.rec_full[i]), 1);
+    for (int i = 0; i < kItemRec; ++i) {
+      mbar_init(smem_u32(&bars.item_full[i]), 1);
+      mbar_init(smem_u32(&bars.item_free[i]), 8);
+    }
     bars.abort = 0;
     fence_mbar_init();
   }

@@ -505,6 +505,10 @@ veda_status veda_block_sparse_attn_bwd(const void* q, const void* k, const void*
   if ((st = encode_rows(tv, v, rows)) != VEDA_OK) return st;
   if ((st = encode_rows(tdo, dout, rows)) != VEDA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the two kernels' work-queue counters live after the B*H*nT*128 values of D
+  int32_t* counters = reinterpret_cast<int32_t*>(delta + rows);
+  cudaError_t ce = cudaMemsetAsync(counters, 0, 2 * sizeof(int32_t), s);
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaMemsetAsync(work counters)");
   // D = rowsum(dO * O)
   const int64_t dblocks = std::min<int64_t>((rows + 15) / 16, static_cast<int64_t>(sms) * 16);
   bwd::delta_kernel<<<static_cast<unsigned>(dblocks), 256, 0, s>>>(
@@ -518,6 +522,7 @@ veda_status veda_block_sparse_attn_bwd(const void* q, const void* k, const void*
   a.nT = nT;
   a.items = static_cast<int64_t>(B) * H * nT;
   a.scale = softmax_scale;
+  a.next_item = counters;
   // dQ: query tiles over the forward lists (fixed Q, dO; streamed K, V)
   a.full_cnt = full_cnt; a.full_idx = full_idx; a.part_cnt = part_cnt; a.part_idx = part_idx;
   a.stride = list_stride;
@@ -531,6 +536,7 @@ veda_status veda_block_sparse_attn_bwd(const void* q, const void* k, const void*
   a.stride = t_stride;
   a.out0 = static_cast<__nv_bfloat16*>(dv);
   a.out1 = static_cast<__nv_bfloat16*>(dk);
+  a.next_item = counters + 1;
   bwd::bwd_kernel<bwd::kModeDKDV><<<grid, bwd::kThreads, bwd::kSmemBytes, s>>>(tk, tv, tq, tdo, a);
   return launched("bwd_kernel<dK,dV>");
 }

@@ -344,7 +344,7 @@ def block_sparse_attn_bwd(q_t: torch.Tensor, k_t: torch.Tensor, v_t: torch.Tenso
     B, H, Npad, D = q_t.shape
     nT = Npad // 128
     dq, dk, dv = torch.empty_like(q_t), torch.empty_like(k_t), torch.empty_like(v_t)
-    delta = torch.empty((B, H, Npad), dtype=torch.float32, device=q_t.device)
+    delta = torch.empty(B * H * Npad + 4, dtype=torch.float32, device=q_t.device)   # D + work counters
     _check("veda_block_sparse_attn_bwd", lib().veda_block_sparse_attn_bwd(
         _ptr(q_t), _ptr(k_t), _ptr(v_t), _ptr(o_t), _ptr(do_t), _ptr(lse), _ptr(maps.tile_valid),
         _ptr(lists.full_cnt), _ptr(lists.full_idx), _ptr(lists.part_cnt), _ptr(lists.part_idx),

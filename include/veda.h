@@ -312,7 +312,8 @@ VEDA_API veda_status veda_transpose_lists(const int32_t* full_cnt, const int32_t
  *   tile_valid    [H][nT] int32 (device)
  *   full_cnt/idx, part_cnt/idx  the forward's lists; t_cnt/t_idx from veda_transpose_lists
  *   dq, dk, dv    [B][H][nT*128][128] bf16 (device, out)
- *   delta         [B][H][nT*128] fp32 (device): scratch, receives D
+ *   delta         B*H*nT*128 + 4 fp32 values (device): scratch; receives D, then the
+ *                 kernels' work-queue counters (the library zeroes them)
  * All tensors 16-byte aligned. Out-of-range indices or counts are flagged
  * VEDA_ERR_DEVICE_CHECK.
  */
