@@ -324,6 +324,20 @@ def run_veda(args):
         rnd_times.append(a0.elapsed_time(a1))
     V.check_device_status()
     rnd_ms = statistics.median(rnd_times)
+    # fused variant of steps 1 + 2 for Q and K (one read of the raster, no second read of the
+    # tiles), against the separate calls' permute of Q, K and pool of Q, K
+    fused_times = []
+    for i in range(args.warmup + max(3, min(args.steps, 12))):
+        a0, a1 = event(), event()
+        a0.record(stream)
+        V.permute_pool(q, maps, out=bufs.q_t, pooled=bufs.pooled_q)
+        V.permute_pool(k, maps, out=bufs.k_t, pooled=bufs.pooled_k)
+        a1.record(stream)
+        a1.synchronize()
+        if i >= args.warmup:
+            fused_times.append(a0.elapsed_time(a1))
+    V.check_device_status()
+    fused_ms = statistics.median(fused_times)
     attn_secondary = {
         "valid_token_tflops": valid_flop / (attn_ms * 1e-3) / 1e12,
         "dense_equivalent_tflops": 4.0 * D * N * N * H * B / (attn_ms * 1e-3) / 1e12,
@@ -337,8 +351,11 @@ def run_veda(args):
         "pool_GBps": (2 * nbytes + 2 * w.nT * H * 3 * D * 4) / (stage_ms["pool_qk"] * 1e-3) / 1e9,
         "unpermute_GBps": 2 * nbytes / (stage_ms["unpermute"] * 1e-3) / 1e9,
     }
+    hbm["permute_pool_qk_fused_GBps"] = (2 * 2 * nbytes + 2 * w.nT * H * 3 * D * 4) / (fused_ms * 1e-3) / 1e9
     for kname in list(hbm):
         hbm[kname.replace("_GBps", "_frac")] = hbm[kname] / peaks["hbm"]
+    hbm["permute_pool_qk_fused_ms"] = fused_ms
+    hbm["permute_pool_qk_separate_ms"] = stage_ms["permute_qkv"] * 2 / 3 + stage_ms["pool_qk"]
     traffic = _attn_traffic() if H == WORKLOAD.H else None
 
     line = {

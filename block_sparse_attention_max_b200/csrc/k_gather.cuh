@@ -189,4 +189,93 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolArgs a) {
   }
 }
 
+// ------------------------------------------------------------------------------------
+// Steps 1 + 2 fused (a variant; the two calls also stay separate): gather a tile as
+// permute_kernel does and reduce mean / max / min over its valid slots on the way, so the
+// tiled tensor is not read a second time. Thread t holds channels 8 (t & 15) .. + 7 of rows
+// (t >> 4) + 16 i; the two row groups of a warp are combined by one shuffle, the eight warps
+// through shared memory.
+// ------------------------------------------------------------------------------------
+struct PermPoolArgs {
+  GatherArgs g;
+  const int32_t* valid;   // [H][nT]
+  float* pooled;          // [B][H][nT][3][128]
+};
+
+__global__ void __launch_bounds__(kCopyThreads) permute_pool_kernel(const PermPoolArgs p) {
+  __shared__ float red[kCopyThreads / 32][3][128];
+  const GatherArgs& a = p.g;
+  const uint32_t c = threadIdx.x & 15, r0 = threadIdx.x >> 4, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t u = blockIdx.x; u < a.units; u += gridDim.x) {
+    int32_t b, h, t;
+    unit_coords(u, a.H, a.nT, b, h, t);
+    int32_t nv = p.valid[static_cast<int64_t>(h) * a.nT + t];
+    nv = nv < 0 ? 0 : (nv > 128 ? 128 : nv);
+    const int32_t* m = a.map + static_cast<int64_t>(h) * a.Npad + static_cast<int64_t>(t) * 128;
+    int32_t tok[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) tok[i] = __ldg(m + r0 + 16 * i);
+    uint4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[i] = make_uint4(0, 0, 0, 0);
+      if (tok[i] >= a.N) flag_status(ST_BAD_MAP);
+      if (tok[i] >= 0 && tok[i] < a.N)
+        v[i] = ld_stream(a.src + ((static_cast<int64_t>(b) * a.N + tok[i]) * a.H + h) * kRowBytes + c * 16);
+    }
+    uint8_t* dst = a.dst + ((static_cast<int64_t>(b) * a.H + h) * a.Npad + static_cast<int64_t>(t) * 128) * kRowBytes;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) st_v4(dst + (r0 + 16 * i) * kRowBytes + c * 16, v[i]);
+    float sum[8], mx[8], mn[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) { sum[k] = 0.f; mx[k] = -INFINITY; mn[k] = INFINITY; }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (static_cast<int32_t>(r0 + 16 * i) < nv) {
+        const __nv_bfloat162* q = reinterpret_cast<const __nv_bfloat162*>(&v[i]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(q[k]);
+          sum[2 * k] += f.x;
+          sum[2 * k + 1] += f.y;
+          mx[2 * k] = fmaxf(mx[2 * k], f.x);
+          mx[2 * k + 1] = fmaxf(mx[2 * k + 1], f.y);
+          mn[2 * k] = fminf(mn[2 * k], f.x);
+          mn[2 * k + 1] = fminf(mn[2 * k + 1], f.y);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      sum[k] += __shfl_xor_sync(0xffffffffu, sum[k], 16);
+      mx[k] = fmaxf(mx[k], __shfl_xor_sync(0xffffffffu, mx[k], 16));
+      mn[k] = fminf(mn[k], __shfl_xor_sync(0xffffffffu, mn[k], 16));
+    }
+    if (lane < 16) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        red[warp][0][c * 8 + k] = sum[k];
+        red[warp][1][c * 8 + k] = mx[k];
+        red[warp][2][c * 8 + k] = mn[k];
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < 128) {
+      const uint32_t ch = threadIdx.x;
+      float s_ = 0.f, x_ = -INFINITY, n_ = INFINITY;
+#pragma unroll
+      for (int w = 0; w < kCopyThreads / 32; ++w) {
+        s_ += red[w][0][ch];
+        x_ = fmaxf(x_, red[w][1][ch]);
+        n_ = fminf(n_, red[w][2][ch]);
+      }
+      float* o = p.pooled + u * 384;
+      o[ch] = nv > 0 ? s_ / static_cast<float>(nv) : 0.f;
+      o[128 + ch] = nv > 0 ? x_ : 0.f;
+      o[256 + ch] = nv > 0 ? n_ : 0.f;
+    }
+    __syncthreads();
+  }
+}
+
 }  // namespace veda

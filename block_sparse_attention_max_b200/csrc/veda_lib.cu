@@ -29,7 +29,7 @@ struct DeviceInfo {
   bool supported = false;
   int sms = 0;
   bool attrs_set = false;
-  int per_sm_copy = 1, per_sm_unpermute = 1, per_sm_pool = 1;   // resident CTAs per SM
+  int per_sm_copy = 1, per_sm_unpermute = 1, per_sm_pool = 1, per_sm_permpool = 1;   // resident CTAs per SM
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -104,11 +104,13 @@ veda_status current_device(int& sms) {
     // persistent grids: as many CTAs as can be resident at once
     if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_copy, permute_kernel, kCopyThreads, 0)) != cudaSuccess ||
         (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_unpermute, unpermute_kernel, kCopyThreads, 0)) != cudaSuccess ||
-        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_pool, pool_kernel, kPoolThreads, 0)) != cudaSuccess)
+        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_pool, pool_kernel, kPoolThreads, 0)) != cudaSuccess ||
+        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_permpool, permute_pool_kernel, kCopyThreads, 0)) != cudaSuccess)
       return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     d.per_sm_copy = d.per_sm_copy < 1 ? 1 : d.per_sm_copy;
     d.per_sm_unpermute = d.per_sm_unpermute < 1 ? 1 : d.per_sm_unpermute;
     d.per_sm_pool = d.per_sm_pool < 1 ? 1 : d.per_sm_pool;
+    d.per_sm_permpool = d.per_sm_permpool < 1 ? 1 : d.per_sm_permpool;
     d.attrs_set = true;
   }
   sms = d.sms;
@@ -196,6 +198,26 @@ veda_status veda_permute_tiles(const void* x, void* x_tiled, const int32_t* tile
   permute_kernel<<<grid_for(a.units, sms, device_info().per_sm_copy), kCopyThreads, 0,
                    reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return launched("permute_kernel");
+}
+
+veda_status veda_permute_pool(const void* x, void* x_tiled, const int32_t* tile_map, const int32_t* tile_valid,
+                              float* pooled, int32_t B, int32_t N, int32_t H, int32_t D, int32_t Npad,
+                              veda_stream_t stream) {
+  if (!x || !x_tiled || !tile_map || !tile_valid || !pooled || B <= 0 || N <= 0 || H <= 0 || Npad <= 0 ||
+      Npad % 128)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_permute_pool: bad pointer or size");
+  if (D != 128) return fail(VEDA_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (!aligned(x, 16) || !aligned(x_tiled, 16) || !aligned(pooled, 4))
+    return fail(VEDA_ERR_INVALID_ARG, "veda_permute_pool: misaligned buffer");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  PermPoolArgs p{{static_cast<const uint8_t*>(x), static_cast<uint8_t*>(x_tiled), tile_map, B, N, H, Npad,
+                  Npad / 128, static_cast<int64_t>(B) * H * (Npad / 128)},
+                 tile_valid, pooled};
+  permute_pool_kernel<<<grid_for(p.g.units, sms, device_info().per_sm_permpool), kCopyThreads, 0,
+                        reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return launched("permute_pool_kernel");
 }
 
 veda_status veda_unpermute(const void* o_tiled, void* o, const int32_t* tile_map, int32_t B, int32_t N,

@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "VEDA_OK", 1: "VEDA_ERR_INVALID_ARG", 2: "VEDA_ERR_UNSUPPORTE
 
 EXPORTED = (
     "veda_abi_version", "veda_status_string", "veda_last_error", "veda_geometry_sizes",
-    "veda_build_tile_map", "veda_permute_tiles", "veda_tile_pool",
+    "veda_build_tile_map", "veda_permute_tiles", "veda_permute_pool", "veda_tile_pool",
     "veda_block_scores_workspace_bytes", "veda_block_scores", "veda_block_scores_noalloc",
     "veda_select_blocks",
     "veda_block_sparse_attn_fwd", "veda_unpermute", "veda_transpose_lists",
@@ -64,6 +64,7 @@ _SIG = {
     "veda_build_tile_map": (_I, [ctypes.POINTER(Geometry), _P, _P, _P, _P]),
     "veda_permute_tiles": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "veda_tile_pool": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
+    "veda_permute_pool": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "veda_block_scores_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "veda_block_scores": (_I, [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _P]),
     "veda_block_scores_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
@@ -202,6 +203,23 @@ def permute_tiles(x: torch.Tensor, maps: DeviceMaps, out: Optional[torch.Tensor]
     _check("veda_permute_tiles", lib().veda_permute_tiles(
         _ptr(x), _ptr(out), _ptr(maps.tile_map), B, N, H, D, maps.Npad, _stream(stream)))
     return out
+
+
+def permute_pool(x: torch.Tensor, maps: DeviceMaps, out: Optional[torch.Tensor] = None,
+                 pooled: Optional[torch.Tensor] = None, stream=None):
+    """veda_permute_pool: the tile gather and the tile pooling in one pass."""
+    _need(x, torch.bfloat16, "x")
+    B, N, H, D = x.shape
+    if out is None:
+        out = torch.empty((B, H, maps.Npad, D), dtype=torch.bfloat16, device=x.device)
+    if pooled is None:
+        pooled = torch.empty((B, H, maps.Npad // 128, 3, D), dtype=torch.float32, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    _need(pooled, torch.float32, "pooled")
+    _check("veda_permute_pool", lib().veda_permute_pool(
+        _ptr(x), _ptr(out), _ptr(maps.tile_map), _ptr(maps.tile_valid), _ptr(pooled), B, N, H, D,
+        maps.Npad, _stream(stream)))
+    return out, pooled
 
 
 def tile_pool(x_tiled: torch.Tensor, maps: DeviceMaps, out: Optional[torch.Tensor] = None,

@@ -270,6 +270,20 @@ VEDA_API veda_status veda_block_sparse_attn_fwd(const void* q, const void* k, co
                                        int32_t H, int32_t nT, int32_t D, veda_stream_t stream);
 
 /*
+ * Steps 1 and 2 fused (device; a variant of the two calls, which stay available): the tile
+ * gather of veda_permute_tiles and, on the way, the mean / max / min of veda_tile_pool over
+ * each tile's valid slots, so that the tiled tensor is not read a second time. Outputs are
+ * those of the two calls: x_tiled bit-identical, pooled max / min identical, pooled mean
+ * equal up to fp32 summation order.
+ *   x, x_tiled, tile_map, B, N, H, D, Npad  as veda_permute_tiles
+ *   tile_valid    [H][Npad/128] int32 (device)
+ *   pooled        [B][H][Npad/128][3][128] fp32 (device, out)
+ */
+VEDA_API veda_status veda_permute_pool(const void* x, void* x_tiled, const int32_t* tile_map,
+                              const int32_t* tile_valid, float* pooled, int32_t B, int32_t N, int32_t H,
+                              int32_t D, int32_t Npad, veda_stream_t stream);
+
+/*
  * Step 6: scatter tile-order rows back to raster order (device).
  *   o_tiled  [B][H][Npad][D] bf16
  *   o        [B][N][H][D] bf16; o[b][tile_map[h][s]][h] = o_tiled[b][h][s] for every

@@ -264,3 +264,23 @@ def test_bounded_wait_runs_out_and_context_survives():
     assert e.value.status == 4
     V.check_device_status()
     _stage_run(synth.TINY)
+
+
+@pytest.mark.parametrize("w", [synth.TINY, synth.SMALL, synth.MIXED], ids=lambda w: w.name)
+def test_fused_permute_pool(w):
+    """Steps 1 + 2 fused: tiles bit-identical to the permute, max / min identical to the
+    oracle's pooling, mean within 1e-5 relative (fp32 summation order)."""
+    V = P.veda()
+    inp = synth.make_inputs(w)
+    orders = inp.tile_order
+    slots, nv, seg, nTh = P.oracle_maps(w, orders)
+    maps = V.build_tile_map(w.grid, w.head_shapes, w.n_tail, orders).to(DEV)
+    for x in (inp.q, inp.k):
+        xd = x.to(DEV)
+        xt, pooled = V.permute_pool(xd, maps)
+        V.check_device_status()
+        assert torch.equal(xt, V.permute_tiles(xd, maps)), "fused tiles differ from the permute"
+        ref = O.pool(O.permute(P.f64(x), slots), nv)
+        g = P.f64(pooled)
+        assert np.array_equal(g[..., 1:, :], ref[..., 1:, :]), "max/min differ"
+        assert np.allclose(g[..., 0, :], ref[..., 0, :], rtol=1e-5, atol=1e-6), "mean differs"
