@@ -15,7 +15,7 @@ Sources (web pages, cited by title and section):
   "Key Features", sub-list "Veda sparse attention"; "NEWS" 2026/09/23).
 
 The pages give the steps in prose only; where they leave a step open the reading
-taken here is stated in the function's docstring (readings R1..R21). Everything
+taken here is stated in the function's docstring (readings R1..R22). Everything
 is computed in float64 from the bf16-rounded inputs (exact upcast).
 
 Steps, in the path's order:
@@ -30,6 +30,7 @@ Steps, in the path's order:
 7b. ``transpose_lists`` + ``attention_backward`` -- gradients over the same lists
 8. ``block_heat`` + ``mask_quality`` -- teacher block heat from dense attention, the
    attention mass a mask keeps and its recall against the oracle mask
+9. ``shape_errors`` + ``tile_plan`` -- oracle tile-plan search over candidate tile shapes
 
 plus ``dense_attention_raster``, an independent dense routine used as a pin.
 Parity status: every function here is pinned by a ``-m "not gpu"`` test
@@ -551,6 +552,59 @@ def mask_quality(heat: np.ndarray, n_valid: np.ndarray, nT_per_head: Sequence[in
                     rsum += recall_rows[b, h, i]
                     rcount += 1
     return mass_rows, recall_rows, (msum / wsum if wsum else 0.0), (rsum / rcount if rcount else 0.0)
+
+
+# ---------------------------------------------------------------------------------------
+# 9. oracle tile-plan search
+# ---------------------------------------------------------------------------------------
+
+def shape_errors(q: np.ndarray, k: np.ndarray, v: np.ndarray, grid: Tuple[int, int, int], n_tail: int,
+                 candidates: Sequence[Tuple[int, int, int]], rho: Sequence[Tuple[int, int]],
+                 scale: float) -> np.ndarray:
+    """Relative output error of every candidate tile shape under its best mask, per head.
+
+    [README] Key Features / Veda sparse attention: "oracle tile-plan search (relative output
+    MSE under the best mask)". Reading R22: for head h and shape s, tile the head with s,
+    take the oracle mask of section 8 (step 4 on the block heat of s's tiling), run the
+    block-sparse attention with it and return sum over valid tokens of |o_s - o_dense|^2
+    divided by sum |o_dense|^2, with o_dense the dense attention (section 6's raster
+    routine). q, k, v: [B, N, H, D] raster. Returns err [H, len(candidates)] (batch summed).
+    """
+    B, N, H, D = q.shape
+    od, _ = dense_attention_raster(q, k, v, scale)
+    err = np.zeros((H, len(candidates)))
+    for ci, shape in enumerate(candidates):
+        m = tile_map(grid, tuple(shape), n_tail)
+        slots, n_valid, segment = stack_maps([m] * H)
+        nT_h = [len(m.n_valid)] * H
+        qt, kt, vt = permute(q, slots), permute(k, slots), permute(v, slots)
+        heat = block_heat(qt, kt, n_valid, nT_h, scale)
+        mask = select(heat, n_valid, segment, nT_h, rho)
+        o_t, _ = attention(qt, kt, vt, n_valid, mask, scale)
+        o = unpermute(np.nan_to_num(o_t), slots, N)
+        for h in range(H):
+            num = ((o[:, :, h] - od[:, :, h]) ** 2).sum()
+            den = (od[:, :, h] ** 2).sum()
+            err[h, ci] = num / den
+    return err
+
+
+def tile_plan(err: np.ndarray, max_shapes: int = 2) -> Tuple[List[int], np.ndarray]:
+    """Majority vote over the heads' best shapes, at most `max_shapes` shapes per layer.
+
+    [README] Key Features: "majority vote, at most two shapes per layer". Reading R22: each
+    head votes for its lowest-error candidate (ties to the earlier candidate); the layer
+    keeps the `max_shapes` candidates with the most votes (ties to the earlier candidate);
+    every head then takes whichever kept candidate has its lower error (ties to the earlier).
+    err: [H, C]. Returns (kept candidate indices, per-head candidate index [H]).
+    """
+    H, C = err.shape
+    votes = np.bincount(np.argmin(err, axis=1), minlength=C)
+    order = sorted(range(C), key=lambda c: (-votes[c], c))
+    kept = [c for c in order[:max_shapes] if votes[c] > 0] or [order[0]]
+    kept = sorted(kept)
+    assign = np.array([kept[int(np.argmin(err[h, kept]))] for h in range(H)])
+    return kept, assign
 
 
 # ---------------------------------------------------------------------------------------
