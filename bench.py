@@ -584,6 +584,39 @@ def run_bwd(args):
     print(json.dumps(line), flush=True)
 
 
+PLAN_CANDIDATES = [(1, 8, 16), (2, 8, 8), (4, 4, 8), (2, 4, 16), (1, 16, 8)]
+
+
+def run_plan(args):
+    """Oracle tile-plan search on the 16:9 clip (not the contract line): for each candidate
+    tile shape, permute, dense attention for the LSE, block heat, oracle mask, sparse
+    attention and relative output error per head, then the vote (at most two shapes)."""
+    from block_sparse_attention_max_b200 import plan
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = workload(args)
+    inp = synth.make_inputs(w)
+    q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+    plan.tile_plan_search(q, k, v, w.grid, w.n_tail, PLAN_CANDIDATES[:1], w.rho, SCALE)   # warm-up
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    res = plan.tile_plan_search(q, k, v, w.grid, w.n_tail, PLAN_CANDIDATES, w.rho, SCALE)
+    ev1.record()
+    torch.cuda.synchronize()
+    line = {
+        "plan": f"clip16x9: B=1 H={w.H} grid 31x30x54 (50220 tokens), density 1/10, "
+                f"{len(PLAN_CANDIDATES)} candidate shapes",
+        "search_ms_gpu": ev0.elapsed_time(ev1), "search_s_wall": time.perf_counter() - t0,
+        "mean_error_per_shape": {f"{t}x{h}x{ww}": float(res.errors[:, c].mean())
+                                 for c, (t, h, ww) in enumerate(PLAN_CANDIDATES)},
+        "kept_shapes": [f"{t}x{h}x{ww}" for (t, h, ww) in (PLAN_CANDIDATES[c] for c in res.kept)],
+        "heads_per_kept_shape": {f"{t}x{h}x{ww}": int((res.assign == c).sum())
+                                 for c, (t, h, ww) in ((c, PLAN_CANDIDATES[c]) for c in res.kept)},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_sweep(args):
     """Density and length sweep of the attention step (not the contract line): for each
     configuration, permute/pool/score/select once, then time the attention call alone
@@ -635,6 +668,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=24)
+    ap.add_argument("--plan", action="store_true",
+                    help="oracle tile-plan search on the clip (one JSON line)")
     ap.add_argument("--bwd", action="store_true",
                     help="backward of the attention step on the clip (one JSON line)")
     ap.add_argument("--heat", action="store_true",
@@ -654,6 +689,8 @@ def main():
         run_heat(args)
     elif args.bwd:
         run_bwd(args)
+    elif args.plan:
+        run_plan(args)
     else:
         run_veda(args)
 

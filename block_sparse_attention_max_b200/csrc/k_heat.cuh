@@ -241,5 +241,52 @@ __global__ void __launch_bounds__(32 * kQualWarps) mask_quality_kernel(const Qua
   }
 }
 
+// ------------------------------------------------------------------------------------
+// Relative output error per head (the tile-plan search's criterion): sums over all tokens of
+// |o - o_ref|^2 and |o_ref|^2 per head, raster [B][N][H][128] bf16. 16 threads per 256-byte
+// row; per-CTA partial sums in shared memory, one atomic pair per CTA and head.
+// ------------------------------------------------------------------------------------
+constexpr int kErrThreads = 256;
+constexpr int kErrMaxHeads = 256;
+
+__global__ void __launch_bounds__(kErrThreads) rel_error_kernel(const __nv_bfloat16* __restrict__ o,
+                                                                const __nv_bfloat16* __restrict__ ref,
+                                                                float* __restrict__ sums, int64_t rows, int32_t H) {
+  __shared__ float part[kErrMaxHeads][2];
+  for (int i = threadIdx.x; i < H * 2; i += blockDim.x) (&part[0][0])[i] = 0.f;
+  __syncthreads();
+  const uint32_t c = threadIdx.x & 15;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * (kErrThreads / 16);
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * (kErrThreads / 16) + (threadIdx.x >> 4); r < rows; r += stride) {
+    const uint4 x = *reinterpret_cast<const uint4*>(o + r * 128 + c * 8);
+    const uint4 y = *reinterpret_cast<const uint4*>(ref + r * 128 + c * 8);
+    const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&x);
+    const __nv_bfloat162* yp = reinterpret_cast<const __nv_bfloat162*>(&y);
+    float e = 0.f, n = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 a2 = __bfloat1622float2(xp[i]), b2 = __bfloat1622float2(yp[i]);
+      const float d0 = a2.x - b2.x, d1 = a2.y - b2.y;
+      e = fmaf(d0, d0, fmaf(d1, d1, e));
+      n = fmaf(b2.x, b2.x, fmaf(b2.y, b2.y, n));
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) {
+      e += __shfl_xor_sync(0xffffffffu, e, off);
+      n += __shfl_xor_sync(0xffffffffu, n, off);
+    }
+    if (c == 0) {
+      const int32_t h = static_cast<int32_t>(r % H);
+      atomicAdd(&part[h][0], e);
+      atomicAdd(&part[h][1], n);
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < H; i += blockDim.x) {
+    atomicAdd(sums + 2 * i, part[i][0]);
+    atomicAdd(sums + 2 * i + 1, part[i][1]);
+  }
+}
+
 }  // namespace heat
 }  // namespace veda

@@ -563,6 +563,27 @@ veda_status veda_block_sparse_attn_bwd(const void* q, const void* k, const void*
   return launched("bwd_kernel<dK,dV>");
 }
 
+veda_status veda_rel_error(const void* o, const void* o_ref, float* sums, int32_t B, int32_t N, int32_t H,
+                           int32_t D, veda_stream_t stream) {
+  if (!o || !o_ref || !sums || B <= 0 || N <= 0 || H <= 0)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_rel_error: bad pointer or size");
+  if (D != 128) return fail(VEDA_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (H > heat::kErrMaxHeads) return fail(VEDA_ERR_INVALID_ARG, "veda_rel_error: too many heads");
+  if (!aligned(o, 16) || !aligned(o_ref, 16) || !aligned(sums, 4))
+    return fail(VEDA_ERR_INVALID_ARG, "veda_rel_error: misaligned buffer");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(sums, 0, 2 * sizeof(float) * H, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(sums)");
+  const int64_t rows = static_cast<int64_t>(B) * N * H;
+  const int64_t blocks = std::min<int64_t>((rows + 15) / 16, static_cast<int64_t>(sms) * 8);
+  heat::rel_error_kernel<<<static_cast<unsigned>(blocks), heat::kErrThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(o_ref), sums, rows, H);
+  return launched("rel_error_kernel");
+}
+
 // Self-test of the bounded waits: one thread waits on an mbarrier that nothing arrives
 // on; the wait gives up after `limit_ns`, records the timeout and the kernel returns.
 __global__ void wait_selftest_kernel(uint64_t limit_ns) {

@@ -28,7 +28,7 @@ EXPORTED = (
     "veda_block_scores_workspace_bytes", "veda_block_scores", "veda_block_scores_noalloc",
     "veda_select_blocks",
     "veda_block_sparse_attn_fwd", "veda_unpermute", "veda_transpose_lists",
-    "veda_block_sparse_attn_bwd", "veda_block_heat", "veda_mask_quality",
+    "veda_block_sparse_attn_bwd", "veda_block_heat", "veda_mask_quality", "veda_rel_error",
     "veda_check_device_status", "veda_selftest_wait_timeout",
 )
 
@@ -75,6 +75,7 @@ _SIG = {
     "veda_transpose_lists": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
     "veda_block_sparse_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I,
                                         _F, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "veda_rel_error": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
     "veda_block_heat": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _F, _P, _I, _I, _I, _I, _P]),
     "veda_mask_quality": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _I, _P, _P, _P,
                                _I, _I, _I, _P]),
@@ -424,6 +425,17 @@ def mask_quality(heat: torch.Tensor, maps: DeviceMaps, pred: BlockLists, oracle:
         oracle.stride, _ptr(q.mass_rows), _ptr(q.recall_rows), _ptr(q.totals), B, H, nT,
         _stream(stream)))
     return q
+
+
+def rel_error(o: torch.Tensor, o_ref: torch.Tensor, stream=None) -> torch.Tensor:
+    """veda_rel_error: [H, 2] sums of |o - o_ref|^2 and |o_ref|^2 per head (raster bf16)."""
+    _need(o, torch.bfloat16, "o")
+    _need(o_ref, torch.bfloat16, "o_ref")
+    B, N, H, D = o.shape
+    sums = torch.empty((H, 2), dtype=torch.float32, device=o.device)
+    _check("veda_rel_error", lib().veda_rel_error(_ptr(o), _ptr(o_ref), _ptr(sums), B, N, H, D,
+                                                  _stream(stream)))
+    return sums
 
 
 def unpermute(o_t: torch.Tensor, maps: DeviceMaps, N: int, out: Optional[torch.Tensor] = None,

@@ -19,6 +19,7 @@
  *   veda_block_sparse_attn_bwd     dQ, dK, dV over the same block lists
  *   veda_block_heat                per-block attention mass of dense attention
  *   veda_mask_quality              attention mass a mask keeps, recall against the oracle mask
+ *   veda_rel_error                 relative output error per head (tile-plan search)
  *
  * Conventions shared by every call:
  *  - Ownership: the caller allocates and owns every buffer. Pointers named *_dev or
@@ -389,6 +390,18 @@ VEDA_API veda_status veda_mask_quality(const float* heat, const int32_t* tile_va
                               const int32_t* orc_part_cnt, const int32_t* orc_part_idx,
                               int32_t orc_stride, float* mass_rows, float* recall_rows, float* totals,
                               int32_t B, int32_t H, int32_t nT, veda_stream_t stream);
+
+/*
+ * Relative output error per head (device), the criterion of the oracle tile-plan search
+ * ("Miowtion" README, Key Features: "relative output MSE under the best mask"):
+ *   sums[2h]     = sum over b, tokens, channels of (o - o_ref)^2 for head h
+ *   sums[2h + 1] = sum of o_ref^2 for head h
+ * so that the relative error of head h is sums[2h] / sums[2h + 1].
+ *   o, o_ref      [B][N][H][128] bf16 (device), raster order
+ *   sums          [H][2] fp32 (device, out, overwritten); H <= 256
+ */
+VEDA_API veda_status veda_rel_error(const void* o, const void* o_ref, float* sums, int32_t B, int32_t N,
+                           int32_t H, int32_t D, veda_stream_t stream);
 
 /*
  * Self-test of the library's failure detection (no counterpart on the pages). Launches
