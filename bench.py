@@ -23,7 +23,9 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
+from typing import Optional
 
 import numpy as np
 import torch
@@ -88,18 +90,25 @@ class Clocks:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, path: Optional[str] = None):
         self.idx = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        self.path = path or os.path.join(tempfile.gettempdir(), f"veda_clocks_rank{device_index}.csv")
 
     def start(self):
+        """Start sampling every 50 ms and return once the first sample is written (at most
+        3 s), so that the samples cover the timed region that follows."""
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            d = os.path.dirname(self.path)
+            if d:
+                os.makedirs(d, exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
+            t0 = time.time()
+            while time.time() - t0 < 3.0 and self.proc.poll() is None and os.path.getsize(self.path) == 0:
+                time.sleep(0.02)
         except Exception:
             self.proc = None
 
@@ -250,7 +259,7 @@ def run_veda(args):
     flop_step = blocks * FLOP_PER_BLOCK
     launches_per_step = 3 + 2 + 2 + 1 + 1 + 1
 
-    clocks = Clocks(dev.index)
+    clocks = Clocks(dev.index, args.clocks_csv)
     clocks.start()
     if dist:
         dist.barrier()
@@ -667,6 +676,8 @@ def main():
     ap.add_argument("--impl", choices=["veda", "reference"], default="veda")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-csv", default=None,
+                    help="where to keep the nvidia-smi samples of the timed region (default: a temp file)")
     ap.add_argument("--ref-rows", type=int, default=24)
     ap.add_argument("--plan", action="store_true",
                     help="oracle tile-plan search on the clip (one JSON line)")
