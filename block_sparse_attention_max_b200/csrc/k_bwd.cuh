@@ -19,8 +19,15 @@
 // operand (dS, P^T, dS^T as bf16) from tensor memory and the streamed tile as an MN-major B
 // operand. Tensor memory: S | dP | acc0 | acc1 (128 columns each). The eight softmax warps
 // use the forward's 16-lane layout (16 rows per warp, rows r0 and r0 + 8 per thread).
-// This version is single-buffered: a block's S/dP MMAs follow the previous block's
-// accumulating MMAs in issue order (so they overwrite S/dP only after those read them).
+// The MMAs of the next block of an item are issued ahead of the current block's
+// accumulating MMAs wherever tensor memory allows, so the tensor core works while the
+// softmax does (one issuing thread: its MMAs run in issue order, so an MMA that overwrites
+// S or dP always follows the MMA that reads what the softmax wrote there):
+//   dQ:    S has two buffers (the fourth 128-column block is free in this mode); per block
+//          ... dP(j+1) [once the softmax has read dP(j)], dQ(j) [dS(j) written], S(j+2) ...
+//   dK/dV: the softmax hands over in two steps, P^T (exponentials only) and then dS^T
+//          (once dP^T has landed); per block ... dV(j) [P^T(j)], S^T(j+1), dK(j) [dS^T(j)],
+//          dP^T(j+1) ... so the exponentials of block j+1 overlap dK(j) and dP^T(j+1).
 #pragma once
 
 #include "k_attn.cuh"
@@ -43,6 +50,7 @@ constexpr uint32_t kSmemTiles = kOffStr + kStrSt * kSlotB;     // 194 KB
 constexpr uint32_t kSmemBytes = kSmemTiles + 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColDP = 128, kColA0 = 256, kColA1 = 384;
+constexpr uint32_t kColS1 = 384;                // dQ mode: second S buffer (acc1 unused)
 constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);   // A, B K-major
 constexpr uint32_t kIdescTS = idesc_bf16_f32(128, 128, 0, 1);   // B MN-major
 constexpr int kRec = 8;
@@ -70,7 +78,13 @@ struct Args {
 
 struct Bars {
   uint64_t fix_full, fix_empty, str_full[kStrSt], str_empty[kStrSt];
-  uint64_t s_full, p_full, o_done, o_free, drain;
+  uint64_t s_full[2];            // S-like MMA of block g landed (dQ: buffer g & 1; dK/dV: [0])
+  uint64_t dp_full, dp_free;     // dP-like MMA landed / the softmax holds dP (dQ) in registers
+  uint64_t pa_full;              // softmax wrote P^T over S^T (dK/dV)
+  // softmax wrote dS over S (dQ: one barrier per S buffer, since the softmax may finish
+  // block g + 1 before the issuer has looked at block g) or dS^T over dP^T (dK/dV: [0])
+  uint64_t pb_full[2];
+  uint64_t o_done, o_free, drain;
   uint64_t rec_full[kRec];
   int32_t rec_nv[kRec];
   // items are taken from a global counter by the producer (transposed lists are very
@@ -180,13 +194,43 @@ __device__ __forceinline__ void role_producer(const Args& a, Bars& bars, uint32_
 }
 
 // ---------------------------------------------------------------- MMA issuer (one thread)
+// 128 x 128 x 128 products as 8 K16 MMAs: score-like F x S^T (both K-major in shared memory)
+// and accumulating A (bf16 in TMEM) x S (MN-major in shared memory).
+__device__ __forceinline__ void mma_score(uint32_t d, uint64_t a0, uint64_t b0) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t koff = static_cast<uint64_t>((kk >> 2) * (kHalfB >> 4) + (kk & 3) * 2);
+    mma_ss(d, a0 + koff, b0 + koff, kIdescSS, kk > 0 ? 1u : 0u);
+  }
+}
+__device__ __forceinline__ void mma_accum(uint32_t d, uint32_t a_tmem, uint64_t b0, uint32_t acc_first) {
+  mma_ts(d, a_tmem, b0, kIdescTS, acc_first);
+#pragma unroll
+  for (int kk = 1; kk < 8; ++kk)
+    mma_ts(d, a_tmem + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescTS, 1u);
+}
+
 template <int MODE>
 __device__ __forceinline__ void role_issuer(Bars& bars, uint32_t sb, uint32_t tmem, volatile int* abort) {
   const uint64_t dF = smem_desc_sw128(sb + kOffFix, 16, 1024);          // fixed tiles, K-major
   const uint64_t dS = smem_desc_sw128(sb + kOffStr, 16, 1024);          // streamed tiles, K-major
   const uint64_t dSm = smem_desc_sw128(sb + kOffStr, kHalfB, 1024);     // streamed tiles, MN-major
+  const uint64_t fix1 = static_cast<uint64_t>(kTileB >> 4);
+  // S-like = F0 x S0^T of block g into its S buffer; dP-like = F1 x S1^T
+  auto slot = [](uint32_t g) { return static_cast<uint64_t>((g % kStrSt) * (kSlotB >> 4)); };
+  auto s_col = [](uint32_t g) { return MODE == kModeDQ ? ((g & 1) ? kColS1 : kColS) : kColS; };
+  auto issue_s = [&](uint32_t g) {
+    mma_score(tmem + s_col(g), attn::opaque(dF), attn::opaque(dS + slot(g)));
+    tc_commit(smem_u32(&bars.s_full[MODE == kModeDQ ? (g & 1) : 0]));
+  };
+  auto issue_dp = [&](uint32_t g) {
+    mma_score(tmem + kColDP, attn::opaque(dF + fix1), attn::opaque(dS + slot(g) + fix1));
+    tc_commit(smem_u32(&bars.dp_full));
+  };
   uint32_t fn = 0, items = 0;
-  for (uint32_t g = 0;; ++g) {
+  bool head = true;   // block g starts an item: its S / dP are not issued yet
+  bool ok = true;
+  for (uint32_t g = 0; ok; ++g) {
     const uint32_t ss = g % kStrSt;
     if (!mbar_wait(smem_u32(&bars.str_full[ss]), (g / kStrSt) & 1, abort, 45)) break;
     const uint32_t op = bars.str_op[ss];
@@ -196,53 +240,56 @@ __device__ __forceinline__ void role_issuer(Bars& bars, uint32_t sb, uint32_t tm
       ++fn;
     }
     tc_fence_after();
-    const uint64_t slot_off = static_cast<uint64_t>(ss * (kSlotB >> 4));
-    // S-like = F0 x S0^T, dP-like = F1 x S1^T
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const uint64_t a0 = attn::opaque(dF + static_cast<uint64_t>(t * (kTileB >> 4)));
-      const uint64_t b0 = attn::opaque(dS + slot_off + static_cast<uint64_t>(t * (kTileB >> 4)));
-      const uint32_t d = tmem + (t == 0 ? kColS : kColDP);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t koff = static_cast<uint64_t>((kk >> 2) * (kHalfB >> 4) + (kk & 3) * 2);
-        mma_ss(d, a0 + koff, b0 + koff, kIdescSS, kk > 0 ? 1u : 0u);
-      }
+    const bool last = (op & kOpLastBlk) != 0;
+    if (head) {
+      // dQ: dP(g) overwrites dP(g - 1), which the softmax must hold in registers by now
+      if (MODE == kModeDQ && g > 0 && !mbar_wait(smem_u32(&bars.dp_free), (g - 1) & 1, abort, 60)) break;
+      tc_fence_after();
+      issue_s(g);
+      issue_dp(g);
     }
-    tc_commit(smem_u32(&bars.s_full));
-    if (!mbar_wait(smem_u32(&bars.p_full), g & 1, abort, 47)) break;
-    // the first accumulation of an item overwrites acc: the previous epilogue must be done
-    if ((op & kOpNewItem) && !(op & kOpFirstItem) && !mbar_wait(smem_u32(&bars.o_free), (items - 1) & 1, abort, 48))
-      break;
-    tc_fence_after();
     const uint32_t acc_first = (op & kOpNewItem) ? 0u : 1u;
+    const bool need_o_free = (op & kOpNewItem) && !(op & kOpFirstItem);
+    // the next block of the item (its slot is the other ring slot, filled once the
+    // previous block's accumulating MMAs released it)
+    const uint32_t gn = g + 1;
+    if (!last && !mbar_wait(smem_u32(&bars.str_full[gn % kStrSt]), (gn / kStrSt) & 1, abort, 61)) break;
     if (MODE == kModeDQ) {
-      // dQ += dS (over S, bf16) x K_j (streamed tile 0, MN-major)
-      const uint64_t b0 = attn::opaque(dSm + slot_off);
-      const uint32_t pa = tmem + kColS;
-      mma_ts(tmem + kColA0, pa, b0, kIdescTS, acc_first);
-#pragma unroll
-      for (int kk = 1; kk < 8; ++kk)
-        mma_ts(tmem + kColA0, pa + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescTS, 1u);
+      if (!last) {
+        // S(g + 1) goes to the buffer of dS(g - 1), which dQ(g - 1), issued before, reads
+        issue_s(gn);
+        // dP(g + 1) overwrites dP(g) once the softmax holds it in registers
+        if (!mbar_wait(smem_u32(&bars.dp_free), g & 1, abort, 62)) break;
+        tc_fence_after();
+        issue_dp(gn);
+      }
+      // dQ += dS (written over S(g)) x K_g (streamed tile 0, MN-major)
+      if (!mbar_wait(smem_u32(&bars.pb_full[g & 1]), (g >> 1) & 1, abort, 47)) break;
+      // the first accumulation of an item overwrites acc: the previous epilogue must be done
+      if (need_o_free && !mbar_wait(smem_u32(&bars.o_free), (items - 1) & 1, abort, 48)) break;
+      tc_fence_after();
+      mma_accum(tmem + kColA0, tmem + s_col(g), attn::opaque(dSm + slot(g)), acc_first);
+      tc_commit(smem_u32(&bars.str_empty[ss]));
     } else {
-      // dV += P^T (over S) x dO_i (streamed tile 1); dK += dS^T (over dP) x Q_i (streamed tile 0)
-      const uint64_t bq = attn::opaque(dSm + slot_off);
-      const uint64_t bo = attn::opaque(dSm + slot_off + static_cast<uint64_t>(kTileB >> 4));
-      mma_ts(tmem + kColA0, tmem + kColS, bo, kIdescTS, acc_first);
-#pragma unroll
-      for (int kk = 1; kk < 8; ++kk)
-        mma_ts(tmem + kColA0, tmem + kColS + kk * 8, bo + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescTS, 1u);
-      mma_ts(tmem + kColA1, tmem + kColDP, bq, kIdescTS, acc_first);
-#pragma unroll
-      for (int kk = 1; kk < 8; ++kk)
-        mma_ts(tmem + kColA1, tmem + kColDP + kk * 8, bq + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescTS, 1u);
+      // dV += P^T (written over S^T) x dO_g (streamed tile 1)
+      if (!mbar_wait(smem_u32(&bars.pa_full), g & 1, abort, 47)) break;
+      if (need_o_free && !mbar_wait(smem_u32(&bars.o_free), (items - 1) & 1, abort, 48)) break;
+      tc_fence_after();
+      mma_accum(tmem + kColA0, tmem + kColS, attn::opaque(dSm + slot(g) + fix1), acc_first);
+      if (!last) issue_s(gn);    // S^T(g + 1) overwrites P^T(g) after dV(g) has read it
+      // dK += dS^T (written over dP^T) x Q_g (streamed tile 0)
+      if (!mbar_wait(smem_u32(&bars.pb_full[0]), g & 1, abort, 63)) break;
+      tc_fence_after();
+      mma_accum(tmem + kColA1, tmem + kColDP, attn::opaque(dSm + slot(g)), acc_first);
+      if (!last) issue_dp(gn);   // dP^T(g + 1) overwrites dS^T(g) after dK(g) has read it
+      tc_commit(smem_u32(&bars.str_empty[ss]));
     }
-    tc_commit(smem_u32(&bars.str_empty[ss]));
-    if (op & kOpLastBlk) {
+    if (last) {
       tc_commit(smem_u32(&bars.fix_empty));
       tc_commit(smem_u32(&bars.o_done));
       ++items;
     }
+    head = last;
   }
   tc_commit(smem_u32(&bars.drain));
   mbar_wait(smem_u32(&bars.drain), 0, nullptr, 49);
@@ -321,14 +368,26 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
         const uint32_t ss = g % kStrSt;
         if (!warp_wait_abort(smem_u32(&bars.str_full[ss]), (g / kStrSt) & 1, abort, 53)) { ok = false; break; }
       }
-      if (!warp_wait_abort(smem_u32(&bars.s_full), g & 1, abort, 51)) { ok = false; break; }
+      // S of this block (dQ: buffer g & 1, one phase per use; dK/dV: one buffer)
+      const uint32_t colS = MODE == kModeDQ ? ((g & 1) ? kColS1 : kColS) : kColS;
+      if (!warp_wait_abort(smem_u32(&bars.s_full[MODE == kModeDQ ? (g & 1) : 0]),
+                           MODE == kModeDQ ? ((g >> 1) & 1) : (g & 1), abort, 51)) { ok = false; break; }
       tc_fence_after();
       uint32_t s[64], dp[64];
-      tmem_ld_16x256b_x16(tmem + lane_off + kColS, s);
-      tmem_ld_16x256b_x16(tmem + lane_off + kColDP, dp);
+      tmem_ld_16x256b_x16(tmem + lane_off + colS, s);
       tmem_wait_ld();
       reg_fence(s);
-      reg_fence(dp);
+      if (MODE == kModeDQ) {
+        // dP as well, then hand its buffer back so that dP of the next block can be issued
+        if (!warp_wait_abort(smem_u32(&bars.dp_full), g & 1, abort, 56)) { ok = false; break; }
+        tc_fence_after();
+        tmem_ld_16x256b_x16(tmem + lane_off + kColDP, dp);
+        tmem_wait_ld();
+        reg_fence(dp);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars.dp_free));
+      }
       if (MODE == kModeDQ && nv < 128) {
         const int32_t kv0 = (nv - 2 * static_cast<int32_t>(c) + 7) >> 3;
         const int32_t kv1 = (nv - 2 * static_cast<int32_t>(c) + 6) >> 3;
@@ -368,7 +427,19 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
         s[4 * k] = __float_as_uint(p0); s[4 * k + 1] = __float_as_uint(p1);
         s[4 * k + 2] = __float_as_uint(q0); s[4 * k + 3] = __float_as_uint(q1);
       }
-      if (MODE == kModeDKDV) tmem_st_16x128b_x16(tmem + lane_off + kColS, pk);
+      if (MODE == kModeDKDV) {
+        // P^T over S^T: dV(g) can start while dP^T(g) is still on the tensor core
+        tmem_st_16x128b_x16(tmem + lane_off + kColS, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars.pa_full));
+        if (!warp_wait_abort(smem_u32(&bars.dp_full), g & 1, abort, 57)) { ok = false; break; }
+        tc_fence_after();
+        tmem_ld_16x256b_x16(tmem + lane_off + kColDP, dp);
+        tmem_wait_ld();
+        reg_fence(dp);
+      }
       // dS = P (dP - D), packed over S (dQ) or over dP (dK/dV)
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
@@ -390,11 +461,11 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
         pk[2 * k] = pack_bf16x2(e0, e1);
         pk[2 * k + 1] = pack_bf16x2(f0, f1);
       }
-      tmem_st_16x128b_x16(tmem + lane_off + (MODE == kModeDQ ? kColS : kColDP), pk);
+      tmem_st_16x128b_x16(tmem + lane_off + (MODE == kModeDQ ? colS : kColDP), pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars.p_full));
+      if (lane == 0) mbar_arrive(smem_u32(&bars.pb_full[MODE == kModeDQ ? (g & 1) : 0]));
     }
     if (!ok) break;
     // epilogue: acc0 (dQ or dV), acc1 (dK) -> bf16 rows; dQ and dK carry the softmax scale
@@ -447,8 +518,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmF0, const __grid_constant__ CUt
       mbar_init(smem_u32(&bars.str_full[i]), 1);
       mbar_init(smem_u32(&bars.str_empty[i]), 1);
     }
-    mbar_init(smem_u32(&bars.s_full), 1);
-    mbar_init(smem_u32(&bars.p_full), 8);
+    mbar_init(smem_u32(&bars.s_full[0]), 1);
+    mbar_init(smem_u32(&bars.s_full[1]), 1);
+    mbar_init(smem_u32(&bars.dp_full), 1);
+    mbar_init(smem_u32(&bars.dp_free), 8);
+    mbar_init(smem_u32(&bars.pa_full), 8);
+    mbar_init(smem_u32(&bars.pb_full[0]), 8);
+    mbar_init(smem_u32(&bars.pb_full[1]), 8);
     mbar_init(smem_u32(&bars.o_done), 1);
     mbar_init(smem_u32(&bars.o_free), 8);
     mbar_init(smem_u32(&bars.drain), 1);
