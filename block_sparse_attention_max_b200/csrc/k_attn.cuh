@@ -23,9 +23,10 @@
 //   warp 10      P V issuer (one thread): O += P_b V_j, P_b read from tensor memory
 // Tensor memory (512 columns): S0 | S1 | O | P0 | P1. With two S buffers, each freed as
 // soon as the softmax holds it in registers, and P in buffers of its own, the tensor core
-// computes S(j+1) and P V(j-1) while the softmax works on block j. The running maximum is
-// only moved (and O rescaled in TMEM after P V(j-1) has landed) when it grows by more
-// than 2^8; otherwise P uses the stale maximum, exact after the division by the row sum.
+// computes S(j+1) and P V(j-1) while the softmax works on block j. The running maximum (in
+// log2 units) is only moved (and O rescaled in TMEM after P V(j-1) has landed) when it grows
+// by more than 30, i.e. when P would exceed 2^30; otherwise P uses the stale maximum, exact
+// after the division by the row sum.
 //
 // Every wait is bounded (veda_ptx.cuh): when one runs out the CTA raises a shared abort
 // flag, all roles leave their loops, in-flight copies and MMAs are drained with bounded
@@ -54,7 +55,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;         // S_b at 128b, P_b at 384 + 64b
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);   // A, B K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);   // B (V) MN-major
-constexpr float kRescaleLog2 = 8.0f;
+constexpr float kRescaleLog2 = 30.0f;
 // register split (setmaxnreg): two softmax warpgroups and one producer/MMA warpgroup;
 // the total equals the block's allocation at launch (384 threads x 168 registers)
 constexpr int kLaunchRegs = 168;
@@ -277,9 +278,26 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
       }
       // Exponentials with the current running maximum m, computed together with the block's
       // row maxima (one basic block, so the scheduler interleaves the MUFU and max chains).
-      // If a row's maximum grew by more than 2^8 (and always for block 0 of an item, whose
-      // reference is not known yet), the reference moves, O is rescaled and the pass is
-      // repeated; otherwise P uses the stale maximum, exact after the division by the row sum.
+      // If a row's maximum (log2 units) grew by more than 30, the reference moves, O is
+      // rescaled and the pass is repeated; otherwise P uses the stale maximum, exact after the
+      // division by the row sum (P stays below 2^30, far inside bf16 and the fp32 sums of at
+      // most nT * 128 terms). Block 0 of an item takes its row maxima first, so that its
+      // single pass has a reference.
+      if (j == 0) {
+        float a4[4], b4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          a4[q] = fmaxf(__uint_as_float(s[4 * q]), __uint_as_float(s[4 * q + 1]));
+          b4[q] = fmaxf(__uint_as_float(s[4 * q + 2]), __uint_as_float(s[4 * q + 3]));
+        }
+#pragma unroll
+        for (int k = 4; k < 16; ++k) {
+          a4[k & 3] = fmax3(a4[k & 3], __uint_as_float(s[4 * k]), __uint_as_float(s[4 * k + 1]));
+          b4[k & 3] = fmax3(b4[k & 3], __uint_as_float(s[4 * k + 2]), __uint_as_float(s[4 * k + 3]));
+        }
+        m0 = quad_max(fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3]))) * a.scale_log2;
+        m1 = quad_max(fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3]))) * a.scale_log2;
+      }
       const uint64_t c2 = f2_pack(__float_as_uint(a.scale_log2), __float_as_uint(a.scale_log2));
       uint64_t acc0[2], acc1[2];
       uint32_t pk[32];
@@ -311,14 +329,9 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
         }
         const float mb0 = quad_max(fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3]))) * a.scale_log2;
         const float mb1 = quad_max(fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3]))) * a.scale_log2;
-        const bool need0 = j == 0 || mb0 > m0 + kRescaleLog2;
-        const bool need1 = j == 0 || mb1 > m1 + kRescaleLog2;
+        const bool need0 = mb0 > m0 + kRescaleLog2;
+        const bool need1 = mb1 > m1 + kRescaleLog2;
         if (pass == 1 || !__any_sync(0xffffffffu, need0 || need1)) break;
-        if (j == 0) {
-          m0 = mb0;   // block 0: O holds nothing yet
-          m1 = mb1;
-          continue;
-        }
         // O must hold P V of every earlier block before it is rescaled
         const uint32_t gp = g - 1;
         if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 31)) { ok = false; break; }
