@@ -166,6 +166,52 @@ def test_full_density_equals_dense_attention():
     assert dmax <= P.ATTN_MAX_ABS and dmean <= P.ATTN_MEAN_ABS, (dmax, dmean)
 
 
+def test_attention_rescales_when_the_row_maximum_grows():
+    """Scores built so that every listed key tile raises a row's maximum by ~64 (log2 units)
+    over the previous one (and, for the other half of the rows, lowers it): the kernel must
+    move its reference and rescale O each time (without rescaling, P would reach 2^190 and
+    overflow fp32). Key tiles 0-2 are full, tile 3 holds 64 valid slots (partial list)."""
+    V = P.veda()
+    grid, shape = (1, 8, 56), (1, 8, 16)
+    maps = V.build_tile_map(grid, [shape]).to(DEV)
+    slots, nv, seg, nTh = P.oracle_maps(synth.Workload("growth", 11, B=1, H=1, grid=grid, head_shapes=(shape,),
+                                                       rho=((1, 1),), field=False), None)
+    nT = int(nTh[0])
+    assert nT == 4 and list(nv[0]) == [128, 128, 128, 64]
+    g = torch.Generator().manual_seed(11011)
+    Npad = nT * 128
+    sign = torch.ones(128)
+    sign[64:] = -1.0
+    q = sign[:, None] + 0.05 * torch.randn((nT, 128, 128), generator=g)          # [tile, row, d]
+    c = torch.tensor([0.0, 500.0, 1000.0, 1500.0])                                # score level of key tile j
+    k = (c[:, None, None] / 128.0) + 0.5 * torch.randn((nT, 128, 128), generator=g)
+    v = torch.randn((nT, 128, 128), generator=g)
+    q, k, v = (x.reshape(1, 1, Npad, 128).to(torch.bfloat16) for x in (q, k, v))
+    valid = torch.from_numpy(slots[0] >= 0)
+    k[0, 0, ~valid] = 0
+    v[0, 0, ~valid] = 0
+    q[0, 0, ~valid] = 0
+    # the construction does what it claims: consecutive listed tiles grow by > 30 (log2)
+    qf, kf = P.f64(q)[0, 0], P.f64(k)[0, 0]
+    s2 = (qf[:64] @ kf.T) * P.SCALE * math.log2(math.e)
+    row_max = [s2[:, j * 128:j * 128 + int(nv[0][j])].max(axis=1) for j in range(nT)]
+    assert all((row_max[j + 1] - row_max[j]).min() > 30 for j in range(nT - 1))
+    assert (row_max[-1] - row_max[0]).min() > 128
+    full = [[[np.arange(3, dtype=np.int64) for _ in range(nT)]]]
+    part = [[[np.array([3], dtype=np.int64) for _ in range(nT)]]]
+    lists = O.BlockLists(full, part)
+    stride = V.list_stride_for(nT, [(1, 1)])
+    o_g, lse_g = V.block_sparse_attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), maps, P.lists_to_device(lists, 1, 1, nT, stride, DEV),
+                                         P.SCALE)
+    V.check_device_status()
+    o_o, lse_o = O.attention(P.f64(q), P.f64(k), P.f64(v), nv, lists, P.SCALE)
+    og, lg = P.f64(o_g), P.f64(lse_g)
+    assert np.isfinite(og).all() and np.isfinite(lg).all()
+    d = np.abs(og - o_o)
+    assert d.max() <= P.ATTN_MAX_ABS and d.mean() <= P.ATTN_MEAN_ABS, (d.max(), d.mean())
+    assert np.all(np.abs(lg - lse_o) <= 2e-3 + 1e-5 * np.abs(lse_o)), np.abs(lg - lse_o).max()
+
+
 def _end_to_end(w, heads=None, rows=None, attn_rows=None):
     """Public API on the whole workload; every intermediate checked on some heads."""
     V = P.veda()
