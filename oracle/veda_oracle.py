@@ -15,7 +15,7 @@ Sources (web pages, cited by title and section):
   "Key Features", sub-list "Veda sparse attention"; "NEWS" 2026/09/23).
 
 The pages give the steps in prose only; where they leave a step open the reading
-taken here is stated in the function's docstring (readings R1..R22). Everything
+taken here is stated in the function's docstring (readings R1..R23). Everything
 is computed in float64 from the bf16-rounded inputs (exact upcast).
 
 Steps, in the path's order:
@@ -31,6 +31,9 @@ Steps, in the path's order:
 8. ``block_heat`` + ``mask_quality`` -- teacher block heat from dense attention, the
    attention mass a mask keeps and its recall against the oracle mask
 9. ``shape_errors`` + ``tile_plan`` -- oracle tile-plan search over candidate tile shapes
+10. ``quantize_fp8`` / ``dequantize_fp8`` (``e4m3_round``, ``e4m3_codes``, ``e4m3_value``) --
+   the e4m3 tensors of the FP8 attention variant, whose attention is ``attention`` on the
+   dequantised tensors
 
 plus ``dense_attention_raster``, an independent dense routine used as a pin.
 Parity status: every function here is pinned by a ``-m "not gpu"`` test
@@ -605,6 +608,87 @@ def tile_plan(err: np.ndarray, max_shapes: int = 2) -> Tuple[List[int], np.ndarr
     kept = sorted(kept)
     assign = np.array([kept[int(np.argmin(err[h, kept]))] for h in range(H)])
     return kept, assign
+
+
+# ---------------------------------------------------------------------------------------
+# 10. FP8 (e4m3) variant of the attention step
+# ---------------------------------------------------------------------------------------
+# The pages ship their predictor in FP8 ([AGENTS] preamble and section 3) but give no FP8
+# attention; the variant here is this build's. Reading R23: Q, K and V tiles are quantised
+# to e4m3 (OCP FP8 E4M3 "fn": 1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no
+# infinities, codes 0x7F / 0xFF are NaN) with one scale per (batch, head) tensor:
+# scale = amax / 448 and code = e4m3(x * (448 / amax)), both in fp32, rounding to nearest
+# even and saturating to +-448; an all-zero tensor gets scale 1. V is stored as transposed
+# tiles (each 128 x 128 tile as [head-dim channel][key slot]). The attention of the FP8
+# variant is then the attention step on the dequantised tensors (code value * scale).
+
+E4M3_MAX = 448.0
+
+
+def e4m3_round(x: np.ndarray) -> np.ndarray:
+    """Nearest e4m3 value of every element of x (float64 in, float64 out), ties to even,
+    saturating at +-448 (R23). The quantum of x's binade is 2^(floor(log2 |x|) - 3) for
+    normals (|x| >= 2^-6) and 2^-9 for subnormals; 448 = 1.75 * 2^8 is the largest finite."""
+    x = np.asarray(x, dtype=np.float64)
+    if not np.all(np.isfinite(x)):
+        raise ValueError("e4m3_round: non-finite input")
+    a = np.abs(x)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.clip(e, -6, 8)
+    quantum = np.ldexp(1.0, (e - 3).astype(np.int64))
+    v = np.minimum(np.round(a / quantum) * quantum, E4M3_MAX)   # np.round: half to even
+    return np.copysign(v, x)
+
+
+def e4m3_codes(x: np.ndarray) -> np.ndarray:
+    """uint8 e4m3 codes of the nearest e4m3 values of x (see e4m3_round); -0 keeps its sign bit."""
+    x = np.asarray(x, dtype=np.float64)
+    v = np.abs(e4m3_round(x))
+    codes = np.zeros(x.shape, dtype=np.uint8)
+    sub = (v > 0) & (v < 2.0 ** -6)
+    codes[sub] = np.round(v[sub] / 2.0 ** -9).astype(np.uint8)          # exponent field 0
+    nrm = v >= 2.0 ** -6
+    E = np.floor(np.log2(v[nrm]))
+    mant = np.round(v[nrm] / np.ldexp(1.0, E.astype(np.int64)) * 8 - 8).astype(np.int64)
+    codes[nrm] = (((E.astype(np.int64) + 7) << 3) | mant).astype(np.uint8)
+    codes[np.signbit(x)] |= np.uint8(0x80)
+    return codes
+
+
+def e4m3_value(codes: np.ndarray) -> np.ndarray:
+    """float64 value of e4m3 codes (NaN codes 0x7F / 0xFF are rejected)."""
+    c = np.asarray(codes, dtype=np.int64)
+    if np.any((c & 0x7F) == 0x7F):
+        raise ValueError("e4m3_value: NaN code")
+    ef, m = (c >> 3) & 0xF, c & 7
+    mag = np.where(ef == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.ldexp(1.0, ef - 7))
+    return np.where(c & 0x80, -mag, mag)
+
+
+def quantize_fp8(x_tiled: np.ndarray, transpose_tiles: bool = False):
+    """Per-(batch, head) e4m3 quantisation of tiled tensors [B, H, nT*128, D] (R23).
+    Returns (codes uint8 [B, H, nT*128, D], scale float32 [B, H]); with transpose_tiles every
+    128 x D tile of the codes is stored transposed (D = 128)."""
+    B, H, Npad, D = x_tiled.shape
+    x32 = x_tiled.astype(np.float32)
+    amax = np.abs(x32).max(axis=(2, 3)).astype(np.float32)
+    safe = np.where(amax > 0, amax, np.float32(E4M3_MAX)).astype(np.float32)
+    inv = (np.float32(E4M3_MAX) / safe).astype(np.float32)               # 1 for a zero tensor
+    scale = (safe / np.float32(E4M3_MAX)).astype(np.float32)
+    y = (x32 * inv[:, :, None, None]).astype(np.float32)
+    codes = e4m3_codes(y.astype(np.float64))
+    if transpose_tiles:
+        codes = codes.reshape(B, H, Npad // TILE, TILE, D).swapaxes(3, 4).reshape(B, H, Npad, D)
+    return codes, scale
+
+
+def dequantize_fp8(codes: np.ndarray, scale: np.ndarray, transposed_tiles: bool = False) -> np.ndarray:
+    """float64 tensor [B, H, nT*128, D] of quantize_fp8's output (code value * scale)."""
+    B, H, Npad, D = codes.shape
+    c = codes
+    if transposed_tiles:
+        c = c.reshape(B, H, Npad // TILE, D, TILE).swapaxes(3, 4).reshape(B, H, Npad, D)
+    return e4m3_value(c) * scale.astype(np.float64)[:, :, None, None]
 
 
 # ---------------------------------------------------------------------------------------
