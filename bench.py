@@ -593,6 +593,68 @@ def run_bwd(args):
     print(json.dumps(line), flush=True)
 
 
+def run_fp8(args):
+    """FP8 variant of the attention step on the 16:9 clip (not the contract line): the
+    predicted path, then e4m3 quantisation of the tiled Q, K and V (V with transposed tiles)
+    and the FP8 attention over the same lists, timed with CUDA events (median of --steps calls
+    after --warmup), beside the bf16 attention of the same lists. Roofline: 4*128^3 FLOP per
+    visited block against twice the measured sustained bf16 peak (the nominal fp8 / bf16
+    ratio of the tensor cores); quantisation against the measured HBM copy rate on its
+    algorithmic bytes (read 2 B and write 1 B per element of the three tensors)."""
+    from block_sparse_attention_max_b200 import veda as V
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = _peaks()
+    w = workload(args)
+    inp = synth.make_inputs(w)
+    maps = V.build_tile_map(w.grid, w.head_shapes, w.n_tail, inp.tile_order).to(dev)
+    q, k, v, wq, wk = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.wq, inp.wk))
+    bufs = V.sparse_attention(q, k, v, wq, wk, maps, w.rho, SCALE)
+    blocks = _visited_blocks(bufs.lists)
+    stream = torch.cuda.current_stream()
+    q8, sq = V.quantize_fp8(bufs.q_t)
+    k8, sk = V.quantize_fp8(bufs.k_t)
+    vt8, sv = V.quantize_fp8(bufs.v_t, transpose_tiles=True)
+    o8 = torch.empty_like(bufs.o_t)
+    lse8 = torch.empty_like(bufs.lse)
+    ob = torch.empty_like(bufs.o_t)
+    q_ms, a8_ms, ab_ms = [], [], []
+    for i in range(args.warmup + args.steps):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record(stream)
+        V.quantize_fp8(bufs.q_t, codes=q8, scale=sq)
+        V.quantize_fp8(bufs.k_t, codes=k8, scale=sk)
+        V.quantize_fp8(bufs.v_t, transpose_tiles=True, codes=vt8, scale=sv)
+        e[1].record(stream)
+        V.block_sparse_attn_fwd_fp8(q8, k8, vt8, sq, sk, sv, maps, bufs.lists, SCALE, out=o8, lse=lse8)
+        e[2].record(stream)
+        V.block_sparse_attn_fwd(bufs.q_t, bufs.k_t, bufs.v_t, maps, bufs.lists, SCALE, out=ob, lse=bufs.lse)
+        e[3].record(stream)
+        e[3].synchronize()
+        if i >= args.warmup:
+            q_ms.append(e[0].elapsed_time(e[1]))
+            a8_ms.append(e[1].elapsed_time(e[2]))
+            ab_ms.append(e[2].elapsed_time(e[3]))
+    V.check_device_status()
+    qms, ams, bms = statistics.median(q_ms), statistics.median(a8_ms), statistics.median(ab_ms)
+    flop = blocks * 4 * 128 ** 3
+    elems = 3 * bufs.q_t.numel()
+    d = (o8.float() - ob.float()).abs()
+    line = {
+        "fp8": f"clip16x9: B=1 H={w.H} grid 31x30x54 (50220 tokens) tile (1,8,16), nT={w.nT}, density 1/10",
+        "blocks": blocks, "quantize_qkv_ms": qms,
+        "quantize_GBps": elems * 3 / (qms * 1e-3) / 1e9,
+        "quantize_frac_hbm": elems * 3 / (qms * 1e-3) / 1e9 / peaks["hbm"],
+        "attn_fp8_ms": ams, "attn_fp8_tflops": flop / (ams * 1e-3) / 1e12,
+        "attn_bf16_ms": bms, "attn_bf16_tflops": flop / (bms * 1e-3) / 1e12,
+        "fp8_roofline": {"bound": "tensor", "achieved": flop / (ams * 1e-3) / 1e12, "unit": "TFLOP/s",
+                         "peak": 2 * peaks["bf16_sus"], "frac": flop / (ams * 1e-3) / 1e12 / (2 * peaks["bf16_sus"]),
+                         "peak_note": "measured sustained bf16 x 2 (nominal fp8 / bf16 ratio)"},
+        "fp8_vs_bf16_output": {"max_abs": float(d.max()), "mean_abs": float(d.mean()),
+                               "mean_abs_bf16_output": float(ob.float().abs().mean())},
+    }
+    print(json.dumps(line), flush=True)
+
+
 PLAN_CANDIDATES = [(1, 8, 16), (2, 8, 8), (4, 4, 8), (2, 4, 16), (1, 16, 8)]
 
 
@@ -685,6 +747,8 @@ def main():
                     help="backward of the attention step on the clip (one JSON line)")
     ap.add_argument("--heat", action="store_true",
                     help="teacher block heat and mask quality on the clip (one JSON line)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="FP8 (e4m3) variant of the attention step on the clip (one JSON line)")
     ap.add_argument("--sweep", action="store_true",
                     help="density / length sweep of the attention step (one JSON line per config)")
     ap.add_argument("--heads", type=int, default=WORKLOAD.H,
@@ -696,6 +760,8 @@ def main():
         run_reference(args)
     elif args.sweep:
         run_sweep(args)
+    elif args.fp8:
+        run_fp8(args)
     elif args.heat:
         run_heat(args)
     elif args.bwd:

@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libveda.so")
 
 SOURCES = ["veda_lib.cu", "veda_tile_map.cpp"]
-HEADERS = ["veda_ptx.cuh", "k_attn.cuh", "k_heat.cuh", "k_bwd.cuh", "k_gather.cuh", "k_scores.cuh", "k_select.cuh"]
+HEADERS = ["veda_ptx.cuh", "k_attn.cuh", "k_heat.cuh", "k_bwd.cuh", "k_fp8.cuh", "k_gather.cuh", "k_scores.cuh", "k_select.cuh"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",

@@ -14,6 +14,7 @@
 #include "k_attn.cuh"
 #include "k_heat.cuh"
 #include "k_bwd.cuh"
+#include "k_fp8.cuh"
 #include "k_gather.cuh"
 #include "k_scores.cuh"
 #include "k_select.cuh"
@@ -80,6 +81,7 @@ veda_status current_device(int& sms) {
     struct { const void* f; int bytes; } attrs[] = {
         {reinterpret_cast<const void*>(attn::attn_fwd_kernel), static_cast<int>(attn::kSmemBytes)},
         {reinterpret_cast<const void*>(heat::heat_kernel), static_cast<int>(attn::kSmemBytes)},
+        {reinterpret_cast<const void*>(fp8::attn_fwd_fp8_kernel), static_cast<int>(fp8::kSmemBytes)},
         {reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDQ>), static_cast<int>(bwd::kSmemBytes)},
         {reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDKDV>), static_cast<int>(bwd::kSmemBytes)},
     };
@@ -91,6 +93,7 @@ veda_status current_device(int& sms) {
     // split assumes the launch allocation it was built for, so refuse any other build
     const void* split_kernels[] = {reinterpret_cast<const void*>(attn::attn_fwd_kernel),
                                    reinterpret_cast<const void*>(heat::heat_kernel),
+                                   reinterpret_cast<const void*>(fp8::attn_fwd_fp8_kernel),
                                    reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDQ>),
                                    reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDKDV>)};
     for (const void* f : split_kernels) {
@@ -142,6 +145,19 @@ veda_status encode_rows(CUtensorMap& m, const void* base, uint64_t rows) {
   const cuuint32_t box[2] = {64, 128};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(r) + ")");
+  return VEDA_OK;
+}
+
+// e4m3 tiles: rows of 128 bytes, one 128 x 128 box per tile, 128-byte swizzle
+veda_status encode_rows8(CUtensorMap& m, const void* base, uint64_t rows) {
+  const cuuint64_t dims[2] = {128, rows};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(r) + ")");
@@ -408,6 +424,75 @@ veda_status veda_block_sparse_attn_fwd(const void* q, const void* k, const void*
   attn::attn_fwd_kernel<<<grid_for(a.items, sms, 1), attn::kThreads, attn::kSmemBytes,
                           reinterpret_cast<cudaStream_t>(stream)>>>(tq, tk, tv, a);
   return launched("attn_fwd_kernel");
+}
+
+veda_status veda_quantize_fp8(const void* x_tiled, void* codes, float* scale, int32_t B, int32_t H, int32_t nT,
+                             int32_t D, int32_t transpose_tiles, veda_stream_t stream) {
+  if (!x_tiled || !codes || !scale || B <= 0 || H <= 0 || nT <= 0)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_quantize_fp8: bad pointer or size");
+  if (D != 128) return fail(VEDA_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (transpose_tiles != 0 && transpose_tiles != 1)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_quantize_fp8: transpose_tiles must be 0 or 1");
+  if (!aligned(x_tiled, 16) || !aligned(codes, 16) || !aligned(scale, 4))
+    return fail(VEDA_ERR_INVALID_ARG, "veda_quantize_fp8: x_tiled / codes must be 16-byte aligned");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t bh = static_cast<int64_t>(B) * H;
+  cudaError_t e = cudaMemsetAsync(scale, 0, static_cast<size_t>(bh) * sizeof(float), s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scale)");
+  fp8::QuantArgs q{};
+  q.x = static_cast<const __nv_bfloat16*>(x_tiled);
+  q.codes = static_cast<uint8_t*>(codes);
+  q.amax_bits = reinterpret_cast<uint32_t*>(scale);
+  q.scale = scale;
+  q.bh = bh;
+  q.rows = static_cast<int64_t>(nT) * 128;
+  q.transpose = transpose_tiles;
+  const int64_t chunks = (q.rows * 128 + fp8::kAmaxChunk - 1) / fp8::kAmaxChunk;
+  fp8::amax_kernel<<<grid_for(bh * chunks, sms, 8), fp8::kQuantThreads, 0, s>>>(q);
+  if ((st = launched("amax_kernel")) != VEDA_OK) return st;
+  fp8::quant_kernel<<<grid_for(bh * nT, sms, 8), fp8::kQuantThreads, 0, s>>>(q);
+  if ((st = launched("quant_kernel")) != VEDA_OK) return st;
+  fp8::scale_kernel<<<static_cast<int>((bh + 255) / 256), 256, 0, s>>>(q.amax_bits, bh);
+  return launched("scale_kernel");
+}
+
+veda_status veda_block_sparse_attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* q_scale,
+                                           const float* k_scale, const float* v_scale, const int32_t* tile_valid,
+                                           const int32_t* full_cnt, const int32_t* full_idx,
+                                           const int32_t* part_cnt, const int32_t* part_idx, int32_t list_stride,
+                                           float softmax_scale, void* o, float* lse, int32_t B, int32_t H,
+                                           int32_t nT, int32_t D, veda_stream_t stream) {
+  if (!q8 || !k8 || !vt8 || !q_scale || !k_scale || !v_scale || !tile_valid || !full_cnt || !full_idx ||
+      !part_cnt || !part_idx || !o || B <= 0 || H <= 0 || nT <= 0 || list_stride <= 0)
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_sparse_attn_fwd_fp8: bad pointer or size");
+  if (D != 128) return fail(VEDA_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_sparse_attn_fwd_fp8: softmax_scale must be positive and finite");
+  if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(vt8, 16) || !aligned(o, 16))
+    return fail(VEDA_ERR_INVALID_ARG, "veda_block_sparse_attn_fwd_fp8: Q/K/V codes and O must be 16-byte aligned");
+  const int64_t rows = static_cast<int64_t>(B) * H * nT * 128;
+  if (rows > INT32_MAX) return fail(VEDA_ERR_INVALID_ARG, "veda_block_sparse_attn_fwd_fp8: too many rows");
+  int sms;
+  veda_status st = current_device(sms);
+  if (st != VEDA_OK) return st;
+  if ((st = get_encoder()) != VEDA_OK) return st;
+  CUtensorMap tq, tk, tv;
+  if ((st = encode_rows8(tq, q8, rows)) != VEDA_OK) return st;
+  if ((st = encode_rows8(tk, k8, rows)) != VEDA_OK) return st;
+  if ((st = encode_rows8(tv, vt8, rows)) != VEDA_OK) return st;
+  fp8::Args p{};
+  p.a.valid = tile_valid; p.a.full_cnt = full_cnt; p.a.full_idx = full_idx; p.a.part_cnt = part_cnt;
+  p.a.part_idx = part_idx; p.a.o = static_cast<__nv_bfloat16*>(o); p.a.lse = lse;
+  p.a.stride = list_stride; p.a.H = H; p.a.nT = nT;
+  p.a.items = static_cast<int64_t>(B) * H * nT;
+  p.a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.q_scale = q_scale; p.k_scale = k_scale; p.v_scale = v_scale;
+  fp8::attn_fwd_fp8_kernel<<<grid_for(p.a.items, sms, 1), fp8::kThreads, fp8::kSmemBytes,
+                              reinterpret_cast<cudaStream_t>(stream)>>>(tq, tk, tv, p);
+  return launched("attn_fwd_fp8_kernel");
 }
 
 veda_status veda_block_heat(const void* q, const void* k, const int32_t* tile_valid, const int32_t* full_cnt,

@@ -29,6 +29,7 @@ EXPORTED = (
     "veda_select_blocks",
     "veda_block_sparse_attn_fwd", "veda_unpermute", "veda_transpose_lists",
     "veda_block_sparse_attn_bwd", "veda_block_heat", "veda_mask_quality", "veda_rel_error",
+    "veda_quantize_fp8", "veda_block_sparse_attn_fwd_fp8",
     "veda_check_device_status", "veda_selftest_wait_timeout",
 )
 
@@ -72,6 +73,9 @@ _SIG = {
     "veda_block_sparse_attn_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _F, _P, _P, _I, _I,
                                         _I, _I, _P]),
     "veda_unpermute": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "veda_quantize_fp8": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "veda_block_sparse_attn_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _F, _P, _P,
+                                            _I, _I, _I, _I, _P]),
     "veda_transpose_lists": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
     "veda_block_sparse_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I,
                                         _F, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
@@ -329,6 +333,47 @@ def block_sparse_attn_fwd(q_t: torch.Tensor, k_t: torch.Tensor, v_t: torch.Tenso
     _check("veda_block_sparse_attn_fwd", lib().veda_block_sparse_attn_fwd(
         _ptr(q_t), _ptr(k_t), _ptr(v_t), _ptr(maps.tile_valid), _ptr(lists.full_cnt),
         _ptr(lists.full_idx), _ptr(lists.part_cnt), _ptr(lists.part_idx), lists.stride,
+        float(scale), _ptr(out), _ptr(lse), B, H, nT, D, _stream(stream)))
+    return out, lse
+
+
+def quantize_fp8(x_t: torch.Tensor, transpose_tiles: bool = False, codes: Optional[torch.Tensor] = None,
+                 scale: Optional[torch.Tensor] = None, stream=None):
+    """Tiled bf16 [B, H, Npad, 128] -> (e4m3 codes uint8 [B, H, Npad, 128], scale fp32 [B, H]);
+    with transpose_tiles every 128 x 128 tile of the codes is stored transposed (V of the FP8
+    attention)."""
+    _need(x_t, torch.bfloat16, "x_t")
+    B, H, Npad, D = x_t.shape
+    if codes is None:
+        codes = torch.empty((B, H, Npad, D), dtype=torch.uint8, device=x_t.device)
+    if scale is None:
+        scale = torch.empty((B, H), dtype=torch.float32, device=x_t.device)
+    _need(codes, torch.uint8, "codes")
+    _need(scale, torch.float32, "scale")
+    _check("veda_quantize_fp8", lib().veda_quantize_fp8(
+        _ptr(x_t), _ptr(codes), _ptr(scale), B, H, Npad // 128, D, 1 if transpose_tiles else 0, _stream(stream)))
+    return codes, scale
+
+
+def block_sparse_attn_fwd_fp8(q8: torch.Tensor, k8: torch.Tensor, vt8: torch.Tensor, q_scale: torch.Tensor,
+                              k_scale: torch.Tensor, v_scale: torch.Tensor, maps: DeviceMaps, lists: BlockLists,
+                              scale: float, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                              want_lse: bool = True, stream=None):
+    """FP8 variant of the attention step: e4m3 codes of Q, K and (transposed tiles) V with
+    their per-(batch, head) scales -> bf16 O [B, H, Npad, 128] and fp32 LSE."""
+    for t, n in ((q8, "q8"), (k8, "k8"), (vt8, "vt8")):
+        _need(t, torch.uint8, n)
+    for t, n in ((q_scale, "q_scale"), (k_scale, "k_scale"), (v_scale, "v_scale")):
+        _need(t, torch.float32, n)
+    B, H, Npad, D = q8.shape
+    nT = Npad // 128
+    if out is None:
+        out = torch.empty((B, H, Npad, D), dtype=torch.bfloat16, device=q8.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, Npad), dtype=torch.float32, device=q8.device)
+    _check("veda_block_sparse_attn_fwd_fp8", lib().veda_block_sparse_attn_fwd_fp8(
+        _ptr(q8), _ptr(k8), _ptr(vt8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale), _ptr(maps.tile_valid),
+        _ptr(lists.full_cnt), _ptr(lists.full_idx), _ptr(lists.part_cnt), _ptr(lists.part_idx), lists.stride,
         float(scale), _ptr(out), _ptr(lse), B, H, nT, D, _stream(stream)))
     return out, lse
 

@@ -21,6 +21,12 @@
  *   veda_mask_quality              attention mass a mask keeps, recall against the oracle mask
  *   veda_rel_error                 relative output error per head (tile-plan search)
  *
+ * and an FP8 variant of step 5 (the pages ship their predictor in FP8, "Deploying this
+ * checkpoint", preamble and section 3; the attention variant is this library's):
+ *
+ *   veda_quantize_fp8              tiled bf16 -> e4m3 codes with one scale per (batch, head)
+ *   veda_block_sparse_attn_fwd_fp8 step 5 with e4m3 Q / K / V and e4m3 P on the tensor cores
+ *
  * Conventions shared by every call:
  *  - Ownership: the caller allocates and owns every buffer. Pointers named *_dev or
  *    documented as "device" must be device memory of the current CUDA device; the
@@ -340,6 +346,47 @@ VEDA_API veda_status veda_block_sparse_attn_bwd(const void* q, const void* k, co
                                        const int32_t* t_cnt, const int32_t* t_idx, int32_t t_stride,
                                        float softmax_scale, void* dq, void* dk, void* dv, float* delta,
                                        int32_t B, int32_t H, int32_t nT, int32_t D, veda_stream_t stream);
+
+/*
+ * FP8 variant, quantisation (device): tiled bf16 tensors -> e4m3 codes (OCP FP8 E4M3, no
+ * infinities) with one scale per (batch, head): scale = max |x| / 448 and
+ * code = e4m3(x * (448 / max |x|)), both in fp32, rounding to nearest even and saturating at
+ * +-448; an all-zero (batch, head) gets scale 1. With transpose_tiles = 1 every 128 x 128
+ * tile of the codes is stored transposed ([channel][key slot]), the layout the FP8 attention
+ * takes for V.
+ *   x_tiled          [B][H][nT*128][D] bf16 (device)
+ *   codes            [B][H][nT*128][D] uint8 e4m3 (device, out)
+ *   scale            [B][H] fp32 (device, out; also used as scratch during the call)
+ *   transpose_tiles  0 or 1
+ * Three launches and one memset on `stream`. Errors: VEDA_ERR_INVALID_ARG (null pointer,
+ * size <= 0, transpose_tiles not 0/1, x_tiled / codes not 16-byte aligned),
+ * VEDA_ERR_UNSUPPORTED (D != 128, device other than sm_100).
+ */
+VEDA_API veda_status veda_quantize_fp8(const void* x_tiled, void* codes, float* scale, int32_t B, int32_t H,
+                                       int32_t nT, int32_t D, int32_t transpose_tiles, veda_stream_t stream);
+
+/*
+ * FP8 variant of step 5 (device): the attention of veda_block_sparse_attn_fwd over the same
+ * lists, from e4m3 operands. S = (Q codes)(K codes)^T on the tensor cores, times
+ * q_scale * k_scale * softmax_scale; P = 2^(s - m + 7) enters P V as e4m3 (the row reference
+ * m moves when a row maximum grows by more than 1.75 in log2 units, so that 2^7 P stays
+ * below 448); O = (P V) * v_scale / l in bf16, LSE as in the bf16 call.
+ *   q8, k8        [B][H][nT*128][D] uint8 e4m3 codes (veda_quantize_fp8, transpose_tiles 0)
+ *   vt8           [B][H][nT*128][D] uint8 e4m3 codes of V with transposed tiles
+ *                 (veda_quantize_fp8, transpose_tiles 1)
+ *   q_scale, k_scale, v_scale   [B][H] fp32 (device) scales of the three tensors
+ *   tile_valid, full_cnt, full_idx, part_cnt, part_idx, list_stride, softmax_scale, o, lse,
+ *   B, H, nT, D   as veda_block_sparse_attn_fwd
+ * Errors as veda_block_sparse_attn_fwd (codes and O 16-byte aligned).
+ */
+VEDA_API veda_status veda_block_sparse_attn_fwd_fp8(const void* q8, const void* k8, const void* vt8,
+                                                    const float* q_scale, const float* k_scale,
+                                                    const float* v_scale, const int32_t* tile_valid,
+                                                    const int32_t* full_cnt, const int32_t* full_idx,
+                                                    const int32_t* part_cnt, const int32_t* part_idx,
+                                                    int32_t list_stride, float softmax_scale, void* o, float* lse,
+                                                    int32_t B, int32_t H, int32_t nT, int32_t D,
+                                                    veda_stream_t stream);
 
 /*
  * Teacher block heat (device). "Miowtion" README, Key Features / Veda sparse attention:

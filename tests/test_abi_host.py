@@ -92,6 +92,16 @@ def test_device_calls_validate_before_cuda(L):
     args = [16] * 7 + [4] + [16] * 4 + [4] + [16] * 3
     assert L.veda_mask_quality(*args, 1, 1, 4096, None) == INVALID                     # nT too large
     assert L.veda_mask_quality(*args[:-1], None, 1, 1, 4, None) == INVALID             # no totals
+    # FP8 variant
+    assert L.veda_quantize_fp8(None, 16, 16, 1, 1, 4, 128, 0, None) == INVALID          # no input
+    assert L.veda_quantize_fp8(16, 16, 16, 1, 1, 4, 128, 2, None) == INVALID            # transpose 2
+    assert L.veda_quantize_fp8(16, 16, 16, 1, 1, 4, 64, 0, None) == UNSUPPORTED         # head_dim 64
+    assert L.veda_quantize_fp8(16, 24, 16, 1, 1, 4, 128, 0, None) == INVALID            # misaligned codes
+    f8 = [16] * 11
+    assert L.veda_block_sparse_attn_fwd_fp8(*([None] + f8[1:]), 4, 0.1, 16, 16, 1, 1, 4, 128, None) == INVALID
+    assert L.veda_block_sparse_attn_fwd_fp8(*f8, 4, -1.0, 16, 16, 1, 1, 4, 128, None) == INVALID   # bad scale
+    assert L.veda_block_sparse_attn_fwd_fp8(*f8, 4, 0.1, 16, 16, 1, 1, 4, 64, None) == UNSUPPORTED
+    assert L.veda_block_sparse_attn_fwd_fp8(*([24] + f8[1:]), 4, 0.1, 16, 16, 1, 1, 4, 128, None) == INVALID
     assert veda.block_scores_workspace_bytes(1, 2, 4) == 2 * 2 * 4 * 128 * 4
 
 

@@ -1,0 +1,137 @@
+"""GPU parity of the FP8 (e4m3) variant of the attention step, through the C ABI.
+
+Quantisation: the GPU's e4m3 codes and per-(batch, head) scales of the tiled Q, K and V
+(V with transposed tiles) equal the oracle's bit for bit (both sides form x * (448 / amax)
+in fp32 and round to nearest even, reading R23).
+Attention: the GPU's FP8 attention over its own block lists is compared with the oracle's
+fp64 attention of the oracle's dequantised tensors over the same lists (fed back as the
+parity rule feeds the selection its scores). The scores then agree up to fp32 summation
+(products of two e4m3 values are exact); what differs is that P enters P V as e4m3 of 2^7 P
+(relative rounding <= 2^-4 on normals) while the row sum stays fp32, so per element
+|dO| <= 2^-4 (P |V|)_d [normal range] + m_tiny max|V| [keys whose 2^7 P falls below e4m3's
+normal range, at most their whole mass m_tiny, taken as the keys more than 11.25 below the
+row maximum in log2 units: 7 + 1.75 headroom + 2.5 of the subnormal range] + 2^-8 |O| [bf16
+output] + 2^-14; the mean error must stay well inside the mean band. LSE: fp32 sums of the
+same scores, |dLSE| <= 2e-3 + 1e-5 |LSE|.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import veda_oracle as O
+import parity as P
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from block_sparse_attention_max_b200 import build
+    build.build()
+    V = P.veda()
+    V.lib()
+    yield
+    V.check_device_status()
+
+
+def _oracle_lists(gl, heads):
+    fc, fi = gl.full_cnt.cpu().numpy(), gl.full_idx.cpu().numpy()
+    pc, pi = gl.part_cnt.cpu().numpy(), gl.part_idx.cpu().numpy()
+    B, _, nT = fc.shape
+    full = [[[fi[b, h, r, :fc[b, h, r]].astype(np.int64) for r in range(nT)] for h in heads] for b in range(B)]
+    part = [[[pi[b, h, r, :pc[b, h, r]].astype(np.int64) for r in range(nT)] for h in heads] for b in range(B)]
+    return O.BlockLists(full, part)
+
+
+def _tiny_mass(qd, kd, nv, lists, rows, scale):
+    """Per checked row: attention mass of the keys more than 11.25 (log2 units) below the
+    row's maximum score."""
+    out = {}
+    for (b, j, r) in rows:
+        keys = np.sort(np.concatenate([lists.full[b][j][r], lists.partial[b][j][r]])).astype(np.int64)
+        if len(keys) == 0:
+            continue
+        idx = np.concatenate([np.arange(t * 128, t * 128 + int(nv[j][t])) for t in keys])
+        x = (qd[b, j, r * 128:(r + 1) * 128] @ kd[b, j, idx].T) * scale * math.log2(math.e)
+        xm = x.max(axis=1, keepdims=True)
+        w = np.exp2(x - xm)
+        w /= w.sum(axis=1, keepdims=True)
+        out[(b, j, r)] = (w * (x < xm - 11.25)).sum(axis=1)
+    return out
+
+
+def _run(w, heads, rows=None):
+    V = P.veda()
+    inp = synth.make_inputs(w)
+    orders = inp.tile_order
+    slots, nv, seg, nTh = P.oracle_maps(w, orders)
+    maps = V.build_tile_map(w.grid, w.head_shapes, w.n_tail, orders).to(DEV)
+    q_d, k_d, v_d, wq, wk = (t.to(DEV) for t in (inp.q, inp.k, inp.v, inp.wq, inp.wk))
+    bufs = V.sparse_attention(q_d, k_d, v_d, wq, wk, maps, w.rho, P.SCALE)
+    q8, sq = V.quantize_fp8(bufs.q_t)
+    k8, sk = V.quantize_fp8(bufs.k_t)
+    vt8, sv = V.quantize_fp8(bufs.v_t, transpose_tiles=True)
+    o8, lse8 = V.block_sparse_attn_fwd_fp8(q8, k8, vt8, sq, sk, sv, maps, bufs.lists, P.SCALE)
+    V.check_device_status()
+
+    # quantisation, bit for bit, on the checked heads
+    qt = O.permute(P.f64(inp.q[:, :, heads]), slots[heads])
+    kt = O.permute(P.f64(inp.k[:, :, heads]), slots[heads])
+    vt = O.permute(P.f64(inp.v[:, :, heads]), slots[heads])
+    cq, s_q = O.quantize_fp8(qt)
+    ck, s_k = O.quantize_fp8(kt)
+    cv, s_v = O.quantize_fp8(vt, transpose_tiles=True)
+    for got, ref, n in ((q8, cq, "q"), (k8, ck, "k"), (vt8, cv, "v")):
+        g = got[:, heads].cpu().numpy()
+        assert np.array_equal(g, ref), f"{n} codes differ at {int((g != ref).sum())} of {ref.size}"
+    for got, ref, n in ((sq, s_q, "q"), (sk, s_k, "k"), (sv, s_v, "v")):
+        assert np.array_equal(got[:, heads].cpu().numpy(), ref), f"{n} scales differ"
+
+    # attention of the dequantised tensors
+    B = w.B
+    qd, kd, vd = O.dequantize_fp8(cq, s_q), O.dequantize_fp8(ck, s_k), O.dequantize_fp8(cv, s_v, True)
+    lists_h = _oracle_lists(bufs.lists, heads)
+    todo = [(b, j, r) for b in range(B) for j, h in enumerate(heads)
+            for r in (range(nTh[h]) if rows is None else [x for x in rows if x < nTh[h]])]
+    o_ref, lse_ref = O.attention(qd, kd, vd, nv[heads], lists_h, P.SCALE, rows=todo)
+    o_abs, _ = O.attention(qd, kd, np.abs(vd), nv[heads], lists_h, P.SCALE, rows=todo)
+    tiny = _tiny_mass(qd, kd, nv[heads], lists_h, todo, P.SCALE)
+    og, lg = P.f64(o8[:, heads]), P.f64(lse8[:, heads])
+    errs, bands = [], []
+    for (b, j, r) in todo:
+        sl = slice(r * 128, (r + 1) * 128)
+        vmax = np.abs(vd[b, j]).max()
+        band = (2.0 ** -4 * o_abs[b, j, sl] + tiny[(b, j, r)][:, None] * vmax
+                + 2.0 ** -8 * np.abs(o_ref[b, j, sl]) + 2.0 ** -14)
+        err = np.abs(og[b, j, sl] - o_ref[b, j, sl])
+        assert np.all(err <= band), f"b{b} h{heads[j]} tile {r}: max err {err.max():.3g}, band {band.min():.3g}"
+        errs.append(err.ravel())
+        bands.append(band.ravel())
+        dl = np.abs(lg[b, j, sl] - lse_ref[b, j, sl])
+        assert np.all(dl <= 2e-3 + 1e-5 * np.abs(lse_ref[b, j, sl])), f"LSE differs by {dl.max():.3g}"
+    e, bd = np.concatenate(errs), np.concatenate(bands)
+    assert e.mean() <= 0.5 * bd.mean(), (e.mean(), bd.mean())
+    return float(e.max()), float(e.mean())
+
+
+def test_fp8_tiny():
+    _run(synth.TINY, [0, 1])
+
+
+def test_fp8_small():
+    _run(synth.SMALL, [0, 5])
+
+
+def test_fp8_mixed_shapes_tail_and_segments():
+    _run(synth.MIXED, [0, 17], rows=[0, 1, 100, 223, 224, 228])
+
+
+def test_fp8_ragged_heads_batch_and_empty_rows():
+    w = synth.Workload("ragged", 9, B=2, H=3, grid=(5, 8, 16),
+                       head_shapes=((1, 8, 16), (2, 8, 8), (4, 4, 8)), n_tail=0,
+                       rho=((1, 2),), field="smooth")
+    _run(w, [0, 1, 2])
