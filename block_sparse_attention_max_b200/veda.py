@@ -565,3 +565,65 @@ def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, wq: torc
                           bufs.lse, stream=stream)
     unpermute(bufs.o_t, maps, N, bufs.o, stream)
     return bufs
+
+
+class HostPipeline:
+    """Clips from pinned host memory through the whole path, one clip per ``submit``.
+
+    Three CUDA streams overlap the host-to-device copy of clip i + 1, the six steps of clip i
+    and the device-to-host copy of clip i - 1's output (the host link carries both directions
+    at once). Device copies of the raster inputs and of the raster output are kept per slot
+    (``depth`` slots); CUDA events order every reuse of a slot after the work that last read
+    it, so a clip's result does not depend on its neighbours. ``synchronize`` waits for every
+    submitted clip's output to be in its host tensor.
+    """
+
+    def __init__(self, B: int, N: int, H: int, maps: DeviceMaps, rho: Sequence[Tuple[int, int]],
+                 scale: float, device, depth: int = 2):
+        if depth < 1:
+            raise ValueError("depth must be >= 1")
+        self.maps, self.rho, self.scale, self.depth = maps, list(rho), float(scale), depth
+        bf = dict(dtype=torch.bfloat16, device=device)
+        f32 = dict(dtype=torch.float32, device=device)
+        self.inputs = [dict(q=torch.empty((B, N, H, 128), **bf), k=torch.empty((B, N, H, 128), **bf),
+                            v=torch.empty((B, N, H, 128), **bf), wq=torch.empty((H, 128, 384), **f32),
+                            wk=torch.empty((H, 128, 384), **f32)) for _ in range(depth)]
+        self.outputs = [torch.empty((B, N, H, 128), **bf) for _ in range(depth)]
+        self.bufs = PathBuffers.allocate(B, N, H, maps, rho, device)
+        self.h2d, self.comp, self.d2h = (torch.cuda.Stream(device) for _ in range(3))
+        ev = lambda: [torch.cuda.Event() for _ in range(depth)]
+        self.in_ready, self.in_free, self.out_ready, self.out_free = ev(), ev(), ev(), ev()
+        self.n = 0
+
+    def submit(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, wq: torch.Tensor, wk: torch.Tensor,
+               out: torch.Tensor) -> None:
+        """Enqueue one clip: q / k / v [B, N, H, 128] bf16, wq / wk [H, 128, 384] fp32 and the
+        output out [B, N, H, 128] bf16, all pinned host tensors; returns at once."""
+        s = self.n % self.depth
+        reuse = self.n >= self.depth
+        slot = self.inputs[s]
+        # inputs of slot s: after the clip that last used them has been computed
+        if reuse:
+            self.h2d.wait_event(self.in_free[s])
+        with torch.cuda.stream(self.h2d):
+            for name, src in (("q", q), ("k", k), ("v", v), ("wq", wq), ("wk", wk)):
+                slot[name].copy_(src, non_blocking=True)
+            self.in_ready[s].record(self.h2d)
+        # the six steps, into output slot s once its previous contents have left the device
+        self.comp.wait_event(self.in_ready[s])
+        if reuse:
+            self.comp.wait_event(self.out_free[s])
+        bufs = dataclasses.replace(self.bufs, o=self.outputs[s])
+        sparse_attention(slot["q"], slot["k"], slot["v"], slot["wq"], slot["wk"], self.maps, self.rho,
+                         self.scale, buffers=bufs, stream=self.comp)
+        self.in_free[s].record(self.comp)
+        self.out_ready[s].record(self.comp)
+        # the output of slot s to the host
+        self.d2h.wait_event(self.out_ready[s])
+        with torch.cuda.stream(self.d2h):
+            out.copy_(self.outputs[s], non_blocking=True)
+            self.out_free[s].record(self.d2h)
+        self.n += 1
+
+    def synchronize(self) -> None:
+        self.d2h.synchronize()

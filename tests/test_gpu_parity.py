@@ -251,6 +251,34 @@ def _end_to_end(w, heads=None, rows=None, attn_rows=None):
     return dict(lists_fp64_mismatch=bad64, total=total)
 
 
+def test_host_pipeline_matches_separate_calls():
+    """Three different clips through the HostPipeline (two slots, so one is reused while its
+    neighbour is in flight) give the outputs of separate sparse_attention calls bit for bit."""
+    V = P.veda()
+    w = synth.SMALL
+    inp = synth.make_inputs(w)
+    maps = V.build_tile_map(w.grid, w.head_shapes, w.n_tail, inp.tile_order).to(DEV)
+    g = torch.Generator().manual_seed(77)
+    clips = []
+    for i in range(3):
+        q = (inp.q.float() * (1.0 + 0.5 * i)).to(torch.bfloat16)
+        k = (inp.k.float() + 0.1 * i).to(torch.bfloat16)
+        v = torch.randn(inp.v.shape, generator=g).to(torch.bfloat16)
+        clips.append((q, k, v))
+    B, N, H, D = inp.q.shape
+    pipe = V.HostPipeline(B, N, H, maps, w.rho, P.SCALE, torch.device(DEV), depth=2)
+    outs = [torch.empty((B, N, H, D), dtype=torch.bfloat16).pin_memory() for _ in clips]
+    wq, wk = inp.wq.pin_memory(), inp.wk.pin_memory()
+    for (q, k, v), o in zip(clips, outs):
+        pipe.submit(q.pin_memory(), k.pin_memory(), v.pin_memory(), wq, wk, o)
+    pipe.synchronize()
+    V.check_device_status()
+    for (q, k, v), o in zip(clips, outs):
+        ref = V.sparse_attention(q.to(DEV), k.to(DEV), v.to(DEV), inp.wq.to(DEV), inp.wk.to(DEV), maps,
+                                 w.rho, P.SCALE)
+        assert torch.equal(o, ref.o.cpu())
+
+
 def test_end_to_end_tiny():
     _end_to_end(synth.TINY)
 
