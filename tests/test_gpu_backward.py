@@ -165,3 +165,9 @@ def test_backward_ragged_heads_batch_and_empty_rows():
                        head_shapes=((1, 8, 16), (2, 8, 8), (4, 4, 8)), n_tail=0,
                        rho=((1, 2),), field="smooth")
     _run(w, [0, 1, 2])
+
+
+def test_backward_clip16x9_one_head():
+    """The 16:9 clip at full size (40 heads launched, the benchmark's configuration), every
+    transposed list checked, the gradients of head 0 against the oracle over all its rows."""
+    _run(synth.CLIP16x9, [0])

@@ -135,3 +135,9 @@ def test_fp8_ragged_heads_batch_and_empty_rows():
                        head_shapes=((1, 8, 16), (2, 8, 8), (4, 4, 8)), n_tail=0,
                        rho=((1, 2),), field="smooth")
     _run(w, [0, 1, 2])
+
+
+def test_fp8_clip16x9_sampled():
+    """The 16:9 clip at full size (40 heads launched, the benchmark's configuration): codes and
+    scales of two heads bit-exact, attention of three query tiles of each against the oracle."""
+    _run(synth.CLIP16x9, [0, 39], rows=[0, 247, 495])
