@@ -403,24 +403,34 @@ def workload(args) -> synth.Workload:
 def _oracle_sample(inp, heads, rows_per_head):
     """The oracle's six steps on some heads of the workload, attention on some query tiles.
 
-    Returns (visited-block FLOPs processed, seconds)."""
+    Returns (visited-block FLOPs processed, seconds, seconds per step)."""
     from oracle import veda_oracle as O
     w = WORKLOAD
     t0 = time.perf_counter()
+    marks = []
     f = lambda t: t[:, :, heads].double().numpy()
     q, k, v = f(inp.q), f(inp.k), f(inp.v)
     maps = [O.tile_map(w.grid, w.head_shapes[h], w.n_tail) for h in heads]
     slots, nv, seg = O.stack_maps(maps, w.nT)
+    marks.append(time.perf_counter())
     qt, kt, vt = O.permute(q, slots), O.permute(k, slots), O.permute(v, slots)
+    marks.append(time.perf_counter())
     pq, pk = O.pool(qt, nv), O.pool(kt, nv)
+    marks.append(time.perf_counter())
     S = O.scores(pq, pk, inp.wq[heads].double().numpy(), inp.wk[heads].double().numpy())
+    marks.append(time.perf_counter())
     lists = O.select(S, nv, seg, [len(m.n_valid) for m in maps], w.rho)
+    marks.append(time.perf_counter())
     rows = [(0, j, r) for j in range(len(heads)) for r in range(rows_per_head)]
     o_t, _ = O.attention(qt, kt, vt, nv, lists, SCALE, rows=rows)
+    marks.append(time.perf_counter())
     O.unpermute(np.nan_to_num(o_t), slots, w.N)
-    dt = time.perf_counter() - t0
+    marks.append(time.perf_counter())
+    dt = marks[-1] - t0
+    names = ["permute_qkv", "pool_qk", "scores", "select", "attention", "unpermute"]
+    stage_s = {n: marks[i + 1] - marks[i] for i, n in enumerate(names)}
     blocks = sum(len(lists.full[0][j][r]) + len(lists.partial[0][j][r]) for (_, j, r) in rows)
-    return blocks * FLOP_PER_BLOCK, dt
+    return blocks * FLOP_PER_BLOCK, dt, stage_s
 
 
 def _cores():
@@ -435,8 +445,8 @@ def _cores():
 def cpu_baseline(seconds: float, inp):
     # whole path on heads 0.., attention on as many query tiles as fit the time budget
     # (calibrated: fixed cost of the non-attention steps + cost per attention query tile)
-    _, t8 = _oracle_sample(inp, [0], 8)
-    _, t24 = _oracle_sample(inp, [0], 24)
+    _, t8, _ = _oracle_sample(inp, [0], 8)
+    _, t24, _ = _oracle_sample(inp, [0], 24)
     per_row = max((t24 - t8) / 16, 1e-4)
     fixed = max(t8 - 8 * per_row, 0.0)
     heads = [0]
@@ -445,10 +455,11 @@ def cpu_baseline(seconds: float, inp):
         heads.append(len(heads))
         rows = int((seconds - fixed * len(heads)) / per_row)
     rows = max(16, min(WORKLOAD.nT, rows // len(heads)))
-    flop, dt = _oracle_sample(inp, heads, rows)
+    flop, dt, stage_s = _oracle_sample(inp, heads, rows)
     return {"value": flop / dt / 1e12, "unit": UNIT, "cores": _cores(), "kind": "oracle",
             "sample": f"fp64 oracle, all six steps on {len(heads)} of 40 heads, attention on {rows} of 496 "
-                      f"query tiles per head ({dt:.1f} s); value = visited-block FLOPs / CPU time"}
+                      f"query tiles per head ({dt:.1f} s); value = visited-block FLOPs / CPU time",
+            "stage_s": stage_s}
 
 
 def run_reference(args):
@@ -461,10 +472,13 @@ def run_reference(args):
     for _ in range(args.warmup):
         _oracle_sample(inp, [0], max(1, rows // 4))
     flops, secs = 0, 0.0
+    stage_s = {}
     for _ in range(args.steps):
-        f, dt = _oracle_sample(inp, [0], rows)
+        f, dt, st = _oracle_sample(inp, [0], rows)
         flops += f
         secs += dt
+        for n, x in st.items():
+            stage_s[n] = stage_s.get(n, 0.0) + x / args.steps
     value = flops / secs / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -476,7 +490,7 @@ def run_reference(args):
                    "parallelism": "cpu"},
         "cpu_baseline": {"kind": "oracle", "cores": _cores(), "value": value, "unit": UNIT,
                          "sample": f"each step: fp64 oracle, all six steps on head 0 of 40, "
-                                   f"attention on {rows} of 496 query tiles"},
+                                   f"attention on {rows} of 496 query tiles", "stage_s": stage_s},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
