@@ -141,3 +141,22 @@ def test_fp8_clip16x9_sampled():
     """The 16:9 clip at full size (40 heads launched, the benchmark's configuration): codes and
     scales of two heads bit-exact, attention of three query tiles of each against the oracle."""
     _run(synth.CLIP16x9, [0, 39], rows=[0, 247, 495])
+
+
+def test_quantize_zero_tensor_negative_zero_and_large_values():
+    """An all-zero (batch, head) tensor (scale 1, codes 0), negative zeros (sign bit kept) and a
+    head scaled by 1000, in both layouts: bit for bit against the oracle."""
+    V = P.veda()
+    g = torch.Generator().manual_seed(2303)
+    x = torch.randn((2, 3, 512, 128), generator=g)
+    x[0, 1] = 0.0
+    x[1, 0] *= 1000.0
+    x[1, 2, :5] = -0.0
+    x = x.to(torch.bfloat16)
+    for tr in (False, True):
+        codes, scale = V.quantize_fp8(x.to(DEV), transpose_tiles=tr)
+        V.check_device_status()
+        c_o, s_o = O.quantize_fp8(P.f64(x), transpose_tiles=tr)
+        assert np.array_equal(scale.cpu().numpy(), s_o)
+        assert np.array_equal(codes.cpu().numpy(), c_o), int((codes.cpu().numpy() != c_o).sum())
+        assert scale[0, 1].item() == 1.0 and not codes[0, 1].any()
