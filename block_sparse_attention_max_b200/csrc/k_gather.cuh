@@ -26,12 +26,15 @@ struct GatherArgs {
   int64_t units;         // B * H * nT
 };
 
+// Units in head-minor order (b, t, h): the CTAs running at one time take the same tile of
+// many heads, so together they read (permute) or write (unpermute) whole raster token rows
+// of H * 256 bytes instead of one head's 256 bytes out of each.
 __device__ __forceinline__ void unit_coords(int64_t u, int32_t H, int32_t nT, int32_t& b,
                                             int32_t& h, int32_t& t) {
-  t = static_cast<int32_t>(u % nT);
-  const int64_t bh = u / nT;
-  h = static_cast<int32_t>(bh % H);
-  b = static_cast<int32_t>(bh / H);
+  h = static_cast<int32_t>(u % H);
+  const int64_t bt = u / H;
+  t = static_cast<int32_t>(bt % nT);
+  b = static_cast<int32_t>(bt / nT);
 }
 
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
@@ -123,9 +126,10 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolArgs a) {
        u += warps) {
     int32_t b, h, t;
     unit_coords(u, a.H, a.nT, b, h, t);
+    const int64_t lin = (static_cast<int64_t>(b) * a.H + h) * a.nT + t;   // tile index in memory
     int32_t nv = a.valid[static_cast<int64_t>(h) * a.nT + t];
     nv = nv < 0 ? 0 : (nv > 128 ? 128 : nv);
-    const uint8_t* tile = a.x + static_cast<int64_t>(u) * kTileBytes + c * 16;
+    const uint8_t* tile = a.x + lin * kTileBytes + c * 16;
     float sum[8];
     __nv_bfloat162 mx[4], mn[4];
 #pragma unroll
@@ -172,7 +176,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolArgs a) {
       fmn[k] = fminf(fmn[k], __shfl_xor_sync(0xffffffffu, fmn[k], 16));
     }
     if (half == 0) {
-      float4* o = reinterpret_cast<float4*>(a.out + static_cast<int64_t>(u) * 384 + c * 8);
+      float4* o = reinterpret_cast<float4*>(a.out + lin * 384 + c * 8);
       if (nv > 0) {
         const float inv = 1.0f / static_cast<float>(nv);
         o[0] = make_float4(sum[0] * inv, sum[1] * inv, sum[2] * inv, sum[3] * inv);
@@ -209,6 +213,7 @@ __global__ void __launch_bounds__(kCopyThreads) permute_pool_kernel(const PermPo
   for (int64_t u = blockIdx.x; u < a.units; u += gridDim.x) {
     int32_t b, h, t;
     unit_coords(u, a.H, a.nT, b, h, t);
+    const int64_t lin = (static_cast<int64_t>(b) * a.H + h) * a.nT + t;   // tile index in memory
     int32_t nv = p.valid[static_cast<int64_t>(h) * a.nT + t];
     nv = nv < 0 ? 0 : (nv > 128 ? 128 : nv);
     const int32_t* m = a.map + static_cast<int64_t>(h) * a.Npad + static_cast<int64_t>(t) * 128;
@@ -269,7 +274,7 @@ __global__ void __launch_bounds__(kCopyThreads) permute_pool_kernel(const PermPo
         x_ = fmaxf(x_, red[w][1][ch]);
         n_ = fminf(n_, red[w][2][ch]);
       }
-      float* o = p.pooled + u * 384;
+      float* o = p.pooled + lin * 384;
       o[ch] = nv > 0 ? s_ / static_cast<float>(nv) : 0.f;
       o[128 + ch] = nv > 0 ? x_ : 0.f;
       o[256 + ch] = nv > 0 ? n_ : 0.f;
