@@ -49,15 +49,24 @@ __global__ void __launch_bounds__(kQuantThreads) amax_kernel(const QuantArgs q) 
     const int64_t end = per_bh < beg + kAmaxChunk ? per_bh : beg + kAmaxChunk;
     const uint4* src = reinterpret_cast<const uint4*>(q.x + b * per_bh);
     float m = 0.f;
-    for (int64_t i = beg / 8 + threadIdx.x; i < end / 8; i += blockDim.x) {
-      const uint4 v = src[i];
+    auto fold = [&](const uint4& v) {
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         m = fmaxf(m, __uint_as_float((w[k] << 16) & 0x7fffffffu));   // |low bf16| as fp32
         m = fmaxf(m, __uint_as_float(w[k] & 0x7fff0000u));           // |high bf16|
       }
+    };
+    int64_t i = beg / 8 + threadIdx.x;
+    // eight independent 16-byte loads in flight per thread, then the remainder
+    for (; i + 7 * kQuantThreads < end / 8; i += 8 * kQuantThreads) {
+      uint4 v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = src[i + k * kQuantThreads];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) fold(v[k]);
     }
+    for (; i < end / 8; i += kQuantThreads) fold(src[i]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
