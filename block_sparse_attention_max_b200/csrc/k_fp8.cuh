@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(kQuantThreads) amax_kernel(const QuantArgs q) 
 
 // e4m3 codes of one 128 x 128 tile per CTA iteration: thread (row r, half) converts 64
 // elements; with transpose the codes go through shared memory and leave as [channel][slot].
+// (kQuantThreads = 256: 128 rows x 2 halves, and 32 channel groups x 8 key groups.)
 __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const QuantArgs q) {
   __shared__ __align__(16) uint8_t tile[128][144];
   const int64_t tiles_per_bh = q.rows / 128;
@@ -114,18 +115,29 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const QuantArgs q)
 #pragma unroll
       for (int i = 0; i < 16; ++i) row[i] = out[i];
       __syncthreads();
-      // output row d = channel r of the tile: key slots half * 64 .. + 63
-      uint32_t o[16];
+      // thread (channel group cg, key group kg): channels 4 cg .. + 3 of key slots 16 kg .. + 15,
+      // read as 32-bit words (consecutive words across the warp) and transposed 4 x 4 bytes at
+      // a time in registers; output rows are channels, 16 key bytes each
+      const int cg = static_cast<int>(threadIdx.x & 31), kg = static_cast<int>(threadIdx.x >> 5);
+      uint32_t o[4][4];   // o[channel j][key word i]
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) w |= static_cast<uint32_t>(tile[half * 64 + 4 * i + k][r]) << (8 * k);
-        o[i] = w;
+      for (int i = 0; i < 4; ++i) {
+        const int k0 = 16 * kg + 4 * i;
+        const uint32_t a0 = *reinterpret_cast<const uint32_t*>(&tile[k0][4 * cg]);
+        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(&tile[k0 + 1][4 * cg]);
+        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(&tile[k0 + 2][4 * cg]);
+        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(&tile[k0 + 3][4 * cg]);
+        const uint32_t t0 = __byte_perm(a0, a1, 0x5140), t1 = __byte_perm(a2, a3, 0x5140);
+        const uint32_t t2 = __byte_perm(a0, a1, 0x7362), t3 = __byte_perm(a2, a3, 0x7362);
+        o[0][i] = __byte_perm(t0, t1, 0x5410);   // channel 4 cg: keys k0 .. k0 + 3
+        o[1][i] = __byte_perm(t0, t1, 0x7632);
+        o[2][i] = __byte_perm(t2, t3, 0x5410);
+        o[3][i] = __byte_perm(t2, t3, 0x7632);
       }
-      uint4* dst = reinterpret_cast<uint4*>(q.codes + (t * 128 + r) * 128 + half * 64);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(q.codes + (t * 128 + 4 * cg + j) * 128 + 16 * kg) =
+            make_uint4(o[j][0], o[j][1], o[j][2], o[j][3]);
       __syncthreads();
     }
   }
