@@ -41,13 +41,24 @@ using attn::kHalfB;
 
 constexpr int kModeDQ = 0;
 constexpr int kModeDKDV = 1;
-constexpr int kStrSt = 2;                       // streamed ring slots
-constexpr uint32_t kStatB = 1024;               // LSE + D rows of a streamed query tile (dK/dV)
-constexpr uint32_t kSlotB = 2 * kTileB + kStatB;
+// Streamed tiles in two rings: ring A holds the tile whose last reader is the block's late
+// accumulating MMA (dQ: K_j, read by dQ(j); dK/dV: Q_i, read by dK(j)), ring B the one whose
+// last reader comes early (dQ: V_j, read by dP(j); dK/dV: dO_i, read by dV(j)), so ring A
+// gets the extra slot: a slot is refilled only after its last reader, and a 32 KB tile
+// takes ~1,400 cycles to arrive from L2.
+constexpr int kStA = 3;                         // ring A slots
+constexpr int kStB = 2;                         // ring B slots
+constexpr int kStStat = 2;                      // dK/dV: LSE + D rows of the streamed query tiles
+constexpr uint32_t kStatB = 1024;
 constexpr uint32_t kOffFix = 0;                 // two fixed tiles
-constexpr uint32_t kOffStr = 2 * kTileB;        // ring of streamed slots
-constexpr uint32_t kSmemTiles = kOffStr + kStrSt * kSlotB;     // 194 KB
-constexpr uint32_t kSmemBytes = kSmemTiles + 1024;
+constexpr uint32_t kOffA = 2 * kTileB;
+constexpr uint32_t kOffB = kOffA + kStA * kTileB;
+constexpr uint32_t kOffStat = kOffB + kStB * kTileB;            // 224 KB
+// dQ: the tiles plus 1 KB of alignment slack; dK/dV: the tiles and the stats ring exactly
+// (226 KB, which with the static barriers is the 227 KB a block may have), so that kernel
+// checks that its dynamic shared memory starts 1024-byte aligned and does no work otherwise
+constexpr uint32_t kSmemBytesDQ = kOffStat + 1024;
+constexpr uint32_t kSmemBytesDKDV = kOffStat + kStStat * kStatB;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColDP = 128, kColA0 = 256, kColA1 = 384;
 constexpr uint32_t kColS1 = 384;                // dQ mode: second S buffer (acc1 unused)
@@ -77,7 +88,9 @@ struct Args {
 };
 
 struct Bars {
-  uint64_t fix_full, fix_empty, str_full[kStrSt], str_empty[kStrSt];
+  uint64_t fix_full, fix_empty;
+  uint64_t a_full[kStA], a_empty[kStA], b_full[kStB], b_empty[kStB];
+  uint64_t st_full[kStStat], st_empty[kStStat];
   uint64_t s_full[2];            // S-like MMA of block g landed (dQ: buffer g & 1; dK/dV: [0])
   uint64_t dp_full, dp_free;     // dP-like MMA landed / the softmax holds dP (dQ) in registers
   uint64_t pa_full;              // softmax wrote P^T over S^T (dK/dV)
@@ -92,7 +105,7 @@ struct Bars {
   // softmax warps through these records (-1 = no more work)
   uint64_t item_full[kItemRec], item_free[kItemRec];
   int32_t item_u[kItemRec];
-  uint32_t str_op[kStrSt];
+  uint32_t a_op[kStA];                 // block flags, written with the ring-A tile
   uint32_t tmem_base;
   int32_t abort;
 };
@@ -118,6 +131,7 @@ __device__ __forceinline__ void role_producer(const Args& a, Bars& bars, uint32_
                                               const CUtensorMap* tmF1, const CUtensorMap* tmS0,
                                               const CUtensorMap* tmS1, volatile int* abort) {
   uint32_t sc = 0, fc = 0;
+  uint32_t na = 0, nb = 0, ns = 0;   // copies issued into ring A, ring B and the stats ring
   bool stop = false;
   for (uint32_t ic = 0; !stop; ++ic) {
     const uint32_t is = ic % kItemRec;
@@ -146,27 +160,52 @@ __device__ __forceinline__ void role_producer(const Args& a, Bars& bars, uint32_
       if (b2) flag_status(ST_BAD_LIST);
       const int64_t t = head_row + idx;                 // streamed tile (b, h, idx)
       const int32_t srow = static_cast<int32_t>(t * 128);
-      const uint32_t ss = sc % kStrSt;
-      if (sc >= kStrSt && !mbar_wait(smem_u32(&bars.str_empty[ss]), (sc / kStrSt - 1) & 1, abort, 41)) {
+      // ring A: tile 0 of the block, plus its flags
+      const uint32_t sa = sc % kStA;
+      if (sc >= kStA && !mbar_wait(smem_u32(&bars.a_empty[sa]), (sc / kStA - 1) & 1, abort, 41)) {
         stop = true;
         break;
       }
-      bars.str_op[ss] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (fc == 0 ? kOpFirstItem : 0u);
-      const uint32_t slot = sb + kOffStr + ss * kSlotB;
-      const uint32_t sbar = smem_u32(&bars.str_full[ss]);
-      mbar_arrive_expect_tx(sbar, 2 * kTileB + (MODE == kModeDKDV ? kStatB : 0u));
-      tma_load_2d(slot, tmS0, sbar, 0, srow);
-      tma_load_2d(slot + kHalfB, tmS0, sbar, 64, srow);
-      tma_load_2d(slot + kTileB, tmS1, sbar, 0, srow);
-      tma_load_2d(slot + kTileB + kHalfB, tmS1, sbar, 64, srow);
+      bars.a_op[sa] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (fc == 0 ? kOpFirstItem : 0u);
+      {
+        const uint32_t dst = sb + kOffA + sa * kTileB;
+        const uint32_t bar = smem_u32(&bars.a_full[sa]);
+        mbar_arrive_expect_tx(bar, kTileB);
+        tma_load_2d(dst, tmS0, bar, 0, srow);
+        tma_load_2d(dst + kHalfB, tmS0, bar, 64, srow);
+        ++na;
+      }
+      // ring B: tile 1 of the block
+      const uint32_t sbb = sc % kStB;
+      if (sc >= kStB && !mbar_wait(smem_u32(&bars.b_empty[sbb]), (sc / kStB - 1) & 1, abort, 64)) {
+        stop = true;
+        break;
+      }
+      {
+        const uint32_t dst = sb + kOffB + sbb * kTileB;
+        const uint32_t bar = smem_u32(&bars.b_full[sbb]);
+        mbar_arrive_expect_tx(bar, kTileB);
+        tma_load_2d(dst, tmS1, bar, 0, srow);
+        tma_load_2d(dst + kHalfB, tmS1, bar, 64, srow);
+        ++nb;
+      }
       if (MODE == kModeDKDV) {
         // the streamed query tile's LSE and D rows (512 B each, 16-byte aligned)
-        bulk_g2s(slot + 2 * kTileB, a.lse + t * 128, 512, sbar);
-        bulk_g2s(slot + 2 * kTileB + 512, a.delta + t * 128, 512, sbar);
+        const uint32_t st = sc % kStStat;
+        if (sc >= kStStat && !mbar_wait(smem_u32(&bars.st_empty[st]), (sc / kStStat - 1) & 1, abort, 65)) {
+          stop = true;
+          break;
+        }
+        const uint32_t dst = sb + kOffStat + st * kStatB;
+        const uint32_t bar = smem_u32(&bars.st_full[st]);
+        mbar_arrive_expect_tx(bar, kStatB);
+        bulk_g2s(dst, a.lse + t * 128, 512, bar);
+        bulk_g2s(dst + 512, a.delta + t * 128, 512, bar);
+        ++ns;
       }
       if (MODE == kModeDQ) {
         // block record for the softmax: valid key slots of the streamed key tile (entry
-        // sc % kRec was last read for block sc - kRec, long before slot sc - kStrSt came back)
+        // sc % kRec was last read for block sc - kRec, long before ring-A slot sc - kStA came back)
         int32_t nv = valid_h[idx];
         if (nv < 0 || nv > 128) {
           flag_status(ST_BAD_LIST);
@@ -180,15 +219,20 @@ __device__ __forceinline__ void role_producer(const Args& a, Bars& bars, uint32_
     ++fc;
   }
   if (!*abort) {
-    const uint32_t ss = sc % kStrSt;
-    if (sc < kStrSt || mbar_wait(smem_u32(&bars.str_empty[ss]), (sc / kStrSt - 1) & 1, abort, 42)) {
-      bars.str_op[ss] = kOpStop;
-      mbar_arrive(smem_u32(&bars.str_full[ss]));
+    const uint32_t sa = sc % kStA;
+    if (sc < kStA || mbar_wait(smem_u32(&bars.a_empty[sa]), (sc / kStA - 1) & 1, abort, 42)) {
+      bars.a_op[sa] = kOpStop;
+      mbar_arrive(smem_u32(&bars.a_full[sa]));
     }
   }
   if (*abort) {
-    for (uint32_t i = sc > kStrSt ? sc - kStrSt : 0; i < sc; ++i)
-      mbar_wait(smem_u32(&bars.str_full[i % kStrSt]), (i / kStrSt) & 1, nullptr, 43);
+    // let the copies this thread issued land before the CTA exits, ring by ring
+    for (uint32_t i = na > kStA ? na - kStA : 0; i < na; ++i)
+      mbar_wait(smem_u32(&bars.a_full[i % kStA]), (i / kStA) & 1, nullptr, 43);
+    for (uint32_t i = nb > kStB ? nb - kStB : 0; i < nb; ++i)
+      mbar_wait(smem_u32(&bars.b_full[i % kStB]), (i / kStB) & 1, nullptr, 66);
+    for (uint32_t i = ns > kStStat ? ns - kStStat : 0; i < ns; ++i)
+      mbar_wait(smem_u32(&bars.st_full[i % kStStat]), (i / kStStat) & 1, nullptr, 67);
     if (fc > 0) mbar_wait(smem_u32(&bars.fix_full), (fc - 1) & 1, nullptr, 44);
   }
 }
@@ -213,27 +257,36 @@ __device__ __forceinline__ void mma_accum(uint32_t d, uint32_t a_tmem, uint64_t 
 template <int MODE>
 __device__ __forceinline__ void role_issuer(Bars& bars, uint32_t sb, uint32_t tmem, volatile int* abort) {
   const uint64_t dF = smem_desc_sw128(sb + kOffFix, 16, 1024);          // fixed tiles, K-major
-  const uint64_t dS = smem_desc_sw128(sb + kOffStr, 16, 1024);          // streamed tiles, K-major
-  const uint64_t dSm = smem_desc_sw128(sb + kOffStr, kHalfB, 1024);     // streamed tiles, MN-major
+  const uint64_t dA = smem_desc_sw128(sb + kOffA, 16, 1024);            // ring A, K-major
+  const uint64_t dAm = smem_desc_sw128(sb + kOffA, kHalfB, 1024);       // ring A, MN-major
+  const uint64_t dB = smem_desc_sw128(sb + kOffB, 16, 1024);            // ring B, K-major
+  const uint64_t dBm = smem_desc_sw128(sb + kOffB, kHalfB, 1024);       // ring B, MN-major
   const uint64_t fix1 = static_cast<uint64_t>(kTileB >> 4);
-  // S-like = F0 x S0^T of block g into its S buffer; dP-like = F1 x S1^T
-  auto slot = [](uint32_t g) { return static_cast<uint64_t>((g % kStrSt) * (kSlotB >> 4)); };
+  auto offA = [](uint32_t g) { return static_cast<uint64_t>((g % kStA) * (kTileB >> 4)); };
+  auto offB = [](uint32_t g) { return static_cast<uint64_t>((g % kStB) * (kTileB >> 4)); };
   auto s_col = [](uint32_t g) { return MODE == kModeDQ ? ((g & 1) ? kColS1 : kColS) : kColS; };
+  // S-like = F0 x (ring-A tile)^T of block g into its S buffer; dP-like = F1 x (ring-B tile)^T
   auto issue_s = [&](uint32_t g) {
-    mma_score(tmem + s_col(g), attn::opaque(dF), attn::opaque(dS + slot(g)));
+    mma_score(tmem + s_col(g), attn::opaque(dF), attn::opaque(dA + offA(g)));
     tc_commit(smem_u32(&bars.s_full[MODE == kModeDQ ? (g & 1) : 0]));
   };
   auto issue_dp = [&](uint32_t g) {
-    mma_score(tmem + kColDP, attn::opaque(dF + fix1), attn::opaque(dS + slot(g) + fix1));
+    mma_score(tmem + kColDP, attn::opaque(dF + fix1), attn::opaque(dB + offB(g)));
     tc_commit(smem_u32(&bars.dp_full));
+    if (MODE == kModeDQ) tc_commit(smem_u32(&bars.b_empty[g % kStB]));   // V_g: last reader
+  };
+  auto wait_a = [&](uint32_t g, uint32_t site) {
+    return mbar_wait(smem_u32(&bars.a_full[g % kStA]), (g / kStA) & 1, abort, site);
+  };
+  auto wait_b = [&](uint32_t g, uint32_t site) {
+    return mbar_wait(smem_u32(&bars.b_full[g % kStB]), (g / kStB) & 1, abort, site);
   };
   uint32_t fn = 0, items = 0;
   bool head = true;   // block g starts an item: its S / dP are not issued yet
   bool ok = true;
   for (uint32_t g = 0; ok; ++g) {
-    const uint32_t ss = g % kStrSt;
-    if (!mbar_wait(smem_u32(&bars.str_full[ss]), (g / kStrSt) & 1, abort, 45)) break;
-    const uint32_t op = bars.str_op[ss];
+    if (!wait_a(g, 45)) break;
+    const uint32_t op = bars.a_op[g % kStA];
     if (op & kOpStop) break;
     if (op & kOpNewItem) {
       if (!mbar_wait(smem_u32(&bars.fix_full), fn & 1, abort, 46)) break;
@@ -244,16 +297,16 @@ __device__ __forceinline__ void role_issuer(Bars& bars, uint32_t sb, uint32_t tm
     if (head) {
       // dQ: dP(g) overwrites dP(g - 1), which the softmax must hold in registers by now
       if (MODE == kModeDQ && g > 0 && !mbar_wait(smem_u32(&bars.dp_free), (g - 1) & 1, abort, 60)) break;
+      if (!wait_b(g, 68)) break;
       tc_fence_after();
       issue_s(g);
       issue_dp(g);
     }
     const uint32_t acc_first = (op & kOpNewItem) ? 0u : 1u;
     const bool need_o_free = (op & kOpNewItem) && !(op & kOpFirstItem);
-    // the next block of the item (its slot is the other ring slot, filled once the
-    // previous block's accumulating MMAs released it)
+    // both tiles of the next block of the item
     const uint32_t gn = g + 1;
-    if (!last && !mbar_wait(smem_u32(&bars.str_full[gn % kStrSt]), (gn / kStrSt) & 1, abort, 61)) break;
+    if (!last && (!wait_a(gn, 61) || !wait_b(gn, 69))) break;
     if (MODE == kModeDQ) {
       if (!last) {
         // S(g + 1) goes to the buffer of dS(g - 1), which dQ(g - 1), issued before, reads
@@ -263,26 +316,27 @@ __device__ __forceinline__ void role_issuer(Bars& bars, uint32_t sb, uint32_t tm
         tc_fence_after();
         issue_dp(gn);
       }
-      // dQ += dS (written over S(g)) x K_g (streamed tile 0, MN-major)
+      // dQ += dS (written over S(g)) x K_g (ring A, MN-major)
       if (!mbar_wait(smem_u32(&bars.pb_full[g & 1]), (g >> 1) & 1, abort, 47)) break;
       // the first accumulation of an item overwrites acc: the previous epilogue must be done
       if (need_o_free && !mbar_wait(smem_u32(&bars.o_free), (items - 1) & 1, abort, 48)) break;
       tc_fence_after();
-      mma_accum(tmem + kColA0, tmem + s_col(g), attn::opaque(dSm + slot(g)), acc_first);
-      tc_commit(smem_u32(&bars.str_empty[ss]));
+      mma_accum(tmem + kColA0, tmem + s_col(g), attn::opaque(dAm + offA(g)), acc_first);
+      tc_commit(smem_u32(&bars.a_empty[g % kStA]));                    // K_g: last reader
     } else {
-      // dV += P^T (written over S^T) x dO_g (streamed tile 1)
+      // dV += P^T (written over S^T) x dO_g (ring B)
       if (!mbar_wait(smem_u32(&bars.pa_full), g & 1, abort, 47)) break;
       if (need_o_free && !mbar_wait(smem_u32(&bars.o_free), (items - 1) & 1, abort, 48)) break;
       tc_fence_after();
-      mma_accum(tmem + kColA0, tmem + kColS, attn::opaque(dSm + slot(g) + fix1), acc_first);
+      mma_accum(tmem + kColA0, tmem + kColS, attn::opaque(dBm + offB(g)), acc_first);
+      tc_commit(smem_u32(&bars.b_empty[g % kStB]));                    // dO_g: last reader
       if (!last) issue_s(gn);    // S^T(g + 1) overwrites P^T(g) after dV(g) has read it
-      // dK += dS^T (written over dP^T) x Q_g (streamed tile 0)
+      // dK += dS^T (written over dP^T) x Q_g (ring A)
       if (!mbar_wait(smem_u32(&bars.pb_full[0]), g & 1, abort, 63)) break;
       tc_fence_after();
-      mma_accum(tmem + kColA1, tmem + kColDP, attn::opaque(dSm + slot(g)), acc_first);
+      mma_accum(tmem + kColA1, tmem + kColDP, attn::opaque(dAm + offA(g)), acc_first);
       if (!last) issue_dp(gn);   // dP^T(g + 1) overwrites dS^T(g) after dK(g) has read it
-      tc_commit(smem_u32(&bars.str_empty[ss]));
+      tc_commit(smem_u32(&bars.a_empty[g % kStA]));                    // Q_g: last reader
     }
     if (last) {
       tc_commit(smem_u32(&bars.fix_empty));
@@ -363,10 +417,11 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
         nv = reinterpret_cast<volatile int32_t*>(bars.rec_nv)[g % kRec];
       }
       if (MODE == kModeDKDV) {
-        // the LSE / D rows were written into the slot by the copy engine: observe the slot's
-        // own barrier (already complete) before reading them
-        const uint32_t ss = g % kStrSt;
-        if (!warp_wait_abort(smem_u32(&bars.str_full[ss]), (g / kStrSt) & 1, abort, 53)) { ok = false; break; }
+        // the LSE / D rows of the streamed query tile, written by the copy engine
+        if (!warp_wait_abort(smem_u32(&bars.st_full[g % kStStat]), (g / kStStat) & 1, abort, 53)) {
+          ok = false;
+          break;
+        }
       }
       // S of this block (dQ: buffer g & 1, one phase per use; dK/dV: one buffer)
       const uint32_t colS = MODE == kModeDQ ? ((g & 1) ? kColS1 : kColS) : kColS;
@@ -397,7 +452,7 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
           if (k >= kv1) { s[4 * k + 1] = 0xFF800000u; s[4 * k + 3] = 0xFF800000u; }
         }
       }
-      const uint32_t stat = sb + kOffStr + (g % kStrSt) * kSlotB + 2 * kTileB;   // dK/dV: LSE, D
+      const uint32_t stat = sb + kOffStat + (g % kStStat) * kStatB;   // dK/dV: LSE, D
       uint32_t pk[32];
       // P (in place of s), and for dK/dV P^T packed over S
 #pragma unroll
@@ -465,7 +520,10 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars.pb_full[MODE == kModeDQ ? (g & 1) : 0]));
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&bars.pb_full[MODE == kModeDQ ? (g & 1) : 0]));
+        if (MODE == kModeDKDV) mbar_arrive(smem_u32(&bars.st_empty[g % kStStat]));   // LSE / D read
+      }
     }
     if (!ok) break;
     // epilogue: acc0 (dQ or dV), acc1 (dK) -> bf16 rows; dQ and dK carry the softmax scale
@@ -511,12 +569,26 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmF0, const __grid_constant__ CUt
   const uint32_t sb = smem_u32(smem);
   const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2;
   volatile int* abort = &bars.abort;
+  // the dK/dV instance's shared memory has no alignment slack: it works only from a
+  // 1024-byte-aligned start (the same for every thread, so the whole CTA leaves together)
+  if (MODE == kModeDKDV && smem != smem_raw) {
+    if (tid == 0) flag_status(ST_SMEM_ALIGN);
+    return;
+  }
   if (tid == 0) {
     mbar_init(smem_u32(&bars.fix_full), 1);
     mbar_init(smem_u32(&bars.fix_empty), 1);
-    for (int i = 0; i < kStrSt; ++i) {
-      mbar_init(smem_u32(&bars.str_full[i]), 1);
-      mbar_init(smem_u32(&bars.str_empty[i]), 1);
+    for (int i = 0; i < kStA; ++i) {
+      mbar_init(smem_u32(&bars.a_full[i]), 1);
+      mbar_init(smem_u32(&bars.a_empty[i]), 1);
+    }
+    for (int i = 0; i < kStB; ++i) {
+      mbar_init(smem_u32(&bars.b_full[i]), 1);
+      mbar_init(smem_u32(&bars.b_empty[i]), 1);
+    }
+    for (int i = 0; i < kStStat; ++i) {
+      mbar_init(smem_u32(&bars.st_full[i]), 1);
+      mbar_init(smem_u32(&bars.st_empty[i]), 8);   // the eight softmax warps
     }
     mbar_init(smem_u32(&bars.s_full[0]), 1);
     mbar_init(smem_u32(&bars.s_full[1]), 1);

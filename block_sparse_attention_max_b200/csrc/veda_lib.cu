@@ -82,8 +82,8 @@ veda_status current_device(int& sms) {
         {reinterpret_cast<const void*>(attn::attn_fwd_kernel), static_cast<int>(attn::kSmemBytes)},
         {reinterpret_cast<const void*>(heat::heat_kernel), static_cast<int>(attn::kSmemBytes)},
         {reinterpret_cast<const void*>(fp8::attn_fwd_fp8_kernel), static_cast<int>(fp8::kSmemBytes)},
-        {reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDQ>), static_cast<int>(bwd::kSmemBytes)},
-        {reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDKDV>), static_cast<int>(bwd::kSmemBytes)},
+        {reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDQ>), static_cast<int>(bwd::kSmemBytesDQ)},
+        {reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDKDV>), static_cast<int>(bwd::kSmemBytesDKDV)},
     };
     for (auto& x : attrs) {
       e = cudaFuncSetAttribute(x.f, cudaFuncAttributeMaxDynamicSharedMemorySize, x.bytes);
@@ -636,7 +636,7 @@ veda_status veda_block_sparse_attn_bwd(const void* q, const void* k, const void*
   a.out0 = static_cast<__nv_bfloat16*>(dq);
   a.out1 = nullptr;
   const unsigned grid = grid_for(a.items, sms, 1);
-  bwd::bwd_kernel<bwd::kModeDQ><<<grid, bwd::kThreads, bwd::kSmemBytes, s>>>(tq, tdo, tk, tv, a);
+  bwd::bwd_kernel<bwd::kModeDQ><<<grid, bwd::kThreads, bwd::kSmemBytesDQ, s>>>(tq, tdo, tk, tv, a);
   if ((st = launched("bwd_kernel<dQ>")) != VEDA_OK) return st;
   // dK, dV: key tiles over the transposed lists (fixed K, V; streamed Q, dO)
   a.full_cnt = t_cnt; a.full_idx = t_idx; a.part_cnt = nullptr; a.part_idx = nullptr;
@@ -644,7 +644,7 @@ veda_status veda_block_sparse_attn_bwd(const void* q, const void* k, const void*
   a.out0 = static_cast<__nv_bfloat16*>(dv);
   a.out1 = static_cast<__nv_bfloat16*>(dk);
   a.next_item = counters + 1;
-  bwd::bwd_kernel<bwd::kModeDKDV><<<grid, bwd::kThreads, bwd::kSmemBytes, s>>>(tk, tv, tq, tdo, a);
+  bwd::bwd_kernel<bwd::kModeDKDV><<<grid, bwd::kThreads, bwd::kSmemBytesDKDV, s>>>(tk, tv, tq, tdo, a);
   return launched("bwd_kernel<dK,dV>");
 }
 

@@ -17,6 +17,7 @@ enum : uint32_t {
   ST_NAN_SCORE = 1u << 2,   // NaN score in the selection
   ST_BAD_LIST = 1u << 3,    // block list index / count out of range
   ST_LIST_OVERFLOW = 1u << 4,  // a row needed more than list_stride entries
+  ST_SMEM_ALIGN = 1u << 5,  // dynamic shared memory not 1024-byte aligned (the kernel did no work)
   ST_WAIT_SITE_SHIFT = 8,   // bits 8..15: site code of the first wait that ran out
 };
 
