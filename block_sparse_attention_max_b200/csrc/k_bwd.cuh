@@ -285,7 +285,9 @@ __device__ __forceinline__ void role_issuer(Bars& bars, uint32_t sb, uint32_t tm
   bool head = true;   // block g starts an item: its S / dP are not issued yet
   bool ok = true;
   for (uint32_t g = 0; ok; ++g) {
-    if (!wait_a(g, 45)) break;
+    // block g's ring-A phase was already observed before its look-ahead MMA unless it
+    // starts an item (or is the stop record, which follows an item's last block)
+    if (head && !wait_a(g, 45)) break;
     const uint32_t op = bars.a_op[g % kStA];
     if (op & kOpStop) break;
     if (op & kOpNewItem) {
@@ -304,15 +306,17 @@ __device__ __forceinline__ void role_issuer(Bars& bars, uint32_t sb, uint32_t tm
     }
     const uint32_t acc_first = (op & kOpNewItem) ? 0u : 1u;
     const bool need_o_free = (op & kOpNewItem) && !(op & kOpFirstItem);
-    // both tiles of the next block of the item
+    // the next block of the item: each of its tiles is waited for just before the MMA that
+    // reads it, so that a wait overlaps MMAs already queued on the tensor core
     const uint32_t gn = g + 1;
-    if (!last && (!wait_a(gn, 61) || !wait_b(gn, 69))) break;
     if (MODE == kModeDQ) {
       if (!last) {
         // S(g + 1) goes to the buffer of dS(g - 1), which dQ(g - 1), issued before, reads
+        if (!wait_a(gn, 61)) break;
+        tc_fence_after();
         issue_s(gn);
         // dP(g + 1) overwrites dP(g) once the softmax holds it in registers
-        if (!mbar_wait(smem_u32(&bars.dp_free), g & 1, abort, 62)) break;
+        if (!mbar_wait(smem_u32(&bars.dp_free), g & 1, abort, 62) || !wait_b(gn, 69)) break;
         tc_fence_after();
         issue_dp(gn);
       }
@@ -330,12 +334,22 @@ __device__ __forceinline__ void role_issuer(Bars& bars, uint32_t sb, uint32_t tm
       tc_fence_after();
       mma_accum(tmem + kColA0, tmem + kColS, attn::opaque(dBm + offB(g)), acc_first);
       tc_commit(smem_u32(&bars.b_empty[g % kStB]));                    // dO_g: last reader
-      if (!last) issue_s(gn);    // S^T(g + 1) overwrites P^T(g) after dV(g) has read it
+      if (!last) {
+        // S^T(g + 1) overwrites P^T(g) after dV(g) has read it
+        if (!wait_a(gn, 61)) break;
+        tc_fence_after();
+        issue_s(gn);
+      }
       // dK += dS^T (written over dP^T) x Q_g (ring A)
       if (!mbar_wait(smem_u32(&bars.pb_full[0]), g & 1, abort, 63)) break;
       tc_fence_after();
       mma_accum(tmem + kColA1, tmem + kColDP, attn::opaque(dAm + offA(g)), acc_first);
-      if (!last) issue_dp(gn);   // dP^T(g + 1) overwrites dS^T(g) after dK(g) has read it
+      if (!last) {
+        // dP^T(g + 1) overwrites dS^T(g) after dK(g) has read it
+        if (!wait_b(gn, 69)) break;
+        tc_fence_after();
+        issue_dp(gn);
+      }
       tc_commit(smem_u32(&bars.a_empty[g % kStA]));                    // Q_g: last reader
     }
     if (last) {
