@@ -30,8 +30,81 @@ struct HeatArgs {
 constexpr uint32_t kTmemCols = 256;   // S0 | S1
 constexpr float kLog2e = 1.4426950408889634f;
 
-// The eight softmax warps: warp w owns tile rows 32 (w % 4) + 16 (w / 4) + [0, 16); a thread
-// holds rows r0 and r0 + 8 and 32 scores of each (16x256b shape, as in the forward kernel).
+// Loads S of blocks g .. g + NB - 1 (handing each TMEM buffer back as soon as it is in
+// registers), then computes their probabilities in one loop, so the exponentials of the NB
+// blocks run back to back and the per-block waits, hand-backs and reductions are paid once
+// per group. A thread holds rows r0 and r0 + 8 and 32 scores of each per block (16x256b
+// shape, as in the forward kernel). Returns false when a wait gave up.
+template <int NB>
+__device__ __forceinline__ bool heat_group(attn::Bars& bars, uint32_t tmem, uint32_t lane_off, uint32_t c,
+                                           uint32_t lane, uint32_t g, uint64_t c2, uint64_t nlx0, uint64_t nlx1,
+                                           float inv_nq, float* heat_row, volatile int* abort) {
+  using namespace attn;
+  uint32_t s[NB][64];
+  int32_t key[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    const uint32_t gb = g + b, sbuf = gb & 1;
+    if (!warp_wait_abort(smem_u32(&bars.rec_full[gb % kRec]), (gb / kRec) & 1, abort, 36)) return false;
+    const int32_t nv = reinterpret_cast<volatile int32_t*>(bars.rec_nv)[gb % kRec];
+    key[b] = reinterpret_cast<volatile int32_t*>(bars.rec_idx)[gb % kRec];
+    if (!warp_wait_abort(smem_u32(&bars.s_full[sbuf]), (gb >> 1) & 1, abort, 30)) return false;
+    tc_fence_after();
+    tmem_ld_16x256b_x16(tmem + lane_off + kColS + sbuf * 128, s[b]);
+    tmem_wait_ld();
+    reg_fence(s[b]);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars.s_free[sbuf]));
+    if (nv < 128) {
+      // column 8k + 2c + e is a key slot < nv exactly for k < ceil((nv - 2c - e) / 8)
+      const int32_t kv0 = (nv - 2 * static_cast<int32_t>(c) + 7) >> 3;
+      const int32_t kv1 = (nv - 2 * static_cast<int32_t>(c) + 6) >> 3;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        if (k >= kv0) { s[b][4 * k] = 0xFF800000u; s[b][4 * k + 2] = 0xFF800000u; }   // -inf
+        if (k >= kv1) { s[b][4 * k + 1] = 0xFF800000u; s[b][4 * k + 3] = 0xFF800000u; }
+      }
+    }
+  }
+  uint64_t acc[NB][2];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) acc[b][0] = acc[b][1] = 0ull;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      float x0, x1, y0, y1;
+      f2_unpack(f2_fma(f2_pack(s[b][4 * k], s[b][4 * k + 1]), c2, nlx0), x0, x1);
+      f2_unpack(f2_fma(f2_pack(s[b][4 * k + 2], s[b][4 * k + 3]), c2, nlx1), y0, y1);
+      const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), q0 = ex2_approx(y0), q1 = ex2_approx(y1);
+      acc[b][k & 1] = f2_add(acc[b][k & 1], f2_add(f2_pack(__float_as_uint(p0), __float_as_uint(p1)),
+                                                   f2_pack(__float_as_uint(q0), __float_as_uint(q1))));
+    }
+  }
+  float t[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    float t0, t1, t2, t3;
+    f2_unpack(acc[b][0], t0, t1);
+    f2_unpack(acc[b][1], t2, t3);
+    t[b] = (t0 + t1) + (t2 + t3);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+    for (int b = 0; b < NB; ++b) t[b] += __shfl_xor_sync(0xffffffffu, t[b], o);
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int b = 0; b < NB; ++b) atomicAdd(heat_row + key[b], t[b] * inv_nq);
+  }
+  return true;
+}
+
+// The eight softmax warps: warp w owns tile rows 32 (w % 4) + 16 (w / 4) + [0, 16) of every
+// block and takes an item's blocks two at a time (the last one alone when the item has an odd
+// count).
 __device__ __forceinline__ void heat_softmax(const HeatArgs& p, attn::Bars& bars, uint32_t tmem, uint32_t warp,
                                              uint32_t lane) {
   using namespace attn;
@@ -63,47 +136,12 @@ __device__ __forceinline__ void heat_softmax(const HeatArgs& p, attn::Bars& bars
     const float inv_nq = nq > 0 ? 1.0f / static_cast<float>(nq) : 0.f;
     float* heat_row = p.heat + u * a.nT;
     bool ok = true;
-    for (int32_t j = 0; j < n; ++j, ++g) {
-      const uint32_t sbuf = g & 1;
-      if (!warp_wait_abort(smem_u32(&bars.rec_full[g % kRec]), (g / kRec) & 1, abort, 36)) { ok = false; break; }
-      const int32_t nv = reinterpret_cast<volatile int32_t*>(bars.rec_nv)[g % kRec];
-      const int32_t key = reinterpret_cast<volatile int32_t*>(bars.rec_idx)[g % kRec];
-      if (!warp_wait_abort(smem_u32(&bars.s_full[sbuf]), (g >> 1) & 1, abort, 30)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t s[64];
-      tmem_ld_16x256b_x16(tmem + lane_off + kColS + sbuf * 128, s);
-      tmem_wait_ld();
-      reg_fence(s);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars.s_free[sbuf]));
-      if (nv < 128) {
-        // column 8k + 2c + e is a key slot < nv exactly for k < ceil((nv - 2c - e) / 8)
-        const int32_t kv0 = (nv - 2 * static_cast<int32_t>(c) + 7) >> 3;
-        const int32_t kv1 = (nv - 2 * static_cast<int32_t>(c) + 6) >> 3;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          if (k >= kv0) { s[4 * k] = 0xFF800000u; s[4 * k + 2] = 0xFF800000u; }   // -inf
-          if (k >= kv1) { s[4 * k + 1] = 0xFF800000u; s[4 * k + 3] = 0xFF800000u; }
-        }
-      }
-      uint64_t acc[2] = {0ull, 0ull};
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        float x0, x1, y0, y1;
-        f2_unpack(f2_fma(f2_pack(s[4 * k], s[4 * k + 1]), c2, nlx0), x0, x1);
-        f2_unpack(f2_fma(f2_pack(s[4 * k + 2], s[4 * k + 3]), c2, nlx1), y0, y1);
-        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), q0 = ex2_approx(y0), q1 = ex2_approx(y1);
-        acc[k & 1] = f2_add(acc[k & 1], f2_add(f2_pack(__float_as_uint(p0), __float_as_uint(p1)),
-                                               f2_pack(__float_as_uint(q0), __float_as_uint(q1))));
-      }
-      float t0, t1, t2, t3;
-      f2_unpack(acc[0], t0, t1);
-      f2_unpack(acc[1], t2, t3);
-      float t = (t0 + t1) + (t2 + t3);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-      if (lane == 0) atomicAdd(heat_row + key, t * inv_nq);
+    int32_t j = 0;
+    for (; j + 2 <= n; j += 2, g += 2)
+      if (!heat_group<2>(bars, tmem, lane_off, c, lane, g, c2, nlx0, nlx1, inv_nq, heat_row, abort)) { ok = false; break; }
+    if (ok && j < n) {
+      ok = heat_group<1>(bars, tmem, lane_off, c, lane, g, c2, nlx0, nlx1, inv_nq, heat_row, abort);
+      ++g;
     }
     if (!ok) break;
   }
