@@ -6,14 +6,18 @@
 // (k_attn.cuh) over the same block lists, with:
 //   * one scale per (batch, head) tensor: scale = amax / 448, code = e4m3(x * 448 / amax),
 //     both in fp32, rounding to nearest even and saturating at +-448 (cvt.rn.satfinite);
-//     V is stored as transposed tiles ([channel][key slot]) so that both products take
-//     K-major operands;
+//     V is stored as transposed tiles ([channel][key position]) so that both products take
+//     K-major operands, with the keys of every group of 16 in the order the softmax packs P
+//     (position 16m + 4c + e holds key slot 16m + 2c + (e & 1) + 8 (e >> 1));
 //   * S = Q K^T from e4m3 operands (kind::f8f6f4, K = 32 per MMA), scaled by
 //     q_scale * k_scale * softmax_scale in the softmax;
+//   * every role visits an item's diagonal key tile first (it holds most rows' maxima), then
+//     the rest of the list in order;
 //   * P = 2^(s - m + 7) in e4m3 (the reference m moves when a row maximum grows by more
 //     than 1.75, so P stays below 2^8.75 = 430 < 448), written by the softmax warps into
-//     shared memory in the 128-byte-swizzled K-major layout the MMA reads; O += P V with V
-//     read from its transposed tile, O = O_acc * v_scale / l in the epilogue.
+//     tensor memory (four keys per 32-bit column, in the order above); O += P V with P read
+//     from tensor memory and V from its transposed tile, O = O_acc * v_scale / l in the
+//     epilogue.
 // Roles, rings, barriers and bounded waits are those of the bf16 kernel (attn::Bars).
 #pragma once
 
@@ -81,7 +85,9 @@ __global__ void __launch_bounds__(kQuantThreads) amax_kernel(const QuantArgs q) 
 }
 
 // e4m3 codes of one 128 x 128 tile per CTA iteration: thread (row r, half) converts 64
-// elements; with transpose the codes go through shared memory and leave as [channel][slot].
+// elements; with transpose the codes go through shared memory and leave as [channel][key
+// position], position 16m + 4c + e of a row holding key slot 16m + 2c + (e & 1) + 8 (e >> 1)
+// (the order in which the attention's softmax packs P into tensor memory).
 // (kQuantThreads = 256: 128 rows x 2 halves, and 32 channel groups x 8 key groups.)
 __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const QuantArgs q) {
   __shared__ __align__(16) uint8_t tile[128][144];
@@ -117,19 +123,20 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const QuantArgs q)
       __syncthreads();
       // thread (channel group cg, key group kg): channels 4 cg .. + 3 of key slots 16 kg .. + 15,
       // read as 32-bit words (consecutive words across the warp) and transposed 4 x 4 bytes at
-      // a time in registers; output rows are channels, 16 key bytes each
+      // a time in registers; output rows are channels, 16 key bytes each, word i of a group
+      // holding key slots 2i, 2i + 1, 2i + 8, 2i + 9 of it
       const int cg = static_cast<int>(threadIdx.x & 31), kg = static_cast<int>(threadIdx.x >> 5);
       uint32_t o[4][4];   // o[channel j][key word i]
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int k0 = 16 * kg + 4 * i;
+        const int k0 = 16 * kg + 2 * i;
         const uint32_t a0 = *reinterpret_cast<const uint32_t*>(&tile[k0][4 * cg]);
         const uint32_t a1 = *reinterpret_cast<const uint32_t*>(&tile[k0 + 1][4 * cg]);
-        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(&tile[k0 + 2][4 * cg]);
-        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(&tile[k0 + 3][4 * cg]);
+        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(&tile[k0 + 8][4 * cg]);
+        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(&tile[k0 + 9][4 * cg]);
         const uint32_t t0 = __byte_perm(a0, a1, 0x5140), t1 = __byte_perm(a2, a3, 0x5140);
         const uint32_t t2 = __byte_perm(a0, a1, 0x7362), t3 = __byte_perm(a2, a3, 0x7362);
-        o[0][i] = __byte_perm(t0, t1, 0x5410);   // channel 4 cg: keys k0 .. k0 + 3
+        o[0][i] = __byte_perm(t0, t1, 0x5410);   // channel 4 cg: keys k0, k0 + 1, k0 + 8, k0 + 9
         o[1][i] = __byte_perm(t0, t1, 0x7632);
         o[2][i] = __byte_perm(t2, t3, 0x5410);
         o[3][i] = __byte_perm(t2, t3, 0x7632);
@@ -170,16 +177,42 @@ using attn::kKSt;
 using attn::kVSt;
 using attn::kRec;
 
+// Position of the diagonal key tile (the query tile's own index) in an item's list, or -1.
+// The full and the partial lists are ascending, so each takes one binary search; every role
+// calls this, so all of them visit the blocks in the same order.
+__device__ __forceinline__ int32_t diag_pos(const attn::Args& a, int64_t u, int32_t nf, int32_t n) {
+  const int32_t i = static_cast<int32_t>(u % a.nT);
+  const int32_t* f = a.full_idx + u * a.stride;
+  int32_t lo = 0, hi = nf;
+  while (lo < hi) {
+    const int32_t mid = (lo + hi) >> 1;
+    if (f[mid] < i) lo = mid + 1; else hi = mid;
+  }
+  if (lo < nf && f[lo] == i) return lo;
+  const int32_t* pp = a.part_idx + u * a.stride;
+  const int32_t np = n - nf;
+  lo = 0;
+  hi = np;
+  while (lo < hi) {
+    const int32_t mid = (lo + hi) >> 1;
+    if (pp[mid] < i) lo = mid + 1; else hi = mid;
+  }
+  return (lo < np && pp[lo] == i) ? nf + lo : -1;
+}
+// List position visited at step j: the diagonal first, then the others in list order.
+__device__ __forceinline__ int32_t visit_pos(int32_t j, int32_t d) {
+  return d < 0 ? j : (j == 0 ? d : (j <= d ? j - 1 : j));
+}
+
 constexpr int kThreads = 384;
 constexpr uint32_t kTileB = 16384;                             // 128 x 128 e4m3
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kQSt * kTileB;
 constexpr uint32_t kOffV = kOffK + kKSt * kTileB;              // V tiles transposed
-constexpr uint32_t kOffP = kOffV + kVSt * kTileB;              // two P buffers
-constexpr uint32_t kSmemTiles = kOffP + 2 * kTileB;            // 144 KB
+constexpr uint32_t kSmemTiles = kOffV + kVSt * kTileB;         // 112 KB
 constexpr uint32_t kSmemBytes = kSmemTiles + 1024;             // + alignment slack
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256;                     // S0 | S1 | O
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;        // S0 | S1 | O | P0 | P1 (32 columns each)
 constexpr uint32_t kIdesc = idesc_e4m3_f32(128, 128);
 constexpr float kPExp = 7.0f;                                  // P as e4m3 of 2^7 p
 constexpr float kRescaleLog2 = 1.75f;                          // 2^(7 + 1.75) = 430 < 448
@@ -212,9 +245,11 @@ __device__ __forceinline__ void role_qk_producer(const attn::Args& a, Bars& bars
     tma_load_2d(sb + kOffQ + qb * kTileB, tmQ, qbar, 0, static_cast<int32_t>(u * 128));
     const int64_t head_row = (u / a.nT) * a.nT;
     const int32_t* valid_h = a.valid + ((u / a.nT) % a.H) * a.nT;
+    const int32_t d = diag_pos(a, u, nf, n);
     for (int32_t j = 0; j < n; ++j) {
       bool b2;
-      const int32_t idx = item_key(a, u, nf, j, b2);
+      const int32_t jj = visit_pos(j, d);
+      const int32_t idx = item_key(a, u, nf, jj, b2);
       if (b2) flag_status(ST_BAD_LIST);
       const int32_t row = static_cast<int32_t>((head_row + idx) * 128);
       const uint32_t ks = kc % kKSt;
@@ -224,7 +259,7 @@ __device__ __forceinline__ void role_qk_producer(const attn::Args& a, Bars& bars
       mbar_arrive_expect_tx(kb, kTileB);
       tma_load_2d(sb + kOffK + ks * kTileB, tmK, kb, 0, row);
       int32_t nv = 128;
-      if (j >= nf) {
+      if (jj >= nf) {
         nv = valid_h[idx];
         if (nv < 1 || nv > 128) {
           flag_status(ST_BAD_LIST);
@@ -266,9 +301,10 @@ __device__ __forceinline__ void role_v_producer(const attn::Args& a, Bars& bars,
     const int32_t n = item_blocks(a, u, nf, bad);
     if (n == 0) continue;
     const int64_t head_row = (u / a.nT) * a.nT;
+    const int32_t d = diag_pos(a, u, nf, n);
     for (int32_t j = 0; j < n; ++j) {
       bool b2;
-      const int32_t idx = item_key(a, u, nf, j, b2);
+      const int32_t idx = item_key(a, u, nf, visit_pos(j, d), b2);
       const int32_t row = static_cast<int32_t>((head_row + idx) * 128);
       const uint32_t vs = vc % kVSt;
       if (vc >= kVSt && !mbar_wait(smem_u32(&bars.v_empty[vs]), (vc / kVSt - 1) & 1, abort, 115)) { stop = true; break; }
@@ -328,9 +364,9 @@ __device__ __forceinline__ void role_qk_issuer(Bars& bars, uint32_t sb, uint32_t
   mbar_wait(smem_u32(&bars.drain[0]), 0, nullptr, 121);
 }
 
-// P V issuer: O += P_b (shared memory, e4m3) x V_j (transposed tile, K-major).
+// P V issuer: O += P_b (tensor memory, e4m3, 8 columns per K = 32 step) x V_j (transposed
+// tile, K-major).
 __device__ __forceinline__ void role_pv_issuer(Bars& bars, uint32_t sb, uint32_t tmem, volatile int* abort) {
-  const uint64_t dP = smem_desc_sw128(sb + kOffP, 16, 1024);
   const uint64_t dV = smem_desc_sw128(sb + kOffV, 16, 1024);
   uint32_t items_done = 0;
   for (uint32_t g = 0;; ++g) {
@@ -344,11 +380,11 @@ __device__ __forceinline__ void role_pv_issuer(Bars& bars, uint32_t sb, uint32_t
         !mbar_wait(smem_u32(&bars.o_free), (items_done - 1) & 1, abort, 124))
       break;
     tc_fence_after();
-    const uint64_t a0 = opaque(dP + static_cast<uint64_t>(pb * (kTileB >> 4)));
+    const uint32_t pa = tmem + kColP + pb * 32;
     const uint64_t b0 = opaque(dV + static_cast<uint64_t>(vs * (kTileB >> 4)));
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_ss_f8(tmem + kColO, a0 + static_cast<uint64_t>(kk * 2), b0 + static_cast<uint64_t>(kk * 2), kIdesc,
+      mma_ts_f8(tmem + kColO, pa + kk * 8, b0 + static_cast<uint64_t>(kk * 2), kIdesc,
                 (kk > 0 || !(op & kOpNewItem)) ? 1u : 0u);
     tc_commit(smem_u32(&bars.o_done[pb]));
     tc_commit(smem_u32(&bars.v_empty[vs]));
@@ -369,7 +405,6 @@ __device__ __forceinline__ void softmax_role(const Args& p, Bars& bars, uint32_t
   const uint32_t base = 32 * (warp & 3) + 16 * (warp >> 2);
   const uint32_t lane_off = base << 16;
   const uint32_t r0 = base + lane / 4, c = lane & 3;
-  const uint32_t swz = r0 & 7;                 // rows r0 and r0 + 8 share the swizzle phase
   uint32_t g = 0;
   for (int64_t mm = 0;; ++mm) {
     const int64_t u = cta_item(mm);
@@ -415,81 +450,98 @@ __device__ __forceinline__ void softmax_role(const Args& p, Bars& bars, uint32_t
           if (k >= kv1) { s[4 * k + 1] = 0xFF800000u; s[4 * k + 3] = 0xFF800000u; }
         }
       }
-      // row maxima of the block (log2 units)
-      float a4[4], b4[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        a4[q] = fmaxf(__uint_as_float(s[4 * q]), __uint_as_float(s[4 * q + 1]));
-        b4[q] = fmaxf(__uint_as_float(s[4 * q + 2]), __uint_as_float(s[4 * q + 3]));
-      }
-#pragma unroll
-      for (int k = 4; k < 16; ++k) {
-        a4[k & 3] = fmax3(a4[k & 3], __uint_as_float(s[4 * k]), __uint_as_float(s[4 * k + 1]));
-        b4[k & 3] = fmax3(b4[k & 3], __uint_as_float(s[4 * k + 2]), __uint_as_float(s[4 * k + 3]));
-      }
-      const float mb0 = quad_max(fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3]))) * cs;
-      const float mb1 = quad_max(fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3]))) * cs;
+      // Exponentials with the current reference m, computed together with the block's row
+      // maxima (one basic block, so the MUFU and max chains interleave). If a row's maximum
+      // (log2 units) grew by more than 1.75, 2^7 P may have passed e4m3's range: the reference
+      // moves, O is rescaled and the pass is repeated. The roles visit the diagonal key tile
+      // first, which holds most rows' maxima, so repeats are rare. Block 0 of an item takes
+      // its row maxima first, so that its single pass has a reference.
       if (j == 0) {
-        m0 = mb0;
-        m1 = mb1;
-      } else {
-        // the reference moves when a row maximum grows by more than 1.75, so that 2^7 P
-        // stays below e4m3's largest value; O (holding P V of every earlier block) is rescaled
-        const bool need0 = mb0 > m0 + kRescaleLog2, need1 = mb1 > m1 + kRescaleLog2;
-        if (__any_sync(0xffffffffu, need0 || need1)) {
-          const uint32_t gp = g - 1;
-          if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 128)) { ok = false; break; }
-          tc_fence_after();
-          const float al0 = need0 ? ex2_approx(m0 - mb0) : 1.0f;
-          const float al1 = need1 ? ex2_approx(m1 - mb1) : 1.0f;
-          const uint64_t al0x2 = f2_pack(__float_as_uint(al0), __float_as_uint(al0));
-          const uint64_t al1x2 = f2_pack(__float_as_uint(al1), __float_as_uint(al1));
-#pragma unroll 1
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t o16[16];
-            const uint32_t oa = tmem + lane_off + kColO + ch * 32;
-            tmem_ld_16x256b_x4(oa, o16);
-            tmem_wait_ld();
-            reg_fence(o16);
+        float a4[4], b4[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float x, y;
-              f2_unpack(f2_mul(f2_pack(o16[4 * q], o16[4 * q + 1]), al0x2), x, y);
-              o16[4 * q] = __float_as_uint(x); o16[4 * q + 1] = __float_as_uint(y);
-              f2_unpack(f2_mul(f2_pack(o16[4 * q + 2], o16[4 * q + 3]), al1x2), x, y);
-              o16[4 * q + 2] = __float_as_uint(x); o16[4 * q + 3] = __float_as_uint(y);
-            }
-            tmem_st_16x256b_x4(oa, o16);
-          }
-          tmem_wait_st();
-          if (need0) { l0 *= al0; m0 = mb0; }
-          if (need1) { l1 *= al1; m1 = mb1; }
+        for (int q = 0; q < 4; ++q) {
+          a4[q] = fmaxf(__uint_as_float(s[4 * q]), __uint_as_float(s[4 * q + 1]));
+          b4[q] = fmaxf(__uint_as_float(s[4 * q + 2]), __uint_as_float(s[4 * q + 3]));
         }
-      }
-      // P buffer g & 1 is free once P V of block g - 2 has completed
-      if (g >= 2) {
-        const uint32_t gp = g - 2;
-        if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 129)) { ok = false; break; }
-      }
-      // 2^(s * cs - m + 7) -> e4m3 pairs at key bytes 8k + 2c of rows r0, r0 + 8 of the
-      // 128-byte-swizzled K-major tile (16-byte chunk k / 2 of a row sits at chunk (k / 2) ^ (row & 7))
-      const uint64_t nm0 = f2_pack(__float_as_uint(kPExp - m0), __float_as_uint(kPExp - m0));
-      const uint64_t nm1 = f2_pack(__float_as_uint(kPExp - m1), __float_as_uint(kPExp - m1));
-      const uint32_t prow = sb + kOffP + sbuf * kTileB + r0 * 128 + 2 * c;
-      uint64_t acc0[2] = {0ull, 0ull}, acc1[2] = {0ull, 0ull};
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        float x0, x1, y0, y1;
-        f2_unpack(f2_fma(f2_pack(s[4 * k], s[4 * k + 1]), c2, nm0), x0, x1);
-        f2_unpack(f2_fma(f2_pack(s[4 * k + 2], s[4 * k + 3]), c2, nm1), y0, y1);
-        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), q0 = ex2_approx(y0), q1 = ex2_approx(y1);
-        acc0[k & 1] = f2_add(acc0[k & 1], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
-        acc1[k & 1] = f2_add(acc1[k & 1], f2_pack(__float_as_uint(q0), __float_as_uint(q1)));
-        const uint32_t off = ((static_cast<uint32_t>(k >> 1) ^ swz) << 4) + 8 * static_cast<uint32_t>(k & 1);
-        const uint16_t e0 = pack_e4m3x2(p0, p1), e1 = pack_e4m3x2(q0, q1);
-        asm volatile("st.shared.b16 [%0], %1;" ::"r"(prow + off), "h"(e0) : "memory");
-        asm volatile("st.shared.b16 [%0], %1;" ::"r"(prow + 8 * 128 + off), "h"(e1) : "memory");
+        for (int k = 4; k < 16; ++k) {
+          a4[k & 3] = fmax3(a4[k & 3], __uint_as_float(s[4 * k]), __uint_as_float(s[4 * k + 1]));
+          b4[k & 3] = fmax3(b4[k & 3], __uint_as_float(s[4 * k + 2]), __uint_as_float(s[4 * k + 3]));
+        }
+        m0 = quad_max(fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3]))) * cs;
+        m1 = quad_max(fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3]))) * cs;
       }
+      // 2^(s * cs - m + 7) -> e4m3. Word m of a row (column 4m + c of the P buffer, 16x128b
+      // shape) packs the pairs of 8-column groups 2m and 2m + 1: key slots 16m + 2c + {0, 1}
+      // and 16m + 8 + 2c + {0, 1}, the order of V's transposed tiles
+      uint32_t pk[16];
+      uint64_t acc0[2], acc1[2];
+#pragma unroll 1
+      for (int pass = 0;; ++pass) {
+        const uint64_t nm0 = f2_pack(__float_as_uint(kPExp - m0), __float_as_uint(kPExp - m0));
+        const uint64_t nm1 = f2_pack(__float_as_uint(kPExp - m1), __float_as_uint(kPExp - m1));
+        acc0[0] = acc0[1] = acc1[0] = acc1[1] = 0ull;
+        float a4[4], b4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          a4[q] = fmaxf(__uint_as_float(s[4 * q]), __uint_as_float(s[4 * q + 1]));
+          b4[q] = fmaxf(__uint_as_float(s[4 * q + 2]), __uint_as_float(s[4 * q + 3]));
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          if (k >= 4) {
+            a4[k & 3] = fmax3(a4[k & 3], __uint_as_float(s[4 * k]), __uint_as_float(s[4 * k + 1]));
+            b4[k & 3] = fmax3(b4[k & 3], __uint_as_float(s[4 * k + 2]), __uint_as_float(s[4 * k + 3]));
+          }
+          float x0, x1, y0, y1;
+          f2_unpack(f2_fma(f2_pack(s[4 * k], s[4 * k + 1]), c2, nm0), x0, x1);
+          f2_unpack(f2_fma(f2_pack(s[4 * k + 2], s[4 * k + 3]), c2, nm1), y0, y1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), q0 = ex2_approx(y0), q1 = ex2_approx(y1);
+          acc0[k & 1] = f2_add(acc0[k & 1], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
+          acc1[k & 1] = f2_add(acc1[k & 1], f2_pack(__float_as_uint(q0), __float_as_uint(q1)));
+          const uint32_t e0 = pack_e4m3x2(p0, p1), e1 = pack_e4m3x2(q0, q1);
+          if (k & 1) {
+            pk[k - 1] |= e0 << 16;
+            pk[k] |= e1 << 16;
+          } else {
+            pk[k] = e0;
+            pk[k + 1] = e1;
+          }
+        }
+        const float mb0 = quad_max(fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3]))) * cs;
+        const float mb1 = quad_max(fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3]))) * cs;
+        const bool need0 = mb0 > m0 + kRescaleLog2, need1 = mb1 > m1 + kRescaleLog2;
+        if (pass == 1 || !__any_sync(0xffffffffu, need0 || need1)) break;
+        // O must hold P V of every earlier block before it is rescaled
+        const uint32_t gp = g - 1;
+        if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 128)) { ok = false; break; }
+        tc_fence_after();
+        const float al0 = need0 ? ex2_approx(m0 - mb0) : 1.0f;
+        const float al1 = need1 ? ex2_approx(m1 - mb1) : 1.0f;
+        const uint64_t al0x2 = f2_pack(__float_as_uint(al0), __float_as_uint(al0));
+        const uint64_t al1x2 = f2_pack(__float_as_uint(al1), __float_as_uint(al1));
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t o16[16];
+          const uint32_t oa = tmem + lane_off + kColO + ch * 32;
+          tmem_ld_16x256b_x4(oa, o16);
+          tmem_wait_ld();
+          reg_fence(o16);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float x, y;
+            f2_unpack(f2_mul(f2_pack(o16[4 * q], o16[4 * q + 1]), al0x2), x, y);
+            o16[4 * q] = __float_as_uint(x); o16[4 * q + 1] = __float_as_uint(y);
+            f2_unpack(f2_mul(f2_pack(o16[4 * q + 2], o16[4 * q + 3]), al1x2), x, y);
+            o16[4 * q + 2] = __float_as_uint(x); o16[4 * q + 3] = __float_as_uint(y);
+          }
+          tmem_st_16x256b_x4(oa, o16);
+        }
+        tmem_wait_st();
+        if (need0) { l0 *= al0; m0 = mb0; }
+        if (need1) { l1 *= al1; m1 = mb1; }
+      }
+      if (!ok) break;
       {
         float t0, t1, t2, t3;
         f2_unpack(acc0[0], t0, t1); f2_unpack(acc0[1], t2, t3);
@@ -497,8 +549,15 @@ __device__ __forceinline__ void softmax_role(const Args& p, Bars& bars, uint32_t
         f2_unpack(acc1[0], t0, t1); f2_unpack(acc1[1], t2, t3);
         l1 += (t0 + t1) + (t2 + t3);
       }
-      // the tensor core reads P through the async proxy
-      fence_proxy_async_smem();
+      // P buffer g & 1 is free once P V of block g - 2 has completed
+      if (g >= 2) {
+        const uint32_t gp = g - 2;
+        if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 129)) { ok = false; break; }
+        tc_fence_after();
+      }
+      tmem_st_16x128b_x8(tmem + lane_off + kColP + sbuf * 32, pk);
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars.p_full[sbuf]));
     }

@@ -340,8 +340,8 @@ def block_sparse_attn_fwd(q_t: torch.Tensor, k_t: torch.Tensor, v_t: torch.Tenso
 def quantize_fp8(x_t: torch.Tensor, transpose_tiles: bool = False, codes: Optional[torch.Tensor] = None,
                  scale: Optional[torch.Tensor] = None, stream=None):
     """Tiled bf16 [B, H, Npad, 128] -> (e4m3 codes uint8 [B, H, Npad, 128], scale fp32 [B, H]);
-    with transpose_tiles every 128 x 128 tile of the codes is stored transposed (V of the FP8
-    attention)."""
+    with transpose_tiles every 128 x 128 tile of the codes is stored transposed, keys in the
+    order veda_quantize_fp8 documents (V of the FP8 attention)."""
     _need(x_t, torch.bfloat16, "x_t")
     B, H, Npad, D = x_t.shape
     if codes is None:

@@ -352,8 +352,10 @@ VEDA_API veda_status veda_block_sparse_attn_bwd(const void* q, const void* k, co
  * infinities) with one scale per (batch, head): scale = max |x| / 448 and
  * code = e4m3(x * (448 / max |x|)), both in fp32, rounding to nearest even and saturating at
  * +-448; an all-zero (batch, head) gets scale 1. With transpose_tiles = 1 every 128 x 128
- * tile of the codes is stored transposed ([channel][key slot]), the layout the FP8 attention
- * takes for V.
+ * tile of the codes is stored transposed ([channel][key position]), the layout the FP8
+ * attention takes for V: within every group of 16 positions, position 16m + 4c + e
+ * (c, e in 0..3) holds key slot 16m + 2c + (e & 1) + 8 (e >> 1), the order in which the
+ * attention's softmax packs P into tensor memory.
  *   x_tiled          [B][H][nT*128][D] bf16 (device)
  *   codes            [B][H][nT*128][D] uint8 e4m3 (device, out)
  *   scale            [B][H] fp32 (device, out; also used as scratch during the call)

@@ -82,6 +82,20 @@ def gpu_lists_equal(gl, lists: O.BlockLists, heads: Sequence[int], rows=None) ->
     return bad, total
 
 
+def fp8_v_key_positions() -> np.ndarray:
+    """Key slot at each key position of a transposed V tile of veda_quantize_fp8: within every
+    group of 16, position 4c + e holds slot 2c + (e % 2) + 8 (e // 2) (include/veda.h)."""
+    pos = np.arange(128)
+    m, c, e = pos // 16, (pos % 16) // 4, pos % 4
+    return 16 * m + 2 * c + (e % 2) + 8 * (e // 2)
+
+
+def fp8_v_layout(codes_t: np.ndarray) -> np.ndarray:
+    """Oracle codes with plainly transposed tiles ([..., channel, key slot]) in the library's
+    key order."""
+    return codes_t[..., fp8_v_key_positions()]
+
+
 def score_errors(gpu: np.ndarray, ref: np.ndarray) -> float:
     """Worst |gpu - ref| / max(|ref|, mean|ref| of the head's matrix) over all entries."""
     worst = 0.0

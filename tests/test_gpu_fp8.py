@@ -2,7 +2,9 @@
 
 Quantisation: the GPU's e4m3 codes and per-(batch, head) scales of the tiled Q, K and V
 (V with transposed tiles) equal the oracle's bit for bit (both sides form x * (448 / amax)
-in fp32 and round to nearest even, reading R23).
+in fp32 and round to nearest even, reading R23); the library's transposed tiles list the
+keys of every group of 16 in the order its softmax packs P, which the comparison applies to
+the oracle's plainly transposed tiles.
 Attention: the GPU's FP8 attention over its own block lists is compared with the oracle's
 fp64 attention of the oracle's dequantised tensors over the same lists (fed back as the
 parity rule feeds the selection its scores). The scores then agree up to fp32 summation
@@ -85,7 +87,7 @@ def _run(w, heads, rows=None):
     cq, s_q = O.quantize_fp8(qt)
     ck, s_k = O.quantize_fp8(kt)
     cv, s_v = O.quantize_fp8(vt, transpose_tiles=True)
-    for got, ref, n in ((q8, cq, "q"), (k8, ck, "k"), (vt8, cv, "v")):
+    for got, ref, n in ((q8, cq, "q"), (k8, ck, "k"), (vt8, P.fp8_v_layout(cv), "v")):
         g = got[:, heads].cpu().numpy()
         assert np.array_equal(g, ref), f"{n} codes differ at {int((g != ref).sum())} of {ref.size}"
     for got, ref, n in ((sq, s_q, "q"), (sk, s_k, "k"), (sv, s_v, "v")):
@@ -157,6 +159,76 @@ def test_quantize_zero_tensor_negative_zero_and_large_values():
         codes, scale = V.quantize_fp8(x.to(DEV), transpose_tiles=tr)
         V.check_device_status()
         c_o, s_o = O.quantize_fp8(P.f64(x), transpose_tiles=tr)
+        if tr:
+            c_o = P.fp8_v_layout(c_o)
         assert np.array_equal(scale.cpu().numpy(), s_o)
         assert np.array_equal(codes.cpu().numpy(), c_o), int((codes.cpu().numpy() != c_o).sum())
         assert scale[0, 1].item() == 1.0 and not codes[0, 1].any()
+
+
+def test_fp8_reference_moves_diagonal_first_and_lists_without_the_diagonal():
+    """Key tile j's scores sit ~5 (log2 units) above tile j - 1's for half the rows and below
+    for the other half, so the e4m3 softmax (which may not let 2^7 P pass 448) must move its
+    reference, rescale O and repeat the block's pass for many blocks, in the order the kernel
+    visits them: the diagonal tile first, then the list in order. Query tile 1's list leaves
+    out its diagonal (list order kept); query tile 3's diagonal is in the partial list (tile 3
+    holds 64 valid slots)."""
+    V = P.veda()
+    grid, shape = (1, 8, 56), (1, 8, 16)
+    maps = V.build_tile_map(grid, [shape]).to(DEV)
+    slots, nv, seg, nTh = P.oracle_maps(synth.Workload("growth8", 12, B=1, H=1, grid=grid, head_shapes=(shape,),
+                                                       rho=((1, 1),), field=False), None)
+    nT = int(nTh[0])
+    assert nT == 4 and list(nv[0]) == [128, 128, 128, 64]
+    g = torch.Generator().manual_seed(12012)
+    Npad = nT * 128
+    sign = torch.ones(128)
+    sign[64:] = -1.0
+    q = sign[:, None] + 0.05 * torch.randn((nT, 128, 128), generator=g)
+    c = torch.tensor([0.0, 40.0, 80.0, 120.0])                                    # score level of key tile j
+    k = (c[:, None, None] / 128.0) + 0.5 * torch.randn((nT, 128, 128), generator=g)
+    v = torch.randn((nT, 128, 128), generator=g)
+    q, k, v = (x.reshape(1, 1, Npad, 128).to(torch.bfloat16) for x in (q, k, v))
+    valid = torch.from_numpy(slots[0] >= 0)
+    for x in (q, k, v):
+        x[0, 0, ~valid] = 0
+
+    cq, s_q = O.quantize_fp8(P.f64(q))
+    ck, s_k = O.quantize_fp8(P.f64(k))
+    cv, s_v = O.quantize_fp8(P.f64(v), transpose_tiles=True)
+    qd, kd, vd = O.dequantize_fp8(cq, s_q), O.dequantize_fp8(ck, s_k), O.dequantize_fp8(cv, s_v, True)
+    # the construction does what it claims on the dequantised tensors: every valid query row's
+    # maximum moves by more than 1.75 (log2 units) from one key tile to the next
+    s2 = (qd[0, 0] @ kd[0, 0].T) * P.SCALE * math.log2(math.e)
+    rows = np.flatnonzero(slots[0] >= 0)
+    row_max = [s2[rows, j * 128:j * 128 + int(nv[0][j])].max(axis=1) for j in range(nT)]
+    assert all(np.abs(row_max[j + 1] - row_max[j]).min() > 1.75 for j in range(nT - 1))
+
+    full = [[[np.array([0, 1, 2]), np.array([0, 2]), np.array([0, 1, 2]), np.array([0, 1, 2])]]]
+    part = [[[np.array([3]) for _ in range(nT)]]]
+    lists = O.BlockLists(full, part)
+    stride = V.list_stride_for(nT, [(1, 1)])
+    q8, sq = V.quantize_fp8(q.to(DEV))
+    k8, sk = V.quantize_fp8(k.to(DEV))
+    vt8, sv = V.quantize_fp8(v.to(DEV), transpose_tiles=True)
+    o8, lse8 = V.block_sparse_attn_fwd_fp8(q8, k8, vt8, sq, sk, sv, maps,
+                                           P.lists_to_device(lists, 1, 1, nT, stride, DEV), P.SCALE)
+    V.check_device_status()
+    for got, ref, n in ((q8, cq, "q"), (k8, ck, "k"), (vt8, P.fp8_v_layout(cv), "v")):
+        assert np.array_equal(got.cpu().numpy(), ref), f"{n} codes differ"
+
+    o_ref, lse_ref = O.attention(qd, kd, vd, nv, lists, P.SCALE)
+    o_abs, _ = O.attention(qd, kd, np.abs(vd), nv, lists, P.SCALE)
+    todo = [(0, 0, r) for r in range(nT)]
+    tiny = _tiny_mass(qd, kd, nv, lists, todo, P.SCALE)
+    og, lg = P.f64(o8), P.f64(lse8)
+    assert np.isfinite(og).all() and np.isfinite(lg).all()
+    vmax = np.abs(vd[0, 0]).max()
+    for (b, j, r) in todo:
+        sl = slice(r * 128, (r + 1) * 128)
+        band = (2.0 ** -4 * o_abs[b, j, sl] + tiny[(b, j, r)][:, None] * vmax
+                + 2.0 ** -8 * np.abs(o_ref[b, j, sl]) + 2.0 ** -14)
+        err = np.abs(og[b, j, sl] - o_ref[b, j, sl])
+        assert np.all(err <= band), f"tile {r}: max err {err.max():.3g}"
+        dl = np.abs(lg[b, j, sl] - lse_ref[b, j, sl])
+        assert np.all(dl <= 2e-3 + 1e-5 * np.abs(lse_ref[b, j, sl])), f"tile {r}: LSE differs by {dl.max():.3g}"
