@@ -395,9 +395,9 @@ __device__ __forceinline__ void role_pv_issuer(Bars& bars, uint32_t sb, uint32_t
 }
 
 // Softmax warps: the bf16 kernel's 16-row layout (thread: rows r0 = base + lane / 4 and
-// r0 + 8, of every 8-column group k the columns 8k + 2c + {0, 1}, c = lane % 4). The row
-// maxima come first; P goes to shared memory as e4m3 pairs.
-__device__ __forceinline__ void softmax_role(const Args& p, Bars& bars, uint32_t sb, uint32_t tmem, uint32_t warp,
+// r0 + 8, of every 8-column group k the columns 8k + 2c + {0, 1}, c = lane % 4). One pass
+// takes the exponentials with the block's row maxima; P goes to tensor memory as e4m3 words.
+__device__ __forceinline__ void softmax_role(const Args& p, Bars& bars, uint32_t tmem, uint32_t warp,
                                              uint32_t lane) {
   using namespace attn;
   const attn::Args& a = p.a;
@@ -631,7 +631,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       fp8::role_pv_issuer(bars, sb, tmem, abort);
   } else {
     attn::reg_alloc<attn::kSoftmaxRegs>();
-    fp8::softmax_role(p, bars, sb, tmem, warp, lane);
+    fp8::softmax_role(p, bars, tmem, warp, lane);
   }
 
   tc_fence_before();
