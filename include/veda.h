@@ -348,8 +348,10 @@ VEDA_API veda_status veda_block_sparse_attn_bwd(const void* q, const void* k, co
                                        int32_t B, int32_t H, int32_t nT, int32_t D, veda_stream_t stream);
 
 /*
- * FP8 variant, quantisation (device): tiled bf16 tensors -> e4m3 codes (OCP FP8 E4M3, no
- * infinities) with one scale per (batch, head): scale = max |x| / 448 and
+ * FP8 variant, quantisation (device). "Deploying this checkpoint", preamble and section 3:
+ * the predictor ships in FP8; the pages give no FP8 attention, so this variant quantises the
+ * tiled Q, K, V per tensor and follows step 5 (the plainest reading). Tiled bf16 tensors ->
+ * e4m3 codes (OCP FP8 E4M3, no infinities) with one scale per (batch, head): scale = max |x| / 448 and
  * code = e4m3(x * (448 / max |x|)), both in fp32, rounding to nearest even and saturating at
  * +-448; an all-zero (batch, head) gets scale 1. With transpose_tiles = 1 every 128 x 128
  * tile of the codes is stored transposed ([channel][key position]), the layout the FP8
@@ -368,8 +370,10 @@ VEDA_API veda_status veda_quantize_fp8(const void* x_tiled, void* codes, float* 
                                        int32_t nT, int32_t D, int32_t transpose_tiles, veda_stream_t stream);
 
 /*
- * FP8 variant of step 5 (device): the attention of veda_block_sparse_attn_fwd over the same
- * lists, from e4m3 operands. S = (Q codes)(K codes)^T on the tensor cores, times
+ * FP8 variant of step 5 (device; same passages as veda_block_sparse_attn_fwd, FP8 as in
+ * veda_quantize_fp8): the attention of veda_block_sparse_attn_fwd over the same lists, from
+ * e4m3 operands. Each query tile visits its own key tile first when its list holds it, then
+ * the rest in list order (the result depends on the order only through fp32 rounding). S = (Q codes)(K codes)^T on the tensor cores, times
  * q_scale * k_scale * softmax_scale; P = 2^(s - m + 7) enters P V as e4m3 (the row reference
  * m moves when a row maximum grows by more than 1.75 in log2 units, so that 2^7 P stays
  * below 448); O = (P V) * v_scale / l in bf16, LSE as in the bf16 call.
