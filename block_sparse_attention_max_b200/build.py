@@ -14,7 +14,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libveda.so")
 
-SOURCES = ["veda_lib.cu", "veda_tile_map.cpp"]
+SOURCES = ["veda_lib.cu", "veda_tile_map.cpp", "veda_plan.cpp"]
 HEADERS = ["veda_ptx.cuh", "k_attn.cuh", "k_heat.cuh", "k_bwd.cuh", "k_fp8.cuh", "k_gather.cuh", "k_scores.cuh", "k_select.cuh"]
 
 NVCC_FLAGS = [

@@ -321,9 +321,31 @@ veda_status veda_block_scores(const float* pooled_q, const float* pooled_k, cons
 
 // Scratch of veda_block_scores_noalloc: part of the library's device image, so no call
 // ever allocates. Host code must not pass `g_noalloc_scratch` itself to a kernel (on the
-// host it is only a stand-in symbol); its device address is looked up once per device.
+// host it is only a stand-in symbol); its device address is looked up once per device and
+// context, with that device current, and cached together with the context it belongs to.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[VEDA_NOALLOC_SCORES_BYTES];
-static void* g_noalloc_ptr[kMaxDevices] = {};
+struct NoallocSlot {
+  CUcontext ctx;   // context the address was looked up in
+  void* ptr;       // device address of g_noalloc_scratch in that context
+};
+static NoallocSlot g_noalloc[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+static CtxGetCurrentFn g_ctx_current = nullptr;
+
+// Current context of the calling thread (null before the runtime has created one).
+static veda_status current_context(CUcontext& ctx) {
+  if (g_ctx_current == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return fail(VEDA_ERR_CUDA, "cuCtxGetCurrent entry point not found");
+    g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+  }
+  ctx = nullptr;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS) return fail(VEDA_ERR_CUDA, "cuCtxGetCurrent failed");
+  return VEDA_OK;
+}
 
 veda_status veda_block_scores_noalloc(const float* pooled_q, const float* pooled_k, const float* Wq,
                                       const float* Wk, float* scores, int32_t B, int32_t H, int32_t nT,
@@ -342,13 +364,21 @@ veda_status veda_block_scores_noalloc(const float* pooled_q, const float* pooled
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    CUcontext ctx = nullptr;
+    veda_status st = current_context(ctx);
+    if (st != VEDA_OK) return st;
+    NoallocSlot& slot = g_noalloc[dev];
+    if (slot.ptr == nullptr || ctx == nullptr || slot.ctx != ctx) {
+      // first call on this device, or its context was replaced (e.g. after a device reset,
+      // which reloads the library's module): look the address up again, `dev` current
       void* p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);   // with `dev` current
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
       if (e != cudaSuccess || p == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
-      g_noalloc_ptr[dev] = p;
+      if ((st = current_context(ctx)) != VEDA_OK) return st;
+      slot.ctx = ctx;
+      slot.ptr = p;
     }
-    scratch = g_noalloc_ptr[dev];
+    scratch = slot.ptr;
   }
   return veda_block_scores(pooled_q, pooled_k, Wq, Wk, scores, scratch, VEDA_NOALLOC_SCORES_BYTES, B, H, nT, D,
                            stream);

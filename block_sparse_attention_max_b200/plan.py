@@ -31,15 +31,6 @@ class TilePlan:
         return [self.candidates[c] for c in self.assign]
 
 
-def _vote(err: np.ndarray, max_shapes: int):
-    H, C = err.shape
-    votes = np.bincount(np.argmin(err, axis=1), minlength=C)
-    order = sorted(range(C), key=lambda c: (-votes[c], c))
-    kept = sorted([c for c in order[:max_shapes] if votes[c] > 0] or [order[0]])
-    assign = np.array([kept[int(np.argmin(err[h, kept]))] for h in range(H)])
-    return kept, assign
-
-
 def shape_errors(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid: Tuple[int, int, int], n_tail: int,
                  candidates: Sequence[Tuple[int, int, int]], rho: Sequence[Tuple[int, int]],
                  scale: float) -> np.ndarray:
@@ -70,5 +61,5 @@ def tile_plan_search(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid: Tu
                      n_tail: int, candidates: Sequence[Tuple[int, int, int]], rho: Sequence[Tuple[int, int]],
                      scale: float, max_shapes: int = 2) -> TilePlan:
     err = shape_errors(q, k, v, grid, n_tail, candidates, rho, scale)
-    kept, assign = _vote(err, max_shapes)
+    kept, assign = V.tile_plan_vote(err, max_shapes)
     return TilePlan(list(map(tuple, candidates)), err, kept, assign)

@@ -10,7 +10,7 @@ from __future__ import annotations
 import ctypes
 import dataclasses
 import os
-from typing import Optional, Sequence, Tuple
+from typing import List, Optional, Sequence, Tuple
 
 import numpy as np
 import torch
@@ -29,6 +29,7 @@ EXPORTED = (
     "veda_select_blocks",
     "veda_block_sparse_attn_fwd", "veda_unpermute", "veda_transpose_lists",
     "veda_block_sparse_attn_bwd", "veda_block_heat", "veda_mask_quality", "veda_rel_error",
+    "veda_tile_plan_vote",
     "veda_quantize_fp8", "veda_block_sparse_attn_fwd_fp8",
     "veda_check_device_status", "veda_selftest_wait_timeout",
 )
@@ -80,6 +81,7 @@ _SIG = {
     "veda_block_sparse_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _I,
                                         _F, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "veda_rel_error": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
+    "veda_tile_plan_vote": (_I, [_P, _I, _I, _I, _P, _P, _P]),
     "veda_block_heat": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _F, _P, _I, _I, _I, _I, _P]),
     "veda_mask_quality": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _I, _P, _P, _P,
                                _I, _I, _I, _P]),
@@ -126,6 +128,9 @@ def _need(t: torch.Tensor, dtype: torch.dtype, name: str, cuda: bool = True) -> 
         raise ValueError(f"{name}: must be contiguous")
     if cuda and not t.is_cuda:
         raise ValueError(f"{name}: must be a CUDA tensor")
+    if cuda and t.device.index != torch.cuda.current_device():
+        # the library launches on the calling thread's current device
+        raise ValueError(f"{name}: on {t.device}, but the current device is cuda:{torch.cuda.current_device()}")
 
 
 # ---------------------------------------------------------------------------------------
@@ -271,10 +276,17 @@ def block_scores_noalloc(pooled_q: torch.Tensor, pooled_k: torch.Tensor, wq: tor
     """
     for t, n in ((pooled_q, "pooled_q"), (pooled_k, "pooled_k"), (wq, "wq"), (wk, "wk")):
         _need(t, torch.float32, n)
-    B, H, nT, _, D = pooled_q.shape
+    B, H, nT, three, D = pooled_q.shape
+    if three != 3 or tuple(pooled_k.shape) != tuple(pooled_q.shape):
+        raise ValueError("pooled_q / pooled_k: expected equal shapes [B, H, nT, 3, D]")
+    for t, n in ((wq, "wq"), (wk, "wk")):
+        if tuple(t.shape) != (H, D, 3 * D):
+            raise ValueError(f"{n}: expected shape {(H, D, 3 * D)}, got {tuple(t.shape)}")
     if out is None:
         out = torch.empty((B, H, nT, nT), dtype=torch.float32, device=pooled_q.device)
     _need(out, torch.float32, "out")
+    if tuple(out.shape) != (B, H, nT, nT):
+        raise ValueError(f"out: expected shape {(B, H, nT, nT)}, got {tuple(out.shape)}")
     _check("veda_block_scores_noalloc", lib().veda_block_scores_noalloc(
         _ptr(pooled_q), _ptr(pooled_k), _ptr(wq), _ptr(wk), _ptr(out), B, H, nT, D,
         _stream(stream)))
@@ -481,6 +493,21 @@ def rel_error(o: torch.Tensor, o_ref: torch.Tensor, stream=None) -> torch.Tensor
     _check("veda_rel_error", lib().veda_rel_error(_ptr(o), _ptr(o_ref), _ptr(sums), B, N, H, D,
                                                   _stream(stream)))
     return sums
+
+
+def tile_plan_vote(errors: np.ndarray, max_shapes: int = 2) -> Tuple[List[int], np.ndarray]:
+    """veda_tile_plan_vote (host): the kept candidates (ascending) and each head's candidate
+    from an [H, C] matrix of relative output errors."""
+    err = np.ascontiguousarray(errors, dtype=np.float64)
+    if err.ndim != 2:
+        raise ValueError("errors: expected [H, C]")
+    H, C = err.shape
+    kept = np.zeros(max(1, min(max_shapes, C)), np.int32)
+    n_kept = np.zeros(1, np.int32)
+    assign = np.zeros(H, np.int32)
+    _check("veda_tile_plan_vote", lib().veda_tile_plan_vote(
+        err.ctypes.data, H, C, max_shapes, kept.ctypes.data, n_kept.ctypes.data, assign.ctypes.data))
+    return [int(c) for c in kept[:int(n_kept[0])]], assign
 
 
 def unpermute(o_t: torch.Tensor, maps: DeviceMaps, N: int, out: Optional[torch.Tensor] = None,

@@ -20,6 +20,7 @@
  *   veda_block_heat                per-block attention mass of dense attention
  *   veda_mask_quality              attention mass a mask keeps, recall against the oracle mask
  *   veda_rel_error                 relative output error per head (tile-plan search)
+ *   veda_tile_plan_vote            the search's vote: kept tile shapes, one per head (host)
  *
  * and an FP8 variant of step 5 (the pages ship their predictor in FP8, "Deploying this
  * checkpoint", preamble and section 3; the attention variant is this library's):
@@ -206,7 +207,8 @@ VEDA_API veda_status veda_block_scores(const float* pooled_q, const float* poole
  *     without launching anything.
  *   - Set-up: the first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call before
- *     any stream capture.
+ *     any stream capture. The address is cached with the context it was looked up in;
+ *     a call made in a different context (after cudaDeviceReset, say) looks it up again.
  *   - Sharing: every call on a device uses the same array and leaves its contents
  *     behind. Nothing in it needs to start at zero (each call overwrites all it reads),
  *     but calls whose executions overlap on the GPU (different streams without
@@ -455,6 +457,24 @@ VEDA_API veda_status veda_mask_quality(const float* heat, const int32_t* tile_va
  */
 VEDA_API veda_status veda_rel_error(const void* o, const void* o_ref, float* sums, int32_t B, int32_t N,
                            int32_t H, int32_t D, veda_stream_t stream);
+
+/*
+ * Vote of the oracle tile-plan search (host). "Miowtion" README, Key Features / Veda sparse
+ * attention: tile shapes per layer by oracle search over the relative output MSE under the
+ * best mask, majority vote, at most two shapes per layer.
+ *   errors     [H][C] fp64 (host): relative output error of candidate c for head h
+ *              (veda_rel_error's sums[2h] / sums[2h + 1] under that candidate's tiling)
+ *   max_shapes shapes the layer may keep (the pages: 2)
+ *   kept       [min(max_shapes, C)] int32 (host, out): kept candidates, ascending
+ *   n_kept     (host, out): how many entries of kept are set (>= 1)
+ *   assign     [H] int32 (host, out): the candidate each head takes
+ * A head votes for its candidate of least error (the earliest of equal errors); the layer
+ * keeps the most voted candidates, at most max_shapes and only voted ones (the earliest of
+ * equal counts first); each head takes its least-error kept candidate (the earliest of
+ * equal errors). NaN errors return VEDA_ERR_INVALID_ARG. No device work.
+ */
+VEDA_API veda_status veda_tile_plan_vote(const double* errors, int32_t H, int32_t C, int32_t max_shapes,
+                                         int32_t* kept, int32_t* n_kept, int32_t* assign);
 
 /*
  * Self-test of the library's failure detection (no counterpart on the pages). Launches

@@ -111,3 +111,41 @@ def test_no_device_means_error_not_fallback(L):
     st = L.veda_permute_tiles(256, 256, 256, 1, 128, 1, 128, 128, None)
     assert st in (2, 3)
     assert L.veda_check_device_status(None, None) == 3
+
+
+def test_tile_plan_vote_hand_examples(L):
+    # the oracle's hand-worked votes, through the C ABI
+    err = np.array([[0.1, 0.2, 0.3],
+                    [0.5, 0.4, 0.3],
+                    [0.9, 0.8, 0.1],
+                    [0.3, 0.1, 0.4],
+                    [0.6, 0.6, 0.5]])
+    kept, assign = veda.tile_plan_vote(err)
+    assert kept == [0, 2] and assign.tolist() == [0, 2, 2, 0, 2]
+    kept, assign = veda.tile_plan_vote(err, max_shapes=1)
+    assert kept == [2] and assign.tolist() == [2] * 5
+    kept, assign = veda.tile_plan_vote(err, max_shapes=3)
+    assert kept == [0, 1, 2] and assign.tolist() == [0, 2, 2, 1, 2]
+    kept, assign = veda.tile_plan_vote(np.array([[0.1, 0.2], [0.2, 0.3]]))
+    assert kept == [0] and assign.tolist() == [0, 0]
+    kept, assign = veda.tile_plan_vote(np.array([[0.2, 0.2, 0.2]]), max_shapes=1)
+    assert kept == [0] and assign.tolist() == [0]
+
+
+def test_tile_plan_vote_matches_oracle_on_random_matrices(L):
+    # errors on a coarse grid, so that equal errors and equal vote counts are common
+    rng = np.random.default_rng(123)
+    for _ in range(300):
+        H, C = int(rng.integers(1, 12)), int(rng.integers(1, 7))
+        err = rng.integers(0, 5, size=(H, C)) / 4.0
+        for ms in (1, 2, 3):
+            kept, assign = veda.tile_plan_vote(err, ms)
+            kept_o, assign_o = O.tile_plan(err, ms)
+            assert kept == list(kept_o) and assign.tolist() == assign_o.tolist(), (err, ms)
+
+
+def test_tile_plan_vote_rejects_nan_and_bad_sizes(L):
+    with pytest.raises(veda.VedaError):
+        veda.tile_plan_vote(np.array([[0.1, np.nan]]))
+    with pytest.raises(veda.VedaError):
+        veda.tile_plan_vote(np.zeros((2, 3)), max_shapes=0)

@@ -319,12 +319,48 @@ def test_device_check_flags_bad_lists_without_fault():
 @pytest.mark.parametrize("name,heads,rows", [
     ("clip16x9_rho1_1", [7], [0, 250, 495]),          # 100% density: dense attention
     ("clip16x9_rho1_2", [3], [1, 300]),
+    ("clip16x9_rho1_5", [30], [2, 251, 494]),         # 20%: rows of 99 and 100 key tiles
+    ("clip16x9_rho1_20", [21], [0, 123, 495]),        # 5%: rows of 24 and 25 key tiles
+    ("len_T15", [5, 38], [0, 120, 239]),              # 24k tokens, nT = 240
     ("len_T62", [11], [0, 500, 991]),                 # 100k tokens, nT = 992
 ])
 def test_sweep_extremes_sampled(name, heads, rows):
     w = synth.get(name)
     attn = [(0, 0, r) for r in rows]
     _end_to_end(w, heads=heads, rows=rows, attn_rows=attn)
+
+
+def test_stages_length_sweep_24k():
+    # the 24k-token point of the length sweep (15 frames of 30 x 54, nT = 240), stage by stage
+    _stage_run(synth.sweep_length(15), heads=[0, 22, 39],
+               attn_rows=[(0, j, r) for j in range(3) for r in (0, 1, 119, 239)])
+
+
+def test_density_one_twentieth_rows_of_only_the_diagonal():
+    """Density 1/20 over 32 key tiles is 1.6 tiles per row: Bresenham gives rows of 1 and 2
+    tiles, and a row whose budget is 1 holds its own (diagonal) tile alone. Checked stage by
+    stage and end to end against the oracle, then row by row on the GPU's lists."""
+    V = P.veda()
+    w = synth.Workload("short_rho1_20", 12, B=1, H=4, grid=(2, 30, 54),
+                       head_shapes=((1, 8, 16),) * 4, rho=((1, 20),))
+    assert w.nT == 32
+    _stage_run(w)
+    _end_to_end(w)
+    inp = synth.make_inputs(w)
+    slots, nv, seg, nTh = P.oracle_maps(w, None)
+    maps = V.build_tile_map(w.grid, w.head_shapes).to(DEV)
+    bufs = V.sparse_attention(inp.q.to(DEV), inp.k.to(DEV), inp.v.to(DEV), inp.wq.to(DEV),
+                              inp.wk.to(DEV), maps, w.rho, P.SCALE)
+    V.check_device_status()
+    k = O.budgets(nTh[0], seg[0], w.rho).sum(axis=1)
+    ones = np.flatnonzero(k == 1)
+    assert len(ones) >= 10 and set(k.tolist()) == {1, 2}
+    fc, fi = bufs.lists.full_cnt.cpu().numpy(), bufs.lists.full_idx.cpu().numpy()
+    pc, pi = bufs.lists.part_cnt.cpu().numpy(), bufs.lists.part_idx.cpu().numpy()
+    for h in range(w.H):
+        for r in ones:
+            got = sorted(fi[0, h, r, :fc[0, h, r]].tolist() + pi[0, h, r, :pc[0, h, r]].tolist())
+            assert got == [r], (h, r, got)
 
 
 def test_bounded_wait_runs_out_and_context_survives():
