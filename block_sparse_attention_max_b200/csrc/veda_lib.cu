@@ -84,6 +84,7 @@ veda_status current_device(int& sms) {
         {reinterpret_cast<const void*>(fp8::attn_fwd_fp8_kernel), static_cast<int>(fp8::kSmemBytes)},
         {reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDQ>), static_cast<int>(bwd::kSmemBytesDQ)},
         {reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDKDV>), static_cast<int>(bwd::kSmemBytesDKDV)},
+        {reinterpret_cast<const void*>(sgemm::nt_gemm_3xtf32_kernel), static_cast<int>(sgemm::kSmemBytes)},
     };
     for (auto& x : attrs) {
       e = cudaFuncSetAttribute(x.f, cudaFuncAttributeMaxDynamicSharedMemorySize, x.bytes);
@@ -158,6 +159,20 @@ veda_status encode_rows8(CUtensorMap& m, const void* base, uint64_t rows) {
   const cuuint32_t box[2] = {128, 128};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(r) + ")");
+  return VEDA_OK;
+}
+
+// fp32 matrix of `cols` columns (row stride cols * 4 bytes, a multiple of 16) and `rows` rows:
+// box 32 columns (128 bytes) x 128 rows, 128-byte swizzle. Rows past the end read as zero.
+veda_status encode_f32_rows(CUtensorMap& m, const void* base, uint64_t cols, uint64_t rows) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 4};
+  const cuuint32_t box[2] = {32, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(VEDA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(r) + ")");
@@ -288,34 +303,42 @@ veda_status veda_block_scores(const float* pooled_q, const float* pooled_k, cons
   int sms;
   veda_status st = current_device(sms);
   if (st != VEDA_OK) return st;
+  if ((st = get_encoder()) != VEDA_OK) return st;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  float* hat = static_cast<float*>(workspace);             // [2][B][H][nT][128]
-  const int64_t per = static_cast<int64_t>(nT) * 128;
+  float* hat = static_cast<float*>(workspace);             // [2][B][H][nT][128]: qhat, khat
+  const int64_t BH = static_cast<int64_t>(B) * H;
+  const int32_t tiles_m = (nT + 127) / 128;
   // projection: hat[which] = mean + pooled . W^T   (M = nT, N = 128, K = 384)
-  NtGemmArgs p{};
-  p.a0[0] = pooled_q; p.a0[1] = pooled_k;
-  p.b0[0] = Wq; p.b0[1] = Wk;
-  p.r0[0] = pooled_q; p.r0[1] = pooled_k;                  // mean = first 128 of each row
-  p.c0 = hat;
-  p.a_bh = static_cast<int64_t>(nT) * 384; p.b_h = 128 * 384; p.b_b = 0; p.r_bh = p.a_bh; p.c_z = per;
-  p.lda = 384; p.ldb = 384; p.ldr = 384; p.ldc = 128;
-  p.M = nT; p.N = 128; p.K = 384; p.B = B; p.H = H;
-  dim3 gp(128 / kGemmBN, (nT + kGemmBM - 1) / kGemmBM, 2 * B * H);
-  nt_gemm_kernel<<<gp, kGemmThreads, 0, s>>>(p);
+  CUtensorMap mPq, mPk, mWq, mWk;
+  if ((st = encode_f32_rows(mPq, pooled_q, 384, static_cast<uint64_t>(BH) * nT)) != VEDA_OK ||
+      (st = encode_f32_rows(mPk, pooled_k, 384, static_cast<uint64_t>(BH) * nT)) != VEDA_OK ||
+      (st = encode_f32_rows(mWq, Wq, 384, static_cast<uint64_t>(H) * 128)) != VEDA_OK ||
+      (st = encode_f32_rows(mWk, Wk, 384, static_cast<uint64_t>(H) * 128)) != VEDA_OK)
+    return st;
+  sgemm::Args p{};
+  p.mode = sgemm::kModeProject;
+  p.nT = nT; p.N = 128; p.k_chunks = 384 / 32;
+  p.tiles_m = tiles_m; p.tiles_n = 1;
+  p.BH = static_cast<int32_t>(BH); p.H = H;
+  p.tiles = 2 * BH * tiles_m;
+  p.res[0] = pooled_q; p.res[1] = pooled_k;             // mean = first 128 of each 384-row
+  p.out = hat;
+  sgemm::nt_gemm_3xtf32_kernel<<<grid_for(p.tiles, sms, 1), sgemm::kThreads, sgemm::kSmemBytes, s>>>(
+      mPq, mPk, mWq, mWk, p);
   st = launched("projection");
   if (st != VEDA_OK) return st;
   // scores = qhat . khat^T  (M = N = nT, K = 128)
-  NtGemmArgs q{};
-  q.a0[0] = hat; q.a0[1] = hat;
-  q.b0[0] = hat + static_cast<int64_t>(B) * H * per; q.b0[1] = q.b0[0];
-  q.r0[0] = nullptr; q.r0[1] = nullptr;
-  q.c0 = scores;
-  q.a_bh = per; q.b_h = per; q.b_b = static_cast<int64_t>(H) * per; q.r_bh = 0;
-  q.c_z = static_cast<int64_t>(nT) * nT;
-  q.lda = 128; q.ldb = 128; q.ldr = 0; q.ldc = nT;
-  q.M = nT; q.N = nT; q.K = 128; q.B = B; q.H = H;
-  dim3 gq((nT + kGemmBN - 1) / kGemmBN, (nT + kGemmBM - 1) / kGemmBM, B * H);
-  nt_gemm_kernel<<<gq, kGemmThreads, 0, s>>>(q);
+  CUtensorMap mHat;
+  if ((st = encode_f32_rows(mHat, hat, 128, static_cast<uint64_t>(2 * BH) * nT)) != VEDA_OK) return st;
+  sgemm::Args q{};
+  q.mode = sgemm::kModeScores;
+  q.nT = nT; q.N = nT; q.k_chunks = 128 / 32;
+  q.tiles_m = tiles_m; q.tiles_n = tiles_m;
+  q.BH = static_cast<int32_t>(BH); q.H = H;
+  q.tiles = BH * tiles_m * tiles_m;
+  q.out = scores;
+  sgemm::nt_gemm_3xtf32_kernel<<<grid_for(q.tiles, sms, 1), sgemm::kThreads, sgemm::kSmemBytes, s>>>(
+      mHat, mHat, mHat, mHat, q);
   return launched("scores");
 }
 

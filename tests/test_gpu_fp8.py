@@ -66,7 +66,7 @@ def _tiny_mass(qd, kd, nv, lists, rows, scale):
     return out
 
 
-def _run(w, heads, rows=None):
+def _run(w, heads, rows=None, exact=False):
     V = P.veda()
     inp = synth.make_inputs(w)
     orders = inp.tile_order
@@ -117,7 +117,18 @@ def _run(w, heads, rows=None):
         assert np.all(dl <= 2e-3 + 1e-5 * np.abs(lse_ref[b, j, sl])), f"LSE differs by {dl.max():.3g}"
     e, bd = np.concatenate(errs), np.concatenate(bands)
     assert e.mean() <= 0.5 * bd.mean(), (e.mean(), bd.mean())
-    return float(e.max()), float(e.mean())
+    if not exact:
+        return float(e.max()), float(e.mean())
+    # distance from the method's result: the oracle's attention of the unquantised (bf16) inputs
+    o_x, _ = O.attention(qt, kt, vt, nv[heads], lists_h, P.SCALE, rows=todo)
+    tiles = [(b, j, slice(r * 128, (r + 1) * 128)) for (b, j, r) in todo]
+    g_x = np.concatenate([np.abs(og[b, j, sl] - o_x[b, j, sl]).ravel() for (b, j, sl) in tiles])
+    q_x = np.concatenate([np.abs(o_ref[b, j, sl] - o_x[b, j, sl]).ravel() for (b, j, sl) in tiles])
+    assert np.all(g_x <= q_x + bd)      # |G - A_x| <= |A_q - A_x| + |G - A_q|, elementwise
+    mag = float(np.concatenate([np.abs(o_x[b, j, sl]).ravel() for (b, j, sl) in tiles]).mean())
+    return dict(gpu_vs_exact_mean=float(g_x.mean()), gpu_vs_exact_max=float(g_x.max()),
+                quant_vs_exact_mean=float(q_x.mean()), quant_vs_exact_max=float(q_x.max()),
+                p_band_mean=float(bd.mean()), mean_abs_o=mag)
 
 
 def test_fp8_tiny():
@@ -143,6 +154,24 @@ def test_fp8_clip16x9_sampled():
     """The 16:9 clip at full size (40 heads launched, the benchmark's configuration): codes and
     scales of two heads bit-exact, attention of three query tiles of each against the oracle."""
     _run(synth.CLIP16x9, [0, 39], rows=[0, 247, 495])
+
+
+@pytest.mark.parametrize("name,heads,rows", [("small", [0, 3, 6], None), ("clip16x9", [5, 30], [0, 100, 333, 495])])
+def test_fp8_distance_from_unquantised_attention(name, heads, rows):
+    """How far the FP8 variant's output sits from the method's own result, the fp64 attention
+    of the unquantised bf16 inputs over the same lists. Two errors add up: rounding Q, K and V
+    to e4m3 (3 mantissa bits: up to 2^-4 relative per element, worst on the Q K^T products),
+    which the oracle measures by itself as |attention(dequantised) - attention(bf16)|, and the
+    kernel's own e4m3 P (the band of the other tests). Bounds: elementwise, the error is at
+    most the quantisation's error plus the P band; the mean error may exceed the
+    quantisation's mean error by at most half the P band's mean; and on these smoothed-field
+    inputs the mean error stays below 8% of mean |O| (the oracle's quantisation alone gives
+    ~5.5%). Per-tile instead of per-(batch, head) scales would not help: e4m3 is a floating
+    format, so a smaller scale changes only values near its subnormal range (the oracle gives
+    0.0124 mean error per head and 0.0124 per tile on the small workload)."""
+    r = _run(synth.get(name), heads, rows=rows, exact=True)
+    assert r["gpu_vs_exact_mean"] <= r["quant_vs_exact_mean"] + 0.5 * r["p_band_mean"], r
+    assert r["gpu_vs_exact_mean"] <= 0.08 * r["mean_abs_o"], r
 
 
 def test_quantize_zero_tensor_negative_zero_and_large_values():
