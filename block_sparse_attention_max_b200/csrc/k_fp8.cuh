@@ -22,6 +22,7 @@
 #pragma once
 
 #include "k_attn.cuh"
+#include "k_heat.cuh"
 
 namespace veda {
 namespace fp8 {
@@ -394,6 +395,12 @@ __device__ __forceinline__ void role_pv_issuer(Bars& bars, uint32_t sb, uint32_t
   mbar_wait(smem_u32(&bars.drain[1]), 0, nullptr, 125);
 }
 
+// Column groups k (bit k) whose exponentials run on the FMA pipe (heat::exp2_fma_x2) instead
+// of the MUFU, for a thread's first row (r0) and second row (r0 + 8): the MUFU sets the pace
+// of this softmax while the FMA pipe is mostly idle.
+constexpr uint32_t kFmaExpRow0 = 0x0000u;
+constexpr uint32_t kFmaExpRow1 = 0xAAAAu;
+
 // Softmax warps: the bf16 kernel's 16-row layout (thread: rows r0 = base + lane / 4 and
 // r0 + 8, of every 8-column group k the columns 8k + 2c + {0, 1}, c = lane % 4). One pass
 // takes the exponentials with the block's row maxima; P goes to tensor memory as e4m3 words.
@@ -493,10 +500,23 @@ __device__ __forceinline__ void softmax_role(const Args& p, Bars& bars, uint32_t
             a4[k & 3] = fmax3(a4[k & 3], __uint_as_float(s[4 * k]), __uint_as_float(s[4 * k + 1]));
             b4[k & 3] = fmax3(b4[k & 3], __uint_as_float(s[4 * k + 2]), __uint_as_float(s[4 * k + 3]));
           }
-          float x0, x1, y0, y1;
-          f2_unpack(f2_fma(f2_pack(s[4 * k], s[4 * k + 1]), c2, nm0), x0, x1);
-          f2_unpack(f2_fma(f2_pack(s[4 * k + 2], s[4 * k + 3]), c2, nm1), y0, y1);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), q0 = ex2_approx(y0), q1 = ex2_approx(y1);
+          const uint64_t xx = f2_fma(f2_pack(s[4 * k], s[4 * k + 1]), c2, nm0);
+          const uint64_t yy = f2_fma(f2_pack(s[4 * k + 2], s[4 * k + 3]), c2, nm1);
+          float p0, p1, q0, q1;
+          if ((kFmaExpRow0 >> k) & 1) {
+            heat::exp2_fma_x2(xx, p0, p1);
+          } else {
+            f2_unpack(xx, p0, p1);
+            p0 = ex2_approx(p0);
+            p1 = ex2_approx(p1);
+          }
+          if ((kFmaExpRow1 >> k) & 1) {
+            heat::exp2_fma_x2(yy, q0, q1);
+          } else {
+            f2_unpack(yy, q0, q1);
+            q0 = ex2_approx(q0);
+            q1 = ex2_approx(q1);
+          }
           acc0[k & 1] = f2_add(acc0[k & 1], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
           acc1[k & 1] = f2_add(acc1[k & 1], f2_pack(__float_as_uint(q0), __float_as_uint(q1)));
           const uint32_t e0 = pack_e4m3x2(p0, p1), e1 = pack_e4m3x2(q0, q1);

@@ -196,9 +196,11 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const PoolArgs a) {
 // ------------------------------------------------------------------------------------
 // Steps 1 + 2 fused (a variant; the two calls also stay separate): gather a tile as
 // permute_kernel does and reduce mean / max / min over its valid slots on the way, so the
-// tiled tensor is not read a second time. Thread t holds channels 8 (t & 15) .. + 7 of rows
-// (t >> 4) + 16 i; the two row groups of a warp are combined by one shuffle, the eight warps
-// through shared memory.
+// tiled tensor is not read a second time. One warp per tile, as in pool_kernel: lane l
+// moves 16-byte chunk (l & 15) of rows (l >> 4) + 2 i, 16 rows per pass, and keeps the
+// running sums / maxima / minima of its eight channels in registers; one shuffle combines
+// the two row groups at the end. No shared memory and no block barrier, so the warps of a
+// CTA never wait for one another and the gather stream does not stall between tiles.
 // ------------------------------------------------------------------------------------
 struct PermPoolArgs {
   GatherArgs g;
@@ -206,47 +208,53 @@ struct PermPoolArgs {
   float* pooled;          // [B][H][nT][3][128]
 };
 
-__global__ void __launch_bounds__(kCopyThreads) permute_pool_kernel(const PermPoolArgs p) {
-  __shared__ float red[kCopyThreads / 32][3][128];
+__global__ void __launch_bounds__(kPoolThreads) permute_pool_kernel(const PermPoolArgs p) {
   const GatherArgs& a = p.g;
-  const uint32_t c = threadIdx.x & 15, r0 = threadIdx.x >> 4, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int64_t u = blockIdx.x; u < a.units; u += gridDim.x) {
+  const uint32_t lane = threadIdx.x & 31;
+  const uint32_t c = lane & 15, half = lane >> 4;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (kPoolThreads / 32);
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * (kPoolThreads / 32) + (threadIdx.x >> 5); u < a.units;
+       u += warps) {
     int32_t b, h, t;
     unit_coords(u, a.H, a.nT, b, h, t);
     const int64_t lin = (static_cast<int64_t>(b) * a.H + h) * a.nT + t;   // tile index in memory
     int32_t nv = p.valid[static_cast<int64_t>(h) * a.nT + t];
     nv = nv < 0 ? 0 : (nv > 128 ? 128 : nv);
-    const int32_t* m = a.map + static_cast<int64_t>(h) * a.Npad + static_cast<int64_t>(t) * 128;
-    int32_t tok[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) tok[i] = __ldg(m + r0 + 16 * i);
-    uint4 v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[i] = make_uint4(0, 0, 0, 0);
-      if (tok[i] >= a.N) flag_status(ST_BAD_MAP);
-      if (tok[i] >= 0 && tok[i] < a.N)
-        v[i] = ld_stream(a.src + ((static_cast<int64_t>(b) * a.N + tok[i]) * a.H + h) * kRowBytes + c * 16);
-    }
-    uint8_t* dst = a.dst + ((static_cast<int64_t>(b) * a.H + h) * a.Npad + static_cast<int64_t>(t) * 128) * kRowBytes;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) st_v4(dst + (r0 + 16 * i) * kRowBytes + c * 16, v[i]);
+    const int32_t* m = a.map + static_cast<int64_t>(h) * a.Npad + static_cast<int64_t>(t) * 128 + half;
+    const uint8_t* src = a.src + (static_cast<int64_t>(b) * a.N * a.H + h) * kRowBytes + c * 16;
+    const int64_t tok_stride = static_cast<int64_t>(a.H) * kRowBytes;
+    uint8_t* dst = a.dst + lin * kTileBytes + half * kRowBytes + c * 16;
     float sum[8], mx[8], mn[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) { sum[k] = 0.f; mx[k] = -INFINITY; mn[k] = INFINITY; }
+#pragma unroll 1
+    for (int32_t r0 = 0; r0 < 128; r0 += 16) {
+      int32_t tok[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (static_cast<int32_t>(r0 + 16 * i) < nv) {
-        const __nv_bfloat162* q = reinterpret_cast<const __nv_bfloat162*>(&v[i]);
+      for (int i = 0; i < 8; ++i) tok[i] = __ldg(m + r0 + 2 * i);
+      uint4 v[8];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 f = __bfloat1622float2(q[k]);
-          sum[2 * k] += f.x;
-          sum[2 * k + 1] += f.y;
-          mx[2 * k] = fmaxf(mx[2 * k], f.x);
-          mx[2 * k + 1] = fmaxf(mx[2 * k + 1], f.y);
-          mn[2 * k] = fminf(mn[2 * k], f.x);
-          mn[2 * k + 1] = fminf(mn[2 * k + 1], f.y);
+      for (int i = 0; i < 8; ++i) {
+        v[i] = make_uint4(0, 0, 0, 0);
+        if (tok[i] >= a.N) flag_status(ST_BAD_MAP);
+        if (tok[i] >= 0 && tok[i] < a.N) v[i] = ld_stream(src + tok[i] * tok_stride);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) st_v4(dst + (r0 + 2 * i) * kRowBytes, v[i]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (r0 + static_cast<int32_t>(half) + 2 * i < nv) {
+          const __nv_bfloat162* q = reinterpret_cast<const __nv_bfloat162*>(&v[i]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(q[k]);
+            sum[2 * k] += f.x;
+            sum[2 * k + 1] += f.y;
+            mx[2 * k] = fmaxf(mx[2 * k], f.x);
+            mx[2 * k + 1] = fmaxf(mx[2 * k + 1], f.y);
+            mn[2 * k] = fminf(mn[2 * k], f.x);
+            mn[2 * k + 1] = fminf(mn[2 * k + 1], f.y);
+          }
         }
       }
     }
@@ -256,30 +264,21 @@ __global__ void __launch_bounds__(kCopyThreads) permute_pool_kernel(const PermPo
       mx[k] = fmaxf(mx[k], __shfl_xor_sync(0xffffffffu, mx[k], 16));
       mn[k] = fminf(mn[k], __shfl_xor_sync(0xffffffffu, mn[k], 16));
     }
-    if (lane < 16) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        red[warp][0][c * 8 + k] = sum[k];
-        red[warp][1][c * 8 + k] = mx[k];
-        red[warp][2][c * 8 + k] = mn[k];
+    if (half == 0) {
+      float4* o = reinterpret_cast<float4*>(p.pooled + lin * 384 + c * 8);
+      if (nv > 0) {
+        const float inv = 1.0f / static_cast<float>(nv);
+        o[0] = make_float4(sum[0] * inv, sum[1] * inv, sum[2] * inv, sum[3] * inv);
+        o[1] = make_float4(sum[4] * inv, sum[5] * inv, sum[6] * inv, sum[7] * inv);
+        o[32] = make_float4(mx[0], mx[1], mx[2], mx[3]);
+        o[33] = make_float4(mx[4], mx[5], mx[6], mx[7]);
+        o[64] = make_float4(mn[0], mn[1], mn[2], mn[3]);
+        o[65] = make_float4(mn[4], mn[5], mn[6], mn[7]);
+      } else {
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        o[0] = z; o[1] = z; o[32] = z; o[33] = z; o[64] = z; o[65] = z;
       }
     }
-    __syncthreads();
-    if (threadIdx.x < 128) {
-      const uint32_t ch = threadIdx.x;
-      float s_ = 0.f, x_ = -INFINITY, n_ = INFINITY;
-#pragma unroll
-      for (int w = 0; w < kCopyThreads / 32; ++w) {
-        s_ += red[w][0][ch];
-        x_ = fmaxf(x_, red[w][1][ch]);
-        n_ = fminf(n_, red[w][2][ch]);
-      }
-      float* o = p.pooled + lin * 384;
-      o[ch] = nv > 0 ? s_ / static_cast<float>(nv) : 0.f;
-      o[128 + ch] = nv > 0 ? x_ : 0.f;
-      o[256 + ch] = nv > 0 ? n_ : 0.f;
-    }
-    __syncthreads();
   }
 }
 

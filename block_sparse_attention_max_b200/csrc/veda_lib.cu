@@ -109,7 +109,7 @@ veda_status current_device(int& sms) {
     if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_copy, permute_kernel, kCopyThreads, 0)) != cudaSuccess ||
         (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_unpermute, unpermute_kernel, kCopyThreads, 0)) != cudaSuccess ||
         (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_pool, pool_kernel, kPoolThreads, 0)) != cudaSuccess ||
-        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_permpool, permute_pool_kernel, kCopyThreads, 0)) != cudaSuccess)
+        (e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.per_sm_permpool, permute_pool_kernel, kPoolThreads, 0)) != cudaSuccess)
       return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     d.per_sm_copy = d.per_sm_copy < 1 ? 1 : d.per_sm_copy;
     d.per_sm_unpermute = d.per_sm_unpermute < 1 ? 1 : d.per_sm_unpermute;
@@ -246,7 +246,8 @@ veda_status veda_permute_pool(const void* x, void* x_tiled, const int32_t* tile_
   PermPoolArgs p{{static_cast<const uint8_t*>(x), static_cast<uint8_t*>(x_tiled), tile_map, B, N, H, Npad,
                   Npad / 128, static_cast<int64_t>(B) * H * (Npad / 128)},
                  tile_valid, pooled};
-  permute_pool_kernel<<<grid_for(p.g.units, sms, device_info().per_sm_permpool), kCopyThreads, 0,
+  const int64_t pp_ctas = (p.g.units + kPoolThreads / 32 - 1) / (kPoolThreads / 32);
+  permute_pool_kernel<<<grid_for(pp_ctas, sms, device_info().per_sm_permpool), kPoolThreads, 0,
                         reinterpret_cast<cudaStream_t>(stream)>>>(p);
   return launched("permute_pool_kernel");
 }
