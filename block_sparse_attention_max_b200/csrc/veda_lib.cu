@@ -322,7 +322,6 @@ veda_status veda_block_scores(const float* pooled_q, const float* pooled_k, cons
   p.tiles_m = tiles_m; p.tiles_n = 1;
   p.BH = static_cast<int32_t>(BH); p.H = H;
   p.tiles = 2 * BH * tiles_m;
-  p.res[0] = pooled_q; p.res[1] = pooled_k;             // mean = first 128 of each 384-row
   p.out = hat;
   sgemm::nt_gemm_3xtf32_kernel<<<grid_for(p.tiles, sms, 1), sgemm::kThreads, sgemm::kSmemBytes, s>>>(
       mPq, mPk, mWq, mWk, p);

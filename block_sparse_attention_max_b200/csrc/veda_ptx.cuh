@@ -264,14 +264,6 @@ __host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
          | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// fp32 -> tf32 (10 explicit mantissa bits), round to nearest with ties away from zero; the
-// result is an fp32 bit pattern whose low 13 bits are zero.
-__device__ __forceinline__ float tf32_round(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return __uint_as_float(r);
-}
-
 // 32 lanes x 32 columns of 32-bit tensor memory -> 32 registers per thread.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
