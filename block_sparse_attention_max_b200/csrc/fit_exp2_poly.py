@@ -1,5 +1,5 @@
-"""Coefficients of the degree-4 polynomial for 2^f, f in [-1/2, 1/2], used by the block-heat
-kernel's FMA-pipe exponentials (k_heat.cuh, exp2_fma_x2).
+"""Coefficients of the degree-4 polynomial for 2^f, f in [-1/2, 1/2], used by the softmax
+kernels' FMA-pipe exponentials (veda_ptx.cuh, exp2_fma_x2).
 
 Relative error is minimised by least squares at Chebyshev nodes, reweighted by Lawson's
 iteration (weights multiplied by the current error) toward the minimax fit. Prints the

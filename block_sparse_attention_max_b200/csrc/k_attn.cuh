@@ -21,6 +21,8 @@
 //   warp 9       Q K^T issuer (one thread): S_b = Q K_j^T, b = block parity, once every
 //                softmax warp has taken S(j-2) out of buffer b
 //   warp 10      P V issuer (one thread): O += P_b V_j, P_b read from tensor memory
+// An eighth of the exponentials (the second row of every fourth column group) run on the FMA
+// pipe (exp2_fma_x2) instead of the MUFU, whose rate sets the pace of the softmax.
 // Tensor memory (512 columns): S0 | S1 | O | P0 | P1. With two S buffers, each freed as
 // soon as the softmax holds it in registers, and P in buffers of its own, the tensor core
 // computes S(j+1) and P V(j-1) while the softmax works on block j. The running maximum (in
@@ -326,10 +328,18 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
             a4[k & 3] = fmax3(a4[k & 3], __uint_as_float(s[4 * k]), __uint_as_float(s[4 * k + 1]));
             b4[k & 3] = fmax3(b4[k & 3], __uint_as_float(s[4 * k + 2]), __uint_as_float(s[4 * k + 3]));
           }
-          float x0, x1, y0, y1;
+          float x0, x1, q0, q1;
           f2_unpack(f2_fma(f2_pack(s[4 * k], s[4 * k + 1]), c2, nm0), x0, x1);
-          f2_unpack(f2_fma(f2_pack(s[4 * k + 2], s[4 * k + 3]), c2, nm1), y0, y1);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), q0 = ex2_approx(y0), q1 = ex2_approx(y1);
+          const uint64_t yy = f2_fma(f2_pack(s[4 * k + 2], s[4 * k + 3]), c2, nm1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          if ((k & 3) == 3) {   // an eighth of the exponentials on the FMA pipe
+            exp2_fma_x2(yy, q0, q1);
+          } else {
+            float y0, y1;
+            f2_unpack(yy, y0, y1);
+            q0 = ex2_approx(y0);
+            q1 = ex2_approx(y1);
+          }
           acc0[k & 1] = f2_add(acc0[k & 1], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
           acc1[k & 1] = f2_add(acc1[k & 1], f2_pack(__float_as_uint(q0), __float_as_uint(q1)));
           pk[2 * k] = pack_bf16x2(p0, p1);

@@ -20,10 +20,19 @@
 
 namespace veda {
 
-constexpr int kSelWarps = 2;                   // query rows per CTA
+constexpr int kSelWarps = 8;                   // query rows per CTA
 constexpr int kSelThreads = 32 * kSelWarps;
 constexpr int kSelMaxTiles = 2048;
 constexpr int kMaxSeg = 4;
+
+// Shared memory of one warp, sized to the launch's tile count and segments (so that short
+// rows leave room for more resident warps): rank images [nT], segment ids [nT] (bytes,
+// rounded to 16), one 256-bin histogram per segment.
+__host__ __device__ constexpr uint32_t sel_warp_bytes(int32_t nT, int32_t n_seg) {
+  return static_cast<uint32_t>(nT) * 4u + ((static_cast<uint32_t>(nT) + 15u) & ~15u) +
+         static_cast<uint32_t>(n_seg) * 1024u;
+}
+constexpr uint32_t kSelMaxSmem = kSelWarps * sel_warp_bytes(kSelMaxTiles, kMaxSeg);
 
 struct SelectArgs {
   const float* scores;          // [B][H][nT][nT]
@@ -56,11 +65,12 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a) {
-  __shared__ uint32_t s_u[kSelWarps][kSelMaxTiles];
-  __shared__ uint8_t s_seg[kSelWarps][kSelMaxTiles];
-  __shared__ uint32_t s_hist[kSelWarps][kMaxSeg][256];
-
+  extern __shared__ __align__(16) uint8_t sel_smem[];
   const int w = threadIdx.x >> 5;
+  uint8_t* wbase = sel_smem + static_cast<uint32_t>(w) * sel_warp_bytes(a.nT, a.n_seg);
+  uint32_t* su = reinterpret_cast<uint32_t*>(wbase);
+  uint8_t* ss = wbase + static_cast<uint32_t>(a.nT) * 4u;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(ss + ((static_cast<uint32_t>(a.nT) + 15u) & ~15u));
   const uint32_t lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kSelWarps + w;
   if (row >= static_cast<int64_t>(a.B) * a.H * a.nT) return;
@@ -79,8 +89,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
   const int32_t* seg_h = a.segment + static_cast<int64_t>(h) * a.nT;
   const int32_t* val_h = a.valid + static_cast<int64_t>(h) * a.nT;
   const float* srow = a.scores + row * a.nT;
-  uint32_t* su = s_u[w];
-  uint8_t* ss = s_seg[w];
 
   // candidates -> shared memory; tiles per segment
   int32_t cnt[kMaxSeg] = {0, 0, 0, 0};
@@ -128,12 +136,12 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
   for (int d = 3; d >= 0; --d) {
     const int shift = 8 * d;
     const uint32_t hi_mask = d == 3 ? 0u : (0xFFFFFFFFu << (shift + 8));
-    for (int i = static_cast<int>(lane); i < nseg * 256; i += 32) (&s_hist[w][0][0])[i] = 0;
+    for (int i = static_cast<int>(lane); i < nseg * 256; i += 32) hist[i] = 0;
     __syncwarp();
     for (int32_t j = static_cast<int32_t>(lane); j < n; j += 32) {
       const uint32_t u = su[j];
       const int sg = ss[j];
-      if (k[sg] > 0 && (u & hi_mask) == prefix[sg]) atomicAdd(&s_hist[w][sg][(u >> shift) & 255u], 1u);
+      if (k[sg] > 0 && (u & hi_mask) == prefix[sg]) atomicAdd(&hist[sg * 256 + ((u >> shift) & 255u)], 1u);
     }
     __syncwarp();
 #pragma unroll
@@ -142,7 +150,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
       uint32_t c8[8];
       uint32_t local = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) { c8[i] = s_hist[w][s][lane * 8 + i]; local += c8[i]; }
+      for (int i = 0; i < 8; ++i) { c8[i] = hist[s * 256 + lane * 8 + i]; local += c8[i]; }
       uint32_t incl = local;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {

@@ -85,6 +85,7 @@ veda_status current_device(int& sms) {
         {reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDQ>), static_cast<int>(bwd::kSmemBytesDQ)},
         {reinterpret_cast<const void*>(bwd::bwd_kernel<bwd::kModeDKDV>), static_cast<int>(bwd::kSmemBytesDKDV)},
         {reinterpret_cast<const void*>(sgemm::nt_gemm_3xtf32_kernel), static_cast<int>(sgemm::kSmemBytes)},
+        {reinterpret_cast<const void*>(select_kernel), static_cast<int>(kSelMaxSmem)},
     };
     for (auto& x : attrs) {
       e = cudaFuncSetAttribute(x.f, cudaFuncAttributeMaxDynamicSharedMemorySize, x.bytes);
@@ -440,8 +441,8 @@ veda_status veda_select_blocks(const float* scores, const int32_t* tile_valid, c
   }
   const int64_t rows = static_cast<int64_t>(B) * H * nT;
   if (rows > INT32_MAX) return fail(VEDA_ERR_INVALID_ARG, "veda_select_blocks: too many rows");
-  select_kernel<<<static_cast<unsigned>((rows + kSelWarps - 1) / kSelWarps), kSelThreads, 0,
-                  reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  select_kernel<<<static_cast<unsigned>((rows + kSelWarps - 1) / kSelWarps), kSelThreads,
+                  kSelWarps * sel_warp_bytes(nT, n_segments), reinterpret_cast<cudaStream_t>(stream)>>>(a);
   return launched("select_kernel");
 }
 

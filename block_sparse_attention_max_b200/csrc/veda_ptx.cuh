@@ -347,6 +347,36 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x for a pair of fp32 values on the FMA pipe, so that part of a softmax's exponentials
+// leave the MUFU, which sets the pace of the attention, FP8 attention and block-heat loops. Range reduction x = j + f with
+// j = round(x) (adding 1.5 * 2^23 + 127 rounds x to an integer and leaves j + 127 in the low
+// mantissa bits), 2^f on [-1/2, 1/2] by a degree-4 polynomial fitted for relative error
+// (Lawson-reweighted least squares, csrc/fit_exp2_poly.py; max relative error 2.6e-6, 5.3e-6
+// with fp32 rounding), and 2^j as the float whose exponent field is j + 127. x is clamped at
+// -127, where that field is 0: -inf and results below 2^-126 give exactly 0, as ex2.approx.ftz.
+constexpr float kExp2C0 = 0.9999992847442627f, kExp2C1 = 0.6931217908859253f, kExp2C2 = 0.240247443318367f,
+                kExp2C3 = 0.05591785907745361f, kExp2C4 = 0.009570101276040077f;
+constexpr float kExp2Shift = 12582912.0f + 127.0f;
+__device__ __forceinline__ uint64_t f2_splat(float v) { return f2_pack(__float_as_uint(v), __float_as_uint(v)); }
+__device__ __forceinline__ void exp2_fma_x2(uint64_t xx, float& r0, float& r1) {
+  float x0, x1;
+  f2_unpack(xx, x0, x1);
+  x0 = fmaxf(x0, -127.0f);
+  x1 = fmaxf(x1, -127.0f);
+  const uint64_t xc = f2_pack(__float_as_uint(x0), __float_as_uint(x1));
+  const uint64_t t = f2_add(xc, f2_splat(kExp2Shift));
+  const uint64_t j = f2_add(t, f2_splat(-kExp2Shift));          // exact: round(x)
+  const uint64_t f = f2_fma(j, f2_splat(-1.0f), xc);             // exact: x - j
+  uint64_t p = f2_fma(f2_splat(kExp2C4), f, f2_splat(kExp2C3));
+  p = f2_fma(p, f, f2_splat(kExp2C2));
+  p = f2_fma(p, f, f2_splat(kExp2C1));
+  p = f2_fma(p, f, f2_splat(kExp2C0));
+  float t0, t1;
+  f2_unpack(t, t0, t1);
+  const uint64_t sc = f2_pack(__float_as_uint(t0) << 23, __float_as_uint(t1) << 23);   // 2^j
+  f2_unpack(f2_mul(p, sc), r0, r1);
+}
+
 // Two fp32 values to e4m3 (round to nearest even, saturating at +-448); lo in the low byte.
 __device__ __forceinline__ uint16_t pack_e4m3x2(float lo, float hi) {
   uint16_t d;

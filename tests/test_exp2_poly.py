@@ -1,4 +1,4 @@
-"""The block-heat kernel's FMA-pipe exponential (k_heat.cuh, exp2_fma_x2), pinned on the CPU
+"""The softmax kernels' FMA-pipe exponential (veda_ptx.cuh, exp2_fma_x2), pinned on the CPU
 against the exact 2^x: its constants are read from the kernel source and its steps are
 emulated in fp32 (each fused multiply-add rounded once, from the exact fp64 product)."""
 import math
@@ -11,7 +11,7 @@ SRC = pathlib.Path(__file__).resolve().parents[1] / "block_sparse_attention_max_
 
 
 def _constants():
-    text = (SRC / "k_heat.cuh").read_text()
+    text = (SRC / "veda_ptx.cuh").read_text()
     c = [float(re.search(rf"kExp2C{k} = ([0-9.e-]+)f", text).group(1)) for k in range(5)]
     shift = re.search(r"kExp2Shift = ([0-9.]+)f \+ ([0-9.]+)f", text)
     return np.array(c, dtype=np.float32), np.float32(float(shift.group(1)) + float(shift.group(2)))
