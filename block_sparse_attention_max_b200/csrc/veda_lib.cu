@@ -128,6 +128,28 @@ const DeviceInfo& device_info() {
   return g_dev[dev];
 }
 
+// The library's second stream of the current device and a fork / join event pair, created on
+// first use and kept until exit (the backward runs its two independent kernels on both).
+veda_status side_stream(cudaStream_t& s, cudaEvent_t& fork, cudaEvent_t& join) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(VEDA_ERR_UNSUPPORTED, "device ordinal out of range");
+  static cudaStream_t streams[kMaxDevices] = {};
+  static cudaEvent_t forks[kMaxDevices] = {}, joins[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (streams[dev] == nullptr) {
+    if ((e = cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&forks[dev], cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&joins[dev], cudaEventDisableTiming)) != cudaSuccess)
+      return cuda_fail(e, "side stream");
+  }
+  s = streams[dev];
+  fork = forks[dev];
+  join = joins[dev];
+  return VEDA_OK;
+}
+
 veda_status get_encoder() {
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_encode) return VEDA_OK;
@@ -684,22 +706,38 @@ veda_status veda_block_sparse_attn_bwd(const void* q, const void* k, const void*
   a.items = static_cast<int64_t>(B) * H * nT;
   a.scale = softmax_scale;
   a.next_item = counters;
+  const unsigned grid = grid_for(a.items, sms, 1);
+  // The two kernels are independent and each holds a whole SM per CTA. dK/dV (uneven items:
+  // a key tile is listed by 0 to hundreds of query tiles) goes first on the caller's stream,
+  // dQ on the library's second stream of this device, so that dQ's CTAs start on the SMs that
+  // dK/dV's last items leave idle; the caller's stream then waits for both.
+  cudaStream_t aux;
+  cudaEvent_t ev_fork, ev_join;
+  if ((st = side_stream(aux, ev_fork, ev_join)) != VEDA_OK) return st;
+  // the fork / join events are shared by the device's calls: enqueue one call at a time
+  static std::mutex fork_mu;
+  std::lock_guard<std::mutex> fork_lk(fork_mu);
+  if ((ce = cudaEventRecord(ev_fork, s)) != cudaSuccess) return cuda_fail(ce, "cudaEventRecord");
+  if ((ce = cudaStreamWaitEvent(aux, ev_fork, 0)) != cudaSuccess) return cuda_fail(ce, "cudaStreamWaitEvent");
+  // dK, dV: key tiles over the transposed lists (fixed K, V; streamed Q, dO)
+  bwd::Args t = a;
+  t.full_cnt = t_cnt; t.full_idx = t_idx; t.part_cnt = nullptr; t.part_idx = nullptr;
+  t.stride = t_stride;
+  t.out0 = static_cast<__nv_bfloat16*>(dv);
+  t.out1 = static_cast<__nv_bfloat16*>(dk);
+  t.next_item = counters + 1;
+  bwd::bwd_kernel<bwd::kModeDKDV><<<grid, bwd::kThreads, bwd::kSmemBytesDKDV, s>>>(tk, tv, tq, tdo, t);
+  if ((st = launched("bwd_kernel<dK,dV>")) != VEDA_OK) return st;
   // dQ: query tiles over the forward lists (fixed Q, dO; streamed K, V)
   a.full_cnt = full_cnt; a.full_idx = full_idx; a.part_cnt = part_cnt; a.part_idx = part_idx;
   a.stride = list_stride;
   a.out0 = static_cast<__nv_bfloat16*>(dq);
   a.out1 = nullptr;
-  const unsigned grid = grid_for(a.items, sms, 1);
-  bwd::bwd_kernel<bwd::kModeDQ><<<grid, bwd::kThreads, bwd::kSmemBytesDQ, s>>>(tq, tdo, tk, tv, a);
+  bwd::bwd_kernel<bwd::kModeDQ><<<grid, bwd::kThreads, bwd::kSmemBytesDQ, aux>>>(tq, tdo, tk, tv, a);
   if ((st = launched("bwd_kernel<dQ>")) != VEDA_OK) return st;
-  // dK, dV: key tiles over the transposed lists (fixed K, V; streamed Q, dO)
-  a.full_cnt = t_cnt; a.full_idx = t_idx; a.part_cnt = nullptr; a.part_idx = nullptr;
-  a.stride = t_stride;
-  a.out0 = static_cast<__nv_bfloat16*>(dv);
-  a.out1 = static_cast<__nv_bfloat16*>(dk);
-  a.next_item = counters + 1;
-  bwd::bwd_kernel<bwd::kModeDKDV><<<grid, bwd::kThreads, bwd::kSmemBytesDKDV, s>>>(tk, tv, tq, tdo, a);
-  return launched("bwd_kernel<dK,dV>");
+  if ((ce = cudaEventRecord(ev_join, aux)) != cudaSuccess) return cuda_fail(ce, "cudaEventRecord");
+  if ((ce = cudaStreamWaitEvent(s, ev_join, 0)) != cudaSuccess) return cuda_fail(ce, "cudaStreamWaitEvent");
+  return VEDA_OK;
 }
 
 veda_status veda_rel_error(const void* o, const void* o_ref, float* sums, int32_t B, int32_t N, int32_t H,

@@ -339,6 +339,10 @@ VEDA_API veda_status veda_transpose_lists(const int32_t* full_cnt, const int32_t
  *                 kernels' work-queue counters (the library zeroes them)
  * All tensors 16-byte aligned. Out-of-range indices or counts are flagged
  * VEDA_ERR_DEVICE_CHECK.
+ * Streams: D and dK/dV run on `stream`; dQ, which is independent of dK/dV, runs on a second
+ * stream the library keeps for the device (created on the first call, kept until exit),
+ * forked from and joined back into `stream` with events, so that the call is ordered on
+ * `stream` like a single kernel. Calls from several host threads enqueue one at a time.
  */
 VEDA_API veda_status veda_block_sparse_attn_bwd(const void* q, const void* k, const void* v,
                                        const void* o, const void* dout, const float* lse,

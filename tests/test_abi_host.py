@@ -79,6 +79,12 @@ def test_device_calls_validate_before_cuda(L):
     den[0] = 2
     assert L.veda_select_blocks(16, 16, 16, 16, 1, ctypes.addressof(num), ctypes.addressof(den),
                                 16, 16, 16, 16, 1, 1, 1, 8, None) == INVALID          # stride too small
+    assert L.veda_select_blocks(16, 16, 16, 16, 1, ctypes.addressof(num), ctypes.addressof(den),
+                                16, 16, 16, 16, 2049, 1, 1, 2049, None) == INVALID    # nT above VEDA_MAX_TILES
+    num5 = (ctypes.c_int32 * 5)(1, 1, 1, 1, 1)
+    den5 = (ctypes.c_int32 * 5)(2, 2, 2, 2, 2)
+    assert L.veda_select_blocks(16, 16, 16, 16, 5, ctypes.addressof(num5), ctypes.addressof(den5),
+                                16, 16, 16, 16, 8, 1, 1, 8, None) == INVALID          # five segments
     assert L.veda_block_sparse_attn_fwd(16, 16, 16, 16, 16, 16, 16, 16, 4, -1.0, 16, None,
                                         1, 1, 4, 128, None) == INVALID                 # bad scale
     assert L.veda_block_sparse_attn_fwd(8, 16, 16, 16, 16, 16, 16, 16, 4, 0.1, 16, None,

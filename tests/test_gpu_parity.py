@@ -382,6 +382,36 @@ def test_density_one_twentieth_rows_of_only_the_diagonal():
             assert got == [r], (h, r, got)
 
 
+def test_maximum_tile_count():
+    """The largest tile count the selection accepts (2,048 tiles per head: 128 frames of 30 x 54,
+    207,360 tokens), stage by stage on two heads: selection on every row (its per-warp shared
+    memory is then above the default 48 KB a launch gets), attention on sampled query tiles."""
+    w = synth.Workload("max_tiles", 13, B=1, H=2, grid=(128, 30, 54), head_shapes=((1, 8, 16),) * 2)
+    assert w.nT == 2048
+    _stage_run(w, attn_rows=[(0, j, r) for j in range(2) for r in (0, 1, 1023, 2046, 2047)])
+
+
+def test_density_zero_keeps_only_the_diagonal():
+    """Density 0: every budget is 0 but the query's own segment, which the forced diagonal
+    raises to 1, so every row's list is its own tile and attention stays inside the tile."""
+    V = P.veda()
+    w = synth.Workload("rho0", 14, B=1, H=3, grid=(6, 17, 40), head_shapes=((1, 8, 16), (2, 8, 8), (4, 4, 8)),
+                       rho=((0, 1),))
+    _stage_run(w)
+    inp = synth.make_inputs(w)
+    maps = V.build_tile_map(w.grid, w.head_shapes).to(DEV)
+    bufs = V.sparse_attention(inp.q.to(DEV), inp.k.to(DEV), inp.v.to(DEV), inp.wq.to(DEV),
+                              inp.wk.to(DEV), maps, w.rho, P.SCALE)
+    V.check_device_status()
+    slots, nv, seg, nTh = P.oracle_maps(w, None)
+    fc, fi = bufs.lists.full_cnt.cpu().numpy(), bufs.lists.full_idx.cpu().numpy()
+    pc, pi = bufs.lists.part_cnt.cpu().numpy(), bufs.lists.part_idx.cpu().numpy()
+    for h in range(w.H):
+        for r in range(w.nT):
+            got = sorted(fi[0, h, r, :fc[0, h, r]].tolist() + pi[0, h, r, :pc[0, h, r]].tolist())
+            assert got == ([r] if r < nTh[h] else []), (h, r, got)
+
+
 def test_bounded_wait_runs_out_and_context_survives():
     # failure detection without a fault: a wait on a barrier nothing arrives on gives up
     # after 2 ms, the status word says VEDA_ERR_TIMEOUT, and the next call works
