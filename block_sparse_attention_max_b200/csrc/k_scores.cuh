@@ -128,10 +128,10 @@ __device__ __forceinline__ void role_producer(const Args& a, Bars& bars, uint32_
       tma_load_2d(st + kOffB, mB, smem_u32(&bars.full[s]), c * 32, tl.b_row);
     }
   }
-  if (*abort) {   // copies still in flight land before the CTA releases its shared memory
-    for (uint32_t i = g > kStages ? g - kStages : 0; i < g; ++i)
-      mbar_wait(smem_u32(&bars.full[i % kStages]), (i / kStages) & 1, nullptr, 61);
-  }
+  // every copy lands before the CTA releases its shared memory, also when another role gave
+  // up after this loop ended (in the normal run these phases have long completed)
+  for (uint32_t i = g > kStages ? g - kStages : 0; i < g; ++i)
+    mbar_wait(smem_u32(&bars.full[i % kStages]), (i / kStages) & 1, nullptr, 61);
 }
 
 // x with its 13 low mantissa bits cleared: a tf32 value, and x - tf32_hi(x) is exact.
