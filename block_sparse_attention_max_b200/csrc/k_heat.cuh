@@ -79,8 +79,8 @@ __device__ __forceinline__ bool heat_group(attn::Bars& bars, uint32_t tmem, uint
       const uint64_t yy = f2_fma(f2_pack(s[b][4 * k + 2], s[b][4 * k + 3]), c2, nlx1);
       const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
       float q0, q1;
-      if (k & 1) {
-        exp2_fma_x2(yy, q0, q1);   // a quarter of the exponentials on the FMA pipe
+      if ((k & 3) == 3) {
+        exp2_fma_x2(yy, q0, q1);   // an eighth of the exponentials on the FMA pipe
       } else {
         f2_unpack(yy, y0, y1);
         q0 = ex2_approx(y0);

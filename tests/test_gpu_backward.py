@@ -171,3 +171,57 @@ def test_backward_clip16x9_one_head():
     """The 16:9 clip at full size (40 heads launched, the benchmark's configuration), every
     transposed list checked, the gradients of head 0 against the oracle over all its rows."""
     _run(synth.CLIP16x9, [0])
+
+
+def test_backward_from_two_host_threads_matches_serial():
+    """The backward runs dQ on a second stream of the library, forked from and joined back
+    into the caller's stream with events the device's calls share. Two host threads, each on
+    a stream of its own with its own output gradient, enqueue backward calls at the same
+    time; every result equals the serial call's bit for bit (every output tile is reduced
+    inside one CTA, so the kernels are deterministic whichever CTA takes an item)."""
+    import threading
+    V = P.veda()
+    w = synth.SMALL
+    inp = synth.make_inputs(w)
+    maps = V.build_tile_map(w.grid, w.head_shapes, w.n_tail, inp.tile_order).to(DEV)
+    bufs = V.sparse_attention(inp.q.to(DEV), inp.k.to(DEV), inp.v.to(DEV), inp.wq.to(DEV), inp.wk.to(DEV),
+                              maps, w.rho, P.SCALE)
+    tl = V.transpose_lists(bufs.lists, maps)
+    grads = []
+    for seed in (1, 2):
+        g = torch.Generator().manual_seed(5000 + seed)
+        grads.append(V.permute_tiles(torch.randn(inp.q.shape, generator=g).to(torch.bfloat16).to(DEV), maps))
+
+    def bwd(do_t):
+        return V.block_sparse_attn_bwd(bufs.q_t, bufs.k_t, bufs.v_t, bufs.o_t, do_t, bufs.lse, maps,
+                                       bufs.lists, tl, P.SCALE)
+
+    ref = [bwd(grads[i]) for i in range(2)]
+    torch.cuda.synchronize()
+    V.check_device_status()
+    reps = 4
+    out = [[None] * reps for _ in range(2)]
+    errors = []
+
+    def worker(i):
+        try:
+            s = torch.cuda.Stream(device=DEV)
+            with torch.cuda.device(DEV), torch.cuda.stream(s):
+                for r in range(reps):
+                    out[i][r] = bwd(grads[i])
+            s.synchronize()
+        except Exception as e:  # pragma: no cover - reported below
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    torch.cuda.synchronize()
+    V.check_device_status()
+    for i in range(2):
+        for r in range(reps):
+            for got, want in zip(out[i][r], ref[i]):
+                assert torch.equal(got, want), (i, r)
