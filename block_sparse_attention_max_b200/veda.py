@@ -577,15 +577,16 @@ def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, wq: torc
                      scale: float, buffers: Optional[PathBuffers] = None, stream=None):
     """All six steps on raster Q/K/V [B, N, H, 128] (bf16, on the device).
 
-    Returns the PathBuffers holding every intermediate; ``.o`` is the raster output.
+    Returns the PathBuffers holding every intermediate; ``.o`` is the raster output. Steps 1
+    and 2 of Q and K run as one call each (``permute_pool``: the tiles of ``permute_tiles``,
+    the pooled features of ``tile_pool`` up to fp32 summation order in the mean), so that the
+    tiled Q and K are not read a second time.
     """
     B, N, H, D = q.shape
     bufs = buffers or PathBuffers.allocate(B, N, H, maps, rho, q.device)
-    permute_tiles(q, maps, bufs.q_t, stream)
-    permute_tiles(k, maps, bufs.k_t, stream)
+    permute_pool(q, maps, bufs.q_t, bufs.pooled_q, stream)
+    permute_pool(k, maps, bufs.k_t, bufs.pooled_k, stream)
     permute_tiles(v, maps, bufs.v_t, stream)
-    tile_pool(bufs.q_t, maps, bufs.pooled_q, stream)
-    tile_pool(bufs.k_t, maps, bufs.pooled_k, stream)
     block_scores(bufs.pooled_q, bufs.pooled_k, wq, wk, bufs.scores, bufs.workspace, stream)
     select_blocks(bufs.scores, maps, rho, bufs.lists.stride, bufs.lists, stream)
     block_sparse_attn_fwd(bufs.q_t, bufs.k_t, bufs.v_t, maps, bufs.lists, scale, bufs.o_t,
