@@ -194,6 +194,23 @@ def _valid_token_flop(lists, tile_valid: np.ndarray) -> float:
     return 4.0 * 128 * total
 
 
+def _executed_flop(lists, tile_valid: np.ndarray) -> float:
+    """Tensor-core FLOP the forward kernel executes: 4 * 128 * 128 * w per visited block, w = 64
+    keys for a partial-list key tile with at most 64 valid slots (its upper half is not
+    computed), else 128."""
+    pc = lists.part_cnt.cpu().numpy()
+    pi = lists.part_idx.cpu().numpy()
+    B, H, nT = pc.shape
+    half = 0
+    for h in range(H):
+        small = tile_valid[h] <= 64
+        col = np.arange(pi.shape[-1])
+        for b in range(B):
+            sel = col[None, :] < pc[b, h][:, None]
+            half += int((sel & small[np.clip(pi[b, h], 0, nT - 1)]).sum())
+    return (_visited_blocks(lists) - half / 2.0) * FLOP_PER_BLOCK
+
+
 def _random_device_lists(rng, lists, tile_valid: np.ndarray, dev):
     """Fresh uniform random block lists with a forced diagonal and the same per-row budget as
     `lists` (the 'new pattern per call' timing), split into full / partial tiles."""
@@ -321,6 +338,7 @@ def run_veda(args):
     # and the same kernel on fresh uniform random lists (same budgets), one pattern per call
     tile_valid = np.asarray(hmaps.tile_valid)
     valid_flop = _valid_token_flop(bufs.lists, tile_valid)
+    exec_flop = _executed_flop(bufs.lists, tile_valid)
     rng = np.random.default_rng(7007)
     patterns = [_random_device_lists(rng, bufs.lists, tile_valid, dev) for _ in range(4)]
     rnd_blocks = statistics.mean(_visited_blocks(p) for p in patterns)
@@ -358,6 +376,10 @@ def run_veda(args):
     perm_ms, pool_ms = statistics.median(perm_times), statistics.median(pool_times)
     attn_secondary = {
         "valid_token_tflops": valid_flop / (attn_ms * 1e-3) / 1e12,
+        "executed_tflops": exec_flop / (attn_ms * 1e-3) / 1e12,
+        "executed_frac_bf16_peak": exec_flop / (attn_ms * 1e-3) / 1e12 / peaks["bf16"],
+        "executed_note": "tensor-core FLOP actually issued: key tiles with at most 64 valid slots are "
+                         "computed over their first 64 keys",
         "dense_equivalent_tflops": 4.0 * D * N * N * H * B / (attn_ms * 1e-3) / 1e12,
         "random_lists_ms": rnd_ms,
         "random_lists_tflops": rnd_blocks * FLOP_PER_BLOCK / (rnd_ms * 1e-3) / 1e12,

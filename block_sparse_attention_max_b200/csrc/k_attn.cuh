@@ -22,7 +22,10 @@
 //                softmax warp has taken S(j-2) out of buffer b
 //   warp 10      P V issuer (one thread): O += P_b V_j, P_b read from tensor memory
 // An eighth of the exponentials (the second row of every fourth column group) run on the FMA
-// pipe (exp2_fma_x2) instead of the MUFU, whose rate sets the pace of the softmax.
+// pipe (exp2_fma_x2) instead of the MUFU. A key tile with at most 64 valid slots (a partial
+// tile whose valid prefix fits in half the tile) is computed over its first 64 keys only:
+// Q K^T with N = 64, P V with K = 64 and half the softmax, flagged by the producers in the
+// ring slot's op word.
 // Tensor memory (512 columns): S0 | S1 | O | P0 | P1. With two S buffers, each freed as
 // soon as the softmax holds it in registers, and P in buffers of its own, the tensor core
 // computes S(j+1) and P V(j-1) while the softmax works on block j. The running maximum (in
@@ -56,6 +59,7 @@ constexpr uint32_t kSmemBytes = kSmemTiles + 1024;             // + alignment sl
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;         // S_b at 128b, P_b at 384 + 64b
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);   // A, B K-major
+constexpr uint32_t kIdescQK64 = idesc_bf16_f32(128, 64, 0, 0);  // the first 64 keys
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 0, 1);   // B (V) MN-major
 constexpr float kRescaleLog2 = 30.0f;
 // register split (setmaxnreg): two softmax warpgroups and one producer/MMA warpgroup;
@@ -84,7 +88,8 @@ enum : uint32_t {
   kOpLastBlk = 1u << 1,   // last block of the item
   kOpFirstItem = 1u << 2, // the CTA's first item (no earlier O to wait for)
   kOpStop = 1u << 3,      // end of the stream (no tile)
-  kOpQBufShift = 4,       // Q buffer of the item (bits 4..)
+  kOpHalf = 1u << 4,      // key tile with at most 64 valid slots: Q K^T and P V over keys 0..63
+  kOpQBufShift = 8,       // Q buffer of the item (bits 8..)
 };
 
 struct Bars {
@@ -158,6 +163,14 @@ __device__ __forceinline__ void reg_dealloc() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// Valid key slots of block j of an item (entries j >= nf come from the partial list), clamped
+// to [1, 128]; the Q / K producer flags out-of-range counts.
+__device__ __forceinline__ int32_t block_nv(const int32_t* valid_h, int32_t j, int32_t nf, int32_t idx) {
+  if (j < nf) return 128;
+  const int32_t nv = valid_h[idx];
+  return nv < 1 ? 1 : (nv > 128 ? 128 : nv);
+}
+
 // CTA-local item m of the persistent loop.
 __device__ __forceinline__ int64_t cta_item(int64_t m) {
   return blockIdx.x + m * static_cast<int64_t>(gridDim.x);
@@ -218,6 +231,17 @@ __device__ __forceinline__ void tmem_st_16x128b_x16(uint32_t taddr, const uint32
       "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+// P columns 16 OFF / 2 .. + 31 from r[OFF .. OFF + 15] (keys 0..63 for OFF = 0, 64..127 for 16).
+template <int OFF>
+__device__ __forceinline__ void tmem_st_p_half(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16};" ::"r"(taddr),
+      "r"(r[OFF + 0]), "r"(r[OFF + 1]), "r"(r[OFF + 2]), "r"(r[OFF + 3]), "r"(r[OFF + 4]), "r"(r[OFF + 5]),
+      "r"(r[OFF + 6]), "r"(r[OFF + 7]), "r"(r[OFF + 8]), "r"(r[OFF + 9]), "r"(r[OFF + 10]), "r"(r[OFF + 11]),
+      "r"(r[OFF + 12]), "r"(r[OFF + 13]), "r"(r[OFF + 14]), "r"(r[OFF + 15])
+      : "memory");
+}
 template <int N>
 __device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
 #pragma unroll
@@ -230,6 +254,154 @@ __device__ __forceinline__ float quad_max(float v) {
 __device__ __forceinline__ float quad_sum(float v) {
   v += __shfl_xor_sync(0xffffffffu, v, 1);
   return v + __shfl_xor_sync(0xffffffffu, v, 2);
+}
+
+// One block of one warp's softmax, S in buffer g & 1: takes S into registers and hands the
+// buffer back, masks key slots >= nv, computes P with the running maximum (moving it and
+// rescaling O when a row's maximum grew by more than 30, in log2 units), adds the row sums
+// and hands P over in buffer g & 1. A key tile with at most 64 valid slots had Q K^T and P V
+// issued over its first 64 keys only: the softmax then covers column groups 0..7 and skips
+// 8..15 by a warp-uniform branch inside the one unrolled loop (a second, narrower copy of the
+// loop measured slower: the two copies compete for the instruction cache). Returns false
+// when a bounded wait ran out.
+__device__ __forceinline__ bool softmax_block(const Args& a, Bars& bars, uint32_t tmem, uint32_t lane_off,
+                                              uint32_t c, uint32_t lane, uint32_t g, bool first, int32_t nv,
+                                              volatile int* abort, float& m0, float& m1, float& l0, float& l1) {
+  const uint32_t sbuf = g & 1;
+  tc_fence_after();
+  const bool hi = nv > 64;   // the upper 64 keys were computed
+  uint32_t s[64];
+  tmem_ld_16x256b_x16(tmem + lane_off + kColS + sbuf * 128, s);
+  tmem_wait_ld();
+  reg_fence(s);
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(smem_u32(&bars.s_free[sbuf]));
+  if (nv < 128) {
+    // column 8k + 2c + e is a key slot < nv exactly for k < kv_e = ceil((nv - 2c - e) / 8)
+    const int32_t kv0 = (nv - 2 * static_cast<int32_t>(c) + 7) >> 3;
+    const int32_t kv1 = (nv - 2 * static_cast<int32_t>(c) + 6) >> 3;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      if (k >= kv0) { s[4 * k] = 0xFF800000u; s[4 * k + 2] = 0xFF800000u; }   // -inf
+      if (k >= kv1) { s[4 * k + 1] = 0xFF800000u; s[4 * k + 3] = 0xFF800000u; }
+    }
+  }
+  // Exponentials with the current running maximum m, computed together with the block's
+  // row maxima (one basic block, so the scheduler interleaves the MUFU and max chains).
+  // If a row's maximum (log2 units) grew by more than 30, the reference moves, O is
+  // rescaled and the pass is repeated; otherwise P uses the stale maximum, exact after the
+  // division by the row sum (P stays below 2^30, far inside bf16 and the fp32 sums of at
+  // most nT * 128 terms). Block 0 of an item takes its row maxima first, so that its
+  // single pass has a reference.
+  if (first) {
+    float a4[4], b4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      a4[q] = fmaxf(__uint_as_float(s[4 * q]), __uint_as_float(s[4 * q + 1]));
+      b4[q] = fmaxf(__uint_as_float(s[4 * q + 2]), __uint_as_float(s[4 * q + 3]));
+    }
+#pragma unroll
+    for (int k = 4; k < 16; ++k) {
+      if (k == 8 && !hi) break;
+      a4[k & 3] = fmax3(a4[k & 3], __uint_as_float(s[4 * k]), __uint_as_float(s[4 * k + 1]));
+      b4[k & 3] = fmax3(b4[k & 3], __uint_as_float(s[4 * k + 2]), __uint_as_float(s[4 * k + 3]));
+    }
+    m0 = quad_max(fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3]))) * a.scale_log2;
+    m1 = quad_max(fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3]))) * a.scale_log2;
+  }
+  const uint64_t c2 = f2_pack(__float_as_uint(a.scale_log2), __float_as_uint(a.scale_log2));
+  uint64_t acc0[2], acc1[2];
+  uint32_t pk[32];
+#pragma unroll 1
+  for (int pass = 0;; ++pass) {
+    const uint64_t nm0 = f2_pack(__float_as_uint(-m0), __float_as_uint(-m0));
+    const uint64_t nm1 = f2_pack(__float_as_uint(-m1), __float_as_uint(-m1));
+    acc0[0] = acc0[1] = acc1[0] = acc1[1] = 0ull;
+    float a4[4], b4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      a4[q] = fmaxf(__uint_as_float(s[4 * q]), __uint_as_float(s[4 * q + 1]));
+      b4[q] = fmaxf(__uint_as_float(s[4 * q + 2]), __uint_as_float(s[4 * q + 3]));
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      if (k == 8 && !hi) break;
+      if (k >= 4) {
+        a4[k & 3] = fmax3(a4[k & 3], __uint_as_float(s[4 * k]), __uint_as_float(s[4 * k + 1]));
+        b4[k & 3] = fmax3(b4[k & 3], __uint_as_float(s[4 * k + 2]), __uint_as_float(s[4 * k + 3]));
+      }
+      float x0, x1, q0, q1;
+      f2_unpack(f2_fma(f2_pack(s[4 * k], s[4 * k + 1]), c2, nm0), x0, x1);
+      const uint64_t yy = f2_fma(f2_pack(s[4 * k + 2], s[4 * k + 3]), c2, nm1);
+      const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+      if ((k & 3) == 3) {   // an eighth of the exponentials on the FMA pipe
+        exp2_fma_x2(yy, q0, q1);
+      } else {
+        float y0, y1;
+        f2_unpack(yy, y0, y1);
+        q0 = ex2_approx(y0);
+        q1 = ex2_approx(y1);
+      }
+      acc0[k & 1] = f2_add(acc0[k & 1], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
+      acc1[k & 1] = f2_add(acc1[k & 1], f2_pack(__float_as_uint(q0), __float_as_uint(q1)));
+      pk[2 * k] = pack_bf16x2(p0, p1);
+      pk[2 * k + 1] = pack_bf16x2(q0, q1);
+    }
+    const float mb0 = quad_max(fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3]))) * a.scale_log2;
+    const float mb1 = quad_max(fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3]))) * a.scale_log2;
+    const bool need0 = mb0 > m0 + kRescaleLog2;
+    const bool need1 = mb1 > m1 + kRescaleLog2;
+    if (pass == 1 || !__any_sync(0xffffffffu, need0 || need1)) break;
+    // O must hold P V of every earlier block before it is rescaled
+    const uint32_t gp = g - 1;
+    if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 31)) return false;
+    tc_fence_after();
+    const float al0 = need0 ? ex2_approx(m0 - mb0) : 1.0f;
+    const float al1 = need1 ? ex2_approx(m1 - mb1) : 1.0f;
+    const uint64_t al0x2 = f2_pack(__float_as_uint(al0), __float_as_uint(al0));
+    const uint64_t al1x2 = f2_pack(__float_as_uint(al1), __float_as_uint(al1));
+#pragma unroll 1
+    for (int ch = 0; ch < 4; ++ch) {
+      uint32_t o16[16];
+      const uint32_t oa = tmem + lane_off + kColO + ch * 32;
+      tmem_ld_16x256b_x4(oa, o16);
+      tmem_wait_ld();
+      reg_fence(o16);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float x, y;
+        f2_unpack(f2_mul(f2_pack(o16[4 * q], o16[4 * q + 1]), al0x2), x, y);
+        o16[4 * q] = __float_as_uint(x); o16[4 * q + 1] = __float_as_uint(y);
+        f2_unpack(f2_mul(f2_pack(o16[4 * q + 2], o16[4 * q + 3]), al1x2), x, y);
+        o16[4 * q + 2] = __float_as_uint(x); o16[4 * q + 3] = __float_as_uint(y);
+      }
+      tmem_st_16x256b_x4(oa, o16);
+    }
+    tmem_wait_st();
+    if (need0) { l0 *= al0; m0 = mb0; }
+    if (need1) { l1 *= al1; m1 = mb1; }
+  }
+  {
+    float t0, t1, t2, t3;
+    f2_unpack(acc0[0], t0, t1); f2_unpack(acc0[1], t2, t3);
+    l0 += (t0 + t1) + (t2 + t3);
+    f2_unpack(acc1[0], t0, t1); f2_unpack(acc1[1], t2, t3);
+    l1 += (t0 + t1) + (t2 + t3);
+  }
+  // P buffer g & 1 is free once P V of block g - 2 has completed
+  if (g >= 2) {
+    const uint32_t gp = g - 2;
+    if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 32)) return false;
+    tc_fence_after();
+  }
+  tmem_st_p_half<0>(tmem + lane_off + kColP + sbuf * 64, pk);
+  if (hi) tmem_st_p_half<16>(tmem + lane_off + kColP + sbuf * 64 + 32, pk);
+  tmem_wait_st();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(smem_u32(&bars.p_full[sbuf]));
+  return true;
 }
 
 // Softmax and epilogue of one warp's 16 rows for every item of the CTA. Thread (lane)
@@ -268,136 +440,10 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
       if (!warp_wait_abort(smem_u32(&bars.rec_full[g % kRec]), (g / kRec) & 1, abort, 36)) { ok = false; break; }
       const int32_t nv = reinterpret_cast<volatile int32_t*>(bars.rec_nv)[g % kRec];
       if (!warp_wait_abort(smem_u32(&bars.s_full[sbuf]), (g >> 1) & 1, abort, 30)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t s[64];
-      tmem_ld_16x256b_x16(tmem + lane_off + kColS + sbuf * 128, s);
-      tmem_wait_ld();
-      reg_fence(s);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars.s_free[sbuf]));
-      if (nv < 128) {
-        // column 8k + 2c + e is a key slot < nv exactly for k < kv_e = ceil((nv - 2c - e) / 8)
-        const int32_t kv0 = (nv - 2 * static_cast<int32_t>(c) + 7) >> 3;
-        const int32_t kv1 = (nv - 2 * static_cast<int32_t>(c) + 6) >> 3;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          if (k >= kv0) { s[4 * k] = 0xFF800000u; s[4 * k + 2] = 0xFF800000u; }   // -inf
-          if (k >= kv1) { s[4 * k + 1] = 0xFF800000u; s[4 * k + 3] = 0xFF800000u; }
-        }
+      if (!softmax_block(a, bars, tmem, lane_off, c, lane, g, j == 0, nv, abort, m0, m1, l0, l1)) {
+        ok = false;
+        break;
       }
-      // Exponentials with the current running maximum m, computed together with the block's
-      // row maxima (one basic block, so the scheduler interleaves the MUFU and max chains).
-      // If a row's maximum (log2 units) grew by more than 30, the reference moves, O is
-      // rescaled and the pass is repeated; otherwise P uses the stale maximum, exact after the
-      // division by the row sum (P stays below 2^30, far inside bf16 and the fp32 sums of at
-      // most nT * 128 terms). Block 0 of an item takes its row maxima first, so that its
-      // single pass has a reference.
-      if (j == 0) {
-        float a4[4], b4[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          a4[q] = fmaxf(__uint_as_float(s[4 * q]), __uint_as_float(s[4 * q + 1]));
-          b4[q] = fmaxf(__uint_as_float(s[4 * q + 2]), __uint_as_float(s[4 * q + 3]));
-        }
-#pragma unroll
-        for (int k = 4; k < 16; ++k) {
-          a4[k & 3] = fmax3(a4[k & 3], __uint_as_float(s[4 * k]), __uint_as_float(s[4 * k + 1]));
-          b4[k & 3] = fmax3(b4[k & 3], __uint_as_float(s[4 * k + 2]), __uint_as_float(s[4 * k + 3]));
-        }
-        m0 = quad_max(fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3]))) * a.scale_log2;
-        m1 = quad_max(fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3]))) * a.scale_log2;
-      }
-      const uint64_t c2 = f2_pack(__float_as_uint(a.scale_log2), __float_as_uint(a.scale_log2));
-      uint64_t acc0[2], acc1[2];
-      uint32_t pk[32];
-#pragma unroll 1
-      for (int pass = 0;; ++pass) {
-        const uint64_t nm0 = f2_pack(__float_as_uint(-m0), __float_as_uint(-m0));
-        const uint64_t nm1 = f2_pack(__float_as_uint(-m1), __float_as_uint(-m1));
-        acc0[0] = acc0[1] = acc1[0] = acc1[1] = 0ull;
-        float a4[4], b4[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          a4[q] = fmaxf(__uint_as_float(s[4 * q]), __uint_as_float(s[4 * q + 1]));
-          b4[q] = fmaxf(__uint_as_float(s[4 * q + 2]), __uint_as_float(s[4 * q + 3]));
-        }
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          if (k >= 4) {
-            a4[k & 3] = fmax3(a4[k & 3], __uint_as_float(s[4 * k]), __uint_as_float(s[4 * k + 1]));
-            b4[k & 3] = fmax3(b4[k & 3], __uint_as_float(s[4 * k + 2]), __uint_as_float(s[4 * k + 3]));
-          }
-          float x0, x1, q0, q1;
-          f2_unpack(f2_fma(f2_pack(s[4 * k], s[4 * k + 1]), c2, nm0), x0, x1);
-          const uint64_t yy = f2_fma(f2_pack(s[4 * k + 2], s[4 * k + 3]), c2, nm1);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-          if ((k & 3) == 3) {   // an eighth of the exponentials on the FMA pipe
-            exp2_fma_x2(yy, q0, q1);
-          } else {
-            float y0, y1;
-            f2_unpack(yy, y0, y1);
-            q0 = ex2_approx(y0);
-            q1 = ex2_approx(y1);
-          }
-          acc0[k & 1] = f2_add(acc0[k & 1], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
-          acc1[k & 1] = f2_add(acc1[k & 1], f2_pack(__float_as_uint(q0), __float_as_uint(q1)));
-          pk[2 * k] = pack_bf16x2(p0, p1);
-          pk[2 * k + 1] = pack_bf16x2(q0, q1);
-        }
-        const float mb0 = quad_max(fmaxf(fmaxf(a4[0], a4[1]), fmaxf(a4[2], a4[3]))) * a.scale_log2;
-        const float mb1 = quad_max(fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3]))) * a.scale_log2;
-        const bool need0 = mb0 > m0 + kRescaleLog2;
-        const bool need1 = mb1 > m1 + kRescaleLog2;
-        if (pass == 1 || !__any_sync(0xffffffffu, need0 || need1)) break;
-        // O must hold P V of every earlier block before it is rescaled
-        const uint32_t gp = g - 1;
-        if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 31)) { ok = false; break; }
-        tc_fence_after();
-        const float al0 = need0 ? ex2_approx(m0 - mb0) : 1.0f;
-        const float al1 = need1 ? ex2_approx(m1 - mb1) : 1.0f;
-        const uint64_t al0x2 = f2_pack(__float_as_uint(al0), __float_as_uint(al0));
-        const uint64_t al1x2 = f2_pack(__float_as_uint(al1), __float_as_uint(al1));
-#pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t o16[16];
-          const uint32_t oa = tmem + lane_off + kColO + ch * 32;
-          tmem_ld_16x256b_x4(oa, o16);
-          tmem_wait_ld();
-          reg_fence(o16);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float x, y;
-            f2_unpack(f2_mul(f2_pack(o16[4 * q], o16[4 * q + 1]), al0x2), x, y);
-            o16[4 * q] = __float_as_uint(x); o16[4 * q + 1] = __float_as_uint(y);
-            f2_unpack(f2_mul(f2_pack(o16[4 * q + 2], o16[4 * q + 3]), al1x2), x, y);
-            o16[4 * q + 2] = __float_as_uint(x); o16[4 * q + 3] = __float_as_uint(y);
-          }
-          tmem_st_16x256b_x4(oa, o16);
-        }
-        tmem_wait_st();
-        if (need0) { l0 *= al0; m0 = mb0; }
-        if (need1) { l1 *= al1; m1 = mb1; }
-      }
-      if (!ok) break;
-      {
-        float t0, t1, t2, t3;
-        f2_unpack(acc0[0], t0, t1); f2_unpack(acc0[1], t2, t3);
-        l0 += (t0 + t1) + (t2 + t3);
-        f2_unpack(acc1[0], t0, t1); f2_unpack(acc1[1], t2, t3);
-        l1 += (t0 + t1) + (t2 + t3);
-      }
-      // P buffer g & 1 is free once P V of block g - 2 has completed
-      if (g >= 2) {
-        const uint32_t gp = g - 2;
-        if (!warp_wait_abort(smem_u32(&bars.o_done[gp & 1]), (gp >> 1) & 1, abort, 32)) { ok = false; break; }
-        tc_fence_after();
-      }
-      tmem_st_16x128b_x16(tmem + lane_off + kColP + sbuf * 64, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars.p_full[sbuf]));
     }
     if (!ok) break;
     // epilogue: row sums over the quad, O / l -> bf16, LSE
@@ -438,6 +484,9 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
 
 // TMA producer of Q (per item) and K_j (kKSt-deep ring), plus one record per block (valid
 // key slots and key tile index) for the softmax warps.
+// kHalfKeys: mark key tiles with at most 64 valid slots (kOpHalf), so that the issuer runs
+// Q K^T over their first 64 keys only (the attention; block heat takes whole tiles).
+template <bool kHalfKeys>
 __device__ __forceinline__ void role_qk_producer(const Args& a, Bars& bars, uint32_t sb, const CUtensorMap* tmQ,
                                                  const CUtensorMap* tmK, volatile int* abort) {
   uint32_t kc = 0, qc = 0;
@@ -464,21 +513,16 @@ __device__ __forceinline__ void role_qk_producer(const Args& a, Bars& bars, uint
       const int32_t row = static_cast<int32_t>((head_row + idx) * 128);
       const uint32_t ks = kc % kKSt;
       if (kc >= kKSt && !mbar_wait(smem_u32(&bars.k_empty[ks]), (kc / kKSt - 1) & 1, abort, 11)) { stop = true; break; }
-      bars.k_op[ks] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (qb << kOpQBufShift);
+      if (j >= nf && (valid_h[idx] < 1 || valid_h[idx] > 128)) flag_status(ST_BAD_LIST);
+      const int32_t nv = block_nv(valid_h, j, nf, idx);
+      bars.k_op[ks] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) |
+                      (kHalfKeys && nv <= 64 ? kOpHalf : 0u) | (qb << kOpQBufShift);
       const uint32_t kb = smem_u32(&bars.k_full[ks]);
       mbar_arrive_expect_tx(kb, kTileB);
       tma_load_2d(sb + kOffK + ks * kTileB, tmK, kb, 0, row);
       tma_load_2d(sb + kOffK + ks * kTileB + kHalfB, tmK, kb, 64, row);
       // block record (entry kc % kRec was last read for block kc - kRec, before the
       // softmax freed S(kc - kRec) and so before K(kc - kRec + kKSt + 2) could load)
-      int32_t nv = 128;
-      if (j >= nf) {
-        nv = valid_h[idx];
-        if (nv < 1 || nv > 128) {
-          flag_status(ST_BAD_LIST);
-          nv = nv < 1 ? 1 : 128;
-        }
-      }
       bars.rec_nv[kc % kRec] = nv;
       bars.rec_idx[kc % kRec] = idx;
       mbar_arrive(smem_u32(&bars.rec_full[kc % kRec]));
@@ -516,13 +560,15 @@ __device__ __forceinline__ void role_v_producer(const Args& a, Bars& bars, uint3
     const int32_t n = item_blocks(a, u, nf, bad);
     if (n == 0) continue;
     const int64_t head_row = (u / a.nT) * a.nT;
+    const int32_t* valid_h = a.valid + ((u / a.nT) % a.H) * a.nT;
     for (int32_t j = 0; j < n; ++j) {
       bool b2;
       const int32_t idx = item_key(a, u, nf, j, b2);
       const int32_t row = static_cast<int32_t>((head_row + idx) * 128);
       const uint32_t vs = vc % kVSt;
       if (vc >= kVSt && !mbar_wait(smem_u32(&bars.v_empty[vs]), (vc / kVSt - 1) & 1, abort, 12)) { stop = true; break; }
-      bars.v_op[vs] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (items == 0 ? kOpFirstItem : 0u);
+      bars.v_op[vs] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (items == 0 ? kOpFirstItem : 0u) |
+                      (block_nv(valid_h, j, nf, idx) <= 64 ? kOpHalf : 0u);
       const uint32_t vb = smem_u32(&bars.v_full[vs]);
       mbar_arrive_expect_tx(vb, kTileB);
       tma_load_2d(sb + kOffV + vs * kTileB, tmV, vb, 0, row);
@@ -570,10 +616,11 @@ __device__ __forceinline__ void role_qk_issuer(Bars& bars, uint32_t sb, uint32_t
     const uint64_t a0 = opaque(dQ + static_cast<uint64_t>(qb * (kTileB >> 4)));
     const uint64_t b0 = opaque(dK + static_cast<uint64_t>(ks * (kTileB >> 4)));
     const uint32_t d = tmem + kColS + sbuf * 128;
+    const uint32_t idesc = (op & kOpHalf) ? kIdescQK64 : kIdescQK;   // N = 64: keys 0..63
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       const uint64_t koff = static_cast<uint64_t>((kk >> 2) * (kHalfB >> 4) + (kk & 3) * 2);
-      mma_ss(d, a0 + koff, b0 + koff, kIdescQK, kk > 0 ? 1u : 0u);
+      mma_ss(d, a0 + koff, b0 + koff, idesc, kk > 0 ? 1u : 0u);
     }
     tc_commit(smem_u32(&bars.s_full[sbuf]));
     if (op & kOpLastBlk) tc_commit(smem_u32(&bars.q_empty[qb]));
@@ -603,8 +650,13 @@ __device__ __forceinline__ void role_pv_issuer(Bars& bars, uint32_t sb, uint32_t
     const uint32_t pa = tmem + kColP + pb * 64;
     mma_ts(tmem + kColO, pa, b0, kIdescPV, (op & kOpNewItem) ? 0u : 1u);
 #pragma unroll
-    for (int kk = 1; kk < 8; ++kk)
+    for (int kk = 1; kk < 4; ++kk)
       mma_ts(tmem + kColO, pa + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescPV, 1u);
+    if (!(op & kOpHalf)) {   // keys 64..127 (P columns 32..63, V rows 64..127)
+#pragma unroll
+      for (int kk = 4; kk < 8; ++kk)
+        mma_ts(tmem + kColO, pa + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescPV, 1u);
+    }
     tc_commit(smem_u32(&bars.o_done[pb]));
     tc_commit(smem_u32(&bars.v_empty[vs]));
     if (op & kOpLastBlk) ++items_done;
@@ -668,7 +720,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   if (wg == 2) {
     reg_dealloc<kControlRegs>();
     if (warp == 8 && lane == 0)
-      role_qk_producer(a, bars, sb, &tmQ, &tmK, abort);
+      role_qk_producer<true>(a, bars, sb, &tmQ, &tmK, abort);
     else if (warp == 11 && lane == 0)
       role_v_producer(a, bars, sb, &tmV, abort);
     else if (warp == 9 && lane == 0)

@@ -182,7 +182,7 @@ heat_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
   if (wg == 2) {
     reg_dealloc<kControlRegs>();
     if (warp == 8 && lane == 0)
-      role_qk_producer(p.a, bars, sb, &tmQ, &tmK, abort);
+      role_qk_producer<false>(p.a, bars, sb, &tmQ, &tmK, abort);
     else if (warp == 9 && lane == 0)
       role_qk_issuer(bars, sb, tmem, abort);
   } else {

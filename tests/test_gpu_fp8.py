@@ -150,6 +150,15 @@ def test_fp8_ragged_heads_batch_and_empty_rows():
     _run(w, [0, 1, 2])
 
 
+@pytest.mark.parametrize("r", [1, 63, 64, 65])
+def test_fp8_partial_key_tiles_of_every_width(r):
+    """Partial key and query tiles of r valid slots (r = 1, 63, 64, 65) between whole ones:
+    tiles of 128, r, 128, r valid slots, density 1, so every item mixes both kinds."""
+    w = synth.Workload(f"halfw{r}", 13, B=1, H=2, grid=(2, 1, 128 + r),
+                       head_shapes=((1, 1, 128), (1, 1, 128)), rho=((1, 1),), field=False)
+    _run(w, [0, 1])
+
+
 def test_fp8_clip16x9_sampled():
     """The 16:9 clip at full size (40 heads launched, the benchmark's configuration): codes and
     scales of two heads bit-exact, attention of three query tiles of each against the oracle."""

@@ -146,6 +146,18 @@ def test_stages_ragged_heads_and_empty_rows():
     _stage_run(w)
 
 
+@pytest.mark.parametrize("r", [1, 8, 63, 64, 65, 127])
+def test_partial_key_tiles_at_the_half_width_boundary(r):
+    """Key tiles with at most 64 valid slots take the half-width path (Q K^T and P V over
+    their first 64 keys, the softmax over 8 column groups), tiles with more the whole tile.
+    Grid 2 x 1 x (128 + r) in (1, 1, 128) tiles gives key tiles of 128, r, 128, r valid slots;
+    at density 1 every query tile (whole or partial) visits all four, so both paths alternate
+    inside every item."""
+    w = synth.Workload(f"halfw{r}", 13, B=1, H=2, grid=(2, 1, 128 + r),
+                       head_shapes=((1, 1, 128), (1, 1, 128)), rho=((1, 1),), field=False)
+    _stage_run(w)
+
+
 def test_stages_length_sweep_shortest():
     _stage_run(synth.sweep_length(5), heads=[0, 17, 39],
                attn_rows=[(0, j, r) for j in range(3) for r in (0, 1, 40, 79)])
