@@ -9,7 +9,8 @@
 //   delta_kernel           D = rowsum(dO * O) per query row (HBM stream)
 //   transpose_lists_kernel query tiles of every key tile (one warp per key tile)
 //   bwd_kernel<kModeDQ>    one query tile per CTA item, over its forward list: S = Q K_j^T,
-//                          dP = dO V_j^T, dS in TMEM, dQ += dS K_j
+//                          dP = dO V_j^T, dS in TMEM, dQ += dS K_j (a key tile with at most
+//                          64 valid slots over its first 64 keys only, as in the forward)
 //   bwd_kernel<kModeDKDV>  one key tile per CTA item, over its transposed list:
 //                          S^T = K Q_i^T, dP^T = V dO_i^T, P^T and dS^T in TMEM,
 //                          dV += P^T dO_i, dK += dS^T Q_i
@@ -63,6 +64,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColDP = 128, kColA0 = 256, kColA1 = 384;
 constexpr uint32_t kColS1 = 384;                // dQ mode: second S buffer (acc1 unused)
 constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);   // A, B K-major
+constexpr uint32_t kIdescSS64 = idesc_bf16_f32(128, 64, 0, 0);  // the first 64 keys (dQ mode)
 constexpr uint32_t kIdescTS = idesc_bf16_f32(128, 128, 0, 1);   // B MN-major
 constexpr int kRec = 8;
 constexpr int kItemRec = 4;                     // item records (dynamic work queue)
@@ -110,7 +112,9 @@ struct Bars {
   int32_t abort;
 };
 
-enum : uint32_t { kOpNewItem = 1u, kOpLastBlk = 2u, kOpFirstItem = 4u, kOpStop = 8u };
+// kOpHalf (dQ mode): the streamed key tile has at most 64 valid slots; S, dP and dQ's
+// accumulation run over its first 64 keys only (pad key slots get no gradient anyway).
+enum : uint32_t { kOpNewItem = 1u, kOpLastBlk = 2u, kOpFirstItem = 4u, kOpStop = 8u, kOpHalf = 16u };
 
 __device__ __forceinline__ int32_t list_len(const Args& a, int64_t u, int32_t& nf, bool& bad) {
   nf = a.full_cnt[u];
@@ -166,7 +170,17 @@ __device__ __forceinline__ void role_producer(const Args& a, Bars& bars, uint32_
         stop = true;
         break;
       }
-      bars.a_op[sa] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (fc == 0 ? kOpFirstItem : 0u);
+      // dQ mode: valid key slots of the streamed key tile (the softmax's record, the half flag)
+      int32_t nv = 128;
+      if (MODE == kModeDQ) {
+        nv = valid_h[idx];
+        if (nv < 0 || nv > 128) {
+          flag_status(ST_BAD_LIST);
+          nv = nv < 0 ? 0 : 128;
+        }
+      }
+      bars.a_op[sa] = (j == 0 ? kOpNewItem : 0u) | (j == n - 1 ? kOpLastBlk : 0u) | (fc == 0 ? kOpFirstItem : 0u) |
+                      (MODE == kModeDQ && nv <= 64 ? kOpHalf : 0u);
       {
         const uint32_t dst = sb + kOffA + sa * kTileB;
         const uint32_t bar = smem_u32(&bars.a_full[sa]);
@@ -206,11 +220,6 @@ __device__ __forceinline__ void role_producer(const Args& a, Bars& bars, uint32_
       if (MODE == kModeDQ) {
         // block record for the softmax: valid key slots of the streamed key tile (entry
         // sc % kRec was last read for block sc - kRec, long before ring-A slot sc - kStA came back)
-        int32_t nv = valid_h[idx];
-        if (nv < 0 || nv > 128) {
-          flag_status(ST_BAD_LIST);
-          nv = nv < 0 ? 0 : 128;
-        }
         bars.rec_nv[sc % kRec] = nv;
         mbar_arrive(smem_u32(&bars.rec_full[sc % kRec]));
       }
@@ -240,18 +249,27 @@ __device__ __forceinline__ void role_producer(const Args& a, Bars& bars, uint32_
 // ---------------------------------------------------------------- MMA issuer (one thread)
 // 128 x 128 x 128 products as 8 K16 MMAs: score-like F x S^T (both K-major in shared memory)
 // and accumulating A (bf16 in TMEM) x S (MN-major in shared memory).
-__device__ __forceinline__ void mma_score(uint32_t d, uint64_t a0, uint64_t b0) {
+// half: the streamed tile's first 64 rows only (N = 64 for the score-like product, K = 64
+// for the accumulating one).
+__device__ __forceinline__ void mma_score(uint32_t d, uint64_t a0, uint64_t b0, bool half = false) {
+  const uint32_t idesc = half ? kIdescSS64 : kIdescSS;
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
     const uint64_t koff = static_cast<uint64_t>((kk >> 2) * (kHalfB >> 4) + (kk & 3) * 2);
-    mma_ss(d, a0 + koff, b0 + koff, kIdescSS, kk > 0 ? 1u : 0u);
+    mma_ss(d, a0 + koff, b0 + koff, idesc, kk > 0 ? 1u : 0u);
   }
 }
-__device__ __forceinline__ void mma_accum(uint32_t d, uint32_t a_tmem, uint64_t b0, uint32_t acc_first) {
+__device__ __forceinline__ void mma_accum(uint32_t d, uint32_t a_tmem, uint64_t b0, uint32_t acc_first,
+                                          bool half = false) {
   mma_ts(d, a_tmem, b0, kIdescTS, acc_first);
 #pragma unroll
-  for (int kk = 1; kk < 8; ++kk)
+  for (int kk = 1; kk < 4; ++kk)
     mma_ts(d, a_tmem + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescTS, 1u);
+  if (!half) {
+#pragma unroll
+    for (int kk = 4; kk < 8; ++kk)
+      mma_ts(d, a_tmem + kk * 8, b0 + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescTS, 1u);
+  }
 }
 
 template <int MODE>
@@ -266,12 +284,14 @@ __device__ __forceinline__ void role_issuer(Bars& bars, uint32_t sb, uint32_t tm
   auto offB = [](uint32_t g) { return static_cast<uint64_t>((g % kStB) * (kTileB >> 4)); };
   auto s_col = [](uint32_t g) { return MODE == kModeDQ ? ((g & 1) ? kColS1 : kColS) : kColS; };
   // S-like = F0 x (ring-A tile)^T of block g into its S buffer; dP-like = F1 x (ring-B tile)^T
+  // half flag of block g (its ring-A slot's op word, read after that slot's phase was seen)
+  auto half_of = [&](uint32_t g) { return MODE == kModeDQ && (bars.a_op[g % kStA] & kOpHalf) != 0; };
   auto issue_s = [&](uint32_t g) {
-    mma_score(tmem + s_col(g), attn::opaque(dF), attn::opaque(dA + offA(g)));
+    mma_score(tmem + s_col(g), attn::opaque(dF), attn::opaque(dA + offA(g)), half_of(g));
     tc_commit(smem_u32(&bars.s_full[MODE == kModeDQ ? (g & 1) : 0]));
   };
   auto issue_dp = [&](uint32_t g) {
-    mma_score(tmem + kColDP, attn::opaque(dF + fix1), attn::opaque(dB + offB(g)));
+    mma_score(tmem + kColDP, attn::opaque(dF + fix1), attn::opaque(dB + offB(g)), half_of(g));
     tc_commit(smem_u32(&bars.dp_full));
     if (MODE == kModeDQ) tc_commit(smem_u32(&bars.b_empty[g % kStB]));   // V_g: last reader
   };
@@ -325,7 +345,7 @@ __device__ __forceinline__ void role_issuer(Bars& bars, uint32_t sb, uint32_t tm
       // the first accumulation of an item overwrites acc: the previous epilogue must be done
       if (need_o_free && !mbar_wait(smem_u32(&bars.o_free), (items - 1) & 1, abort, 48)) break;
       tc_fence_after();
-      mma_accum(tmem + kColA0, tmem + s_col(g), attn::opaque(dAm + offA(g)), acc_first);
+      mma_accum(tmem + kColA0, tmem + s_col(g), attn::opaque(dAm + offA(g)), acc_first, (op & kOpHalf) != 0);
       tc_commit(smem_u32(&bars.a_empty[g % kStA]));                    // K_g: last reader
     } else {
       // dV += P^T (written over S^T) x dO_g (ring B)
@@ -467,10 +487,14 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
         }
       }
       const uint32_t stat = sb + kOffStat + (g % kStStat) * kStatB;   // dK/dV: LSE, D
+      // dQ mode, key tile with at most 64 valid slots: S, dP and dQ's accumulation cover its
+      // first 64 keys only; column groups 8..15 are skipped by a warp-uniform branch
+      const bool hi = MODE != kModeDQ || nv > 64;
       uint32_t pk[32];
       // P (in place of s), and for dK/dV P^T packed over S
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
+        if (k == 8 && !hi) break;
         uint64_t na, nb;
         if (MODE == kModeDQ) {
           na = nl0;
@@ -512,6 +536,7 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
       // dS = P (dP - D), packed over S (dQ) or over dP (dK/dV)
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
+        if (k == 8 && !hi) break;
         float da0, da1, db0, db1;
         if (MODE == kModeDQ) {
           da0 = da1 = d0;
@@ -530,7 +555,12 @@ __device__ __forceinline__ void softmax_role(const Args& a, Bars& bars, uint32_t
         pk[2 * k] = pack_bf16x2(e0, e1);
         pk[2 * k + 1] = pack_bf16x2(f0, f1);
       }
-      tmem_st_16x128b_x16(tmem + lane_off + (MODE == kModeDQ ? colS : kColDP), pk);
+      if (MODE == kModeDQ) {
+        attn::tmem_st_p_half<0>(tmem + lane_off + colS, pk);
+        if (hi) attn::tmem_st_p_half<16>(tmem + lane_off + colS + 32, pk);
+      } else {
+        tmem_st_16x128b_x16(tmem + lane_off + kColDP, pk);
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();

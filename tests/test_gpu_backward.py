@@ -167,6 +167,16 @@ def test_backward_ragged_heads_batch_and_empty_rows():
     _run(w, [0, 1, 2])
 
 
+@pytest.mark.parametrize("r", [1, 63, 64, 65])
+def test_backward_partial_key_tiles_at_the_half_width_boundary(r):
+    """In the dQ pass, key tiles with at most 64 valid slots run S, dP and dQ's accumulation
+    over their first 64 keys: tiles of 128, r, 128, r valid slots, density 1, so every item
+    mixes both kinds (and the dK/dV pass sees partial query and key tiles of r rows)."""
+    w = synth.Workload(f"halfw{r}", 13, B=1, H=2, grid=(2, 1, 128 + r),
+                       head_shapes=((1, 1, 128), (1, 1, 128)), rho=((1, 1),), field=False)
+    _run(w, [0, 1])
+
+
 def test_backward_clip16x9_one_head():
     """The 16:9 clip at full size (40 heads launched, the benchmark's configuration), every
     transposed list checked, the gradients of head 0 against the oracle over all its rows."""
