@@ -614,7 +614,7 @@ def tile_plan(err: np.ndarray, max_shapes: int = 2) -> Tuple[List[int], np.ndarr
 # 10. FP8 (e4m3) variant of the attention step
 # ---------------------------------------------------------------------------------------
 # The pages ship their predictor in FP8 ([AGENTS] preamble and section 3) but give no FP8
-# attention; the variant here is this build's. Reading R23: Q, K and V tiles are quantised
+# attention; the variant here is defined by this module. Reading R23: Q, K and V tiles are quantised
 # to e4m3 (OCP FP8 E4M3 "fn": 1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no
 # infinities, codes 0x7F / 0xFF are NaN) with one scale per (batch, head) tensor:
 # scale = amax / 448 and code = e4m3(x * (448 / amax)), both in fp32, rounding to nearest
