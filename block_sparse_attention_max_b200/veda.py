@@ -121,9 +121,14 @@ def _stream(stream: Optional[torch.cuda.Stream]) -> int:
     return s.cuda_stream
 
 
-def _need(t: torch.Tensor, dtype: torch.dtype, name: str, cuda: bool = True) -> None:
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str, cuda: bool = True,
+          shape: Optional[Sequence[int]] = None) -> None:
+    """Type, shape, layout and device of a tensor handed to the library: a wrong shape would
+    send a kernel outside the buffer, so every one is checked before its pointer is passed."""
     if t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(int(x) for x in shape):
+        raise ValueError(f"{name}: expected shape {tuple(int(x) for x in shape)}, got {tuple(t.shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name}: must be contiguous")
     if cuda and not t.is_cuda:
@@ -131,6 +136,26 @@ def _need(t: torch.Tensor, dtype: torch.dtype, name: str, cuda: bool = True) -> 
     if cuda and t.device.index != torch.cuda.current_device():
         # the library launches on the calling thread's current device
         raise ValueError(f"{name}: on {t.device}, but the current device is cuda:{torch.cuda.current_device()}")
+
+
+def _need_maps(maps: "DeviceMaps", H: int, Npad: int, cuda: bool = True) -> None:
+    """The device tile map of H heads with Npad slots each (and its per-tile arrays)."""
+    if maps.Npad != Npad or maps.nT * 128 != Npad:
+        raise ValueError(f"tile map of {maps.Npad} slots per head, tensors have {Npad}")
+    _need(maps.tile_map, torch.int32, "tile_map", cuda, shape=(H, Npad))
+    for t, n in ((maps.tile_valid, "tile_valid"), (maps.tile_segment, "tile_segment")):
+        _need(t, torch.int32, n, cuda, shape=(H, Npad // 128))
+    _need(maps.nT_per_head, torch.int32, "nT_per_head", cuda, shape=(H,))
+
+
+def _need_lists(lists: "BlockLists", B: int, H: int, nT: int, name: str = "lists", cuda: bool = True) -> None:
+    """Block lists of a [B, H, nT] problem: counts [B, H, nT], indices [B, H, nT, stride]."""
+    if not 0 < lists.stride <= nT:
+        raise ValueError(f"{name}: stride {lists.stride} outside [1, {nT}]")
+    for t, n in ((lists.full_cnt, "full_cnt"), (lists.part_cnt, "part_cnt")):
+        _need(t, torch.int32, f"{name}.{n}", cuda, shape=(B, H, nT))
+    for t, n in ((lists.full_idx, "full_idx"), (lists.part_idx, "part_idx")):
+        _need(t, torch.int32, f"{name}.{n}", cuda, shape=(B, H, nT, lists.stride))
 
 
 # ---------------------------------------------------------------------------------------
@@ -207,9 +232,10 @@ def permute_tiles(x: torch.Tensor, maps: DeviceMaps, out: Optional[torch.Tensor]
                   stream=None) -> torch.Tensor:
     _need(x, torch.bfloat16, "x")
     B, N, H, D = x.shape
+    _need_maps(maps, H, maps.Npad)
     if out is None:
         out = torch.empty((B, H, maps.Npad, D), dtype=torch.bfloat16, device=x.device)
-    _need(out, torch.bfloat16, "out")
+    _need(out, torch.bfloat16, "out", shape=(B, H, maps.Npad, D))
     _check("veda_permute_tiles", lib().veda_permute_tiles(
         _ptr(x), _ptr(out), _ptr(maps.tile_map), B, N, H, D, maps.Npad, _stream(stream)))
     return out
@@ -220,12 +246,13 @@ def permute_pool(x: torch.Tensor, maps: DeviceMaps, out: Optional[torch.Tensor] 
     """veda_permute_pool: the tile gather and the tile pooling in one pass."""
     _need(x, torch.bfloat16, "x")
     B, N, H, D = x.shape
+    _need_maps(maps, H, maps.Npad)
     if out is None:
         out = torch.empty((B, H, maps.Npad, D), dtype=torch.bfloat16, device=x.device)
     if pooled is None:
         pooled = torch.empty((B, H, maps.Npad // 128, 3, D), dtype=torch.float32, device=x.device)
-    _need(out, torch.bfloat16, "out")
-    _need(pooled, torch.float32, "pooled")
+    _need(out, torch.bfloat16, "out", shape=(B, H, maps.Npad, D))
+    _need(pooled, torch.float32, "pooled", shape=(B, H, maps.Npad // 128, 3, D))
     _check("veda_permute_pool", lib().veda_permute_pool(
         _ptr(x), _ptr(out), _ptr(maps.tile_map), _ptr(maps.tile_valid), _ptr(pooled), B, N, H, D,
         maps.Npad, _stream(stream)))
@@ -237,9 +264,10 @@ def tile_pool(x_tiled: torch.Tensor, maps: DeviceMaps, out: Optional[torch.Tenso
     _need(x_tiled, torch.bfloat16, "x_tiled")
     B, H, Npad, D = x_tiled.shape
     nT = Npad // 128
+    _need_maps(maps, H, Npad)
     if out is None:
         out = torch.empty((B, H, nT, 3, D), dtype=torch.float32, device=x_tiled.device)
-    _need(out, torch.float32, "out")
+    _need(out, torch.float32, "out", shape=(B, H, nT, 3, D))
     _check("veda_tile_pool", lib().veda_tile_pool(
         _ptr(x_tiled), _ptr(maps.tile_valid), _ptr(out), B, H, nT, D, _stream(stream)))
     return out
@@ -252,14 +280,20 @@ def block_scores_workspace_bytes(B: int, H: int, nT: int, D: int = 128) -> int:
 def block_scores(pooled_q: torch.Tensor, pooled_k: torch.Tensor, wq: torch.Tensor,
                  wk: torch.Tensor, out: Optional[torch.Tensor] = None,
                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    for t, n in ((pooled_q, "pooled_q"), (pooled_k, "pooled_k"), (wq, "wq"), (wk, "wk")):
-        _need(t, torch.float32, n)
-    B, H, nT, _, D = pooled_q.shape
+    _need(pooled_q, torch.float32, "pooled_q")
+    B, H, nT, three, D = pooled_q.shape
+    if three != 3:
+        raise ValueError("pooled_q: expected shape [B, H, nT, 3, D]")
+    _need(pooled_k, torch.float32, "pooled_k", shape=pooled_q.shape)
+    for t, n in ((wq, "wq"), (wk, "wk")):
+        _need(t, torch.float32, n, shape=(H, D, 3 * D))
     if out is None:
         out = torch.empty((B, H, nT, nT), dtype=torch.float32, device=pooled_q.device)
+    _need(out, torch.float32, "out", shape=(B, H, nT, nT))
     nbytes = block_scores_workspace_bytes(B, H, nT, D)
     if workspace is None:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=pooled_q.device)
+    _need(workspace, workspace.dtype, "workspace")
     _check("veda_block_scores", lib().veda_block_scores(
         _ptr(pooled_q), _ptr(pooled_k), _ptr(wq), _ptr(wk), _ptr(out), _ptr(workspace),
         workspace.numel() * workspace.element_size(), B, H, nT, D, _stream(stream)))
@@ -312,7 +346,10 @@ def select_blocks(scores: torch.Tensor, maps: DeviceMaps, rho: Sequence[Tuple[in
                   list_stride: Optional[int] = None, out: Optional[BlockLists] = None,
                   stream=None) -> BlockLists:
     _need(scores, torch.float32, "scores")
-    B, H, nT, _ = scores.shape
+    B, H, nT, nT2 = scores.shape
+    if nT2 != nT:
+        raise ValueError("scores: expected shape [B, H, nT, nT]")
+    _need_maps(maps, H, nT * 128)
     stride = list_stride or list_stride_for(nT, rho)
     if out is None:
         dev = scores.device
@@ -320,6 +357,7 @@ def select_blocks(scores: torch.Tensor, maps: DeviceMaps, rho: Sequence[Tuple[in
                          torch.zeros((B, H, nT, stride), dtype=torch.int32, device=dev),
                          torch.empty((B, H, nT), dtype=torch.int32, device=dev),
                          torch.zeros((B, H, nT, stride), dtype=torch.int32, device=dev), stride)
+    _need_lists(out, B, H, nT, "out")
     num = (ctypes.c_int32 * len(rho))(*[int(p) for p, _ in rho])
     den = (ctypes.c_int32 * len(rho))(*[int(q) for _, q in rho])
     _check("veda_select_blocks", lib().veda_select_blocks(
@@ -334,14 +372,20 @@ def block_sparse_attn_fwd(q_t: torch.Tensor, k_t: torch.Tensor, v_t: torch.Tenso
                           maps: DeviceMaps, lists: BlockLists, scale: float,
                           out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                           want_lse: bool = True, stream=None):
-    for t, n in ((q_t, "q"), (k_t, "k"), (v_t, "v")):
-        _need(t, torch.bfloat16, n)
+    _need(q_t, torch.bfloat16, "q")
     B, H, Npad, D = q_t.shape
     nT = Npad // 128
+    for t, n in ((k_t, "k"), (v_t, "v")):
+        _need(t, torch.bfloat16, n, shape=q_t.shape)
+    _need_maps(maps, H, Npad)
+    _need_lists(lists, B, H, nT)
     if out is None:
         out = torch.empty_like(q_t)
     if lse is None and want_lse:
         lse = torch.empty((B, H, Npad), dtype=torch.float32, device=q_t.device)
+    _need(out, torch.bfloat16, "out", shape=q_t.shape)
+    if lse is not None:
+        _need(lse, torch.float32, "lse", shape=(B, H, Npad))
     _check("veda_block_sparse_attn_fwd", lib().veda_block_sparse_attn_fwd(
         _ptr(q_t), _ptr(k_t), _ptr(v_t), _ptr(maps.tile_valid), _ptr(lists.full_cnt),
         _ptr(lists.full_idx), _ptr(lists.part_cnt), _ptr(lists.part_idx), lists.stride,
@@ -360,8 +404,8 @@ def quantize_fp8(x_t: torch.Tensor, transpose_tiles: bool = False, codes: Option
         codes = torch.empty((B, H, Npad, D), dtype=torch.uint8, device=x_t.device)
     if scale is None:
         scale = torch.empty((B, H), dtype=torch.float32, device=x_t.device)
-    _need(codes, torch.uint8, "codes")
-    _need(scale, torch.float32, "scale")
+    _need(codes, torch.uint8, "codes", shape=(B, H, Npad, D))
+    _need(scale, torch.float32, "scale", shape=(B, H))
     _check("veda_quantize_fp8", lib().veda_quantize_fp8(
         _ptr(x_t), _ptr(codes), _ptr(scale), B, H, Npad // 128, D, 1 if transpose_tiles else 0, _stream(stream)))
     return codes, scale
@@ -373,16 +417,22 @@ def block_sparse_attn_fwd_fp8(q8: torch.Tensor, k8: torch.Tensor, vt8: torch.Ten
                               want_lse: bool = True, stream=None):
     """FP8 variant of the attention step: e4m3 codes of Q, K and (transposed tiles) V with
     their per-(batch, head) scales -> bf16 O [B, H, Npad, 128] and fp32 LSE."""
-    for t, n in ((q8, "q8"), (k8, "k8"), (vt8, "vt8")):
-        _need(t, torch.uint8, n)
-    for t, n in ((q_scale, "q_scale"), (k_scale, "k_scale"), (v_scale, "v_scale")):
-        _need(t, torch.float32, n)
+    _need(q8, torch.uint8, "q8")
     B, H, Npad, D = q8.shape
     nT = Npad // 128
+    for t, n in ((k8, "k8"), (vt8, "vt8")):
+        _need(t, torch.uint8, n, shape=q8.shape)
+    for t, n in ((q_scale, "q_scale"), (k_scale, "k_scale"), (v_scale, "v_scale")):
+        _need(t, torch.float32, n, shape=(B, H))
+    _need_maps(maps, H, Npad)
+    _need_lists(lists, B, H, nT)
     if out is None:
         out = torch.empty((B, H, Npad, D), dtype=torch.bfloat16, device=q8.device)
     if lse is None and want_lse:
         lse = torch.empty((B, H, Npad), dtype=torch.float32, device=q8.device)
+    _need(out, torch.bfloat16, "out", shape=(B, H, Npad, D))
+    if lse is not None:
+        _need(lse, torch.float32, "lse", shape=(B, H, Npad))
     _check("veda_block_sparse_attn_fwd_fp8", lib().veda_block_sparse_attn_fwd_fp8(
         _ptr(q8), _ptr(k8), _ptr(vt8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale), _ptr(maps.tile_valid),
         _ptr(lists.full_cnt), _ptr(lists.full_idx), _ptr(lists.part_cnt), _ptr(lists.part_idx), lists.stride,
@@ -400,6 +450,8 @@ class TransposedLists:
 def transpose_lists(lists: BlockLists, maps: DeviceMaps, stream=None) -> TransposedLists:
     """veda_transpose_lists: the query tiles of every key tile (the backward's lists)."""
     B, H, nT = lists.full_cnt.shape
+    _need_lists(lists, B, H, nT)
+    _need_maps(maps, H, nT * 128)
     dev = lists.full_cnt.device
     t = TransposedLists(torch.empty((B, H, nT), dtype=torch.int32, device=dev),
                         torch.zeros((B, H, nT, nT), dtype=torch.int32, device=dev), nT)
@@ -414,11 +466,18 @@ def block_sparse_attn_bwd(q_t: torch.Tensor, k_t: torch.Tensor, v_t: torch.Tenso
                           do_t: torch.Tensor, lse: torch.Tensor, maps: DeviceMaps, lists: BlockLists,
                           tlists: TransposedLists, scale: float, stream=None):
     """veda_block_sparse_attn_bwd: dQ, dK, dV (tile order, bf16) over the forward's lists."""
-    for t, n in ((q_t, "q"), (k_t, "k"), (v_t, "v"), (o_t, "o"), (do_t, "dout")):
-        _need(t, torch.bfloat16, n)
-    _need(lse, torch.float32, "lse")
+    _need(q_t, torch.bfloat16, "q")
     B, H, Npad, D = q_t.shape
     nT = Npad // 128
+    for t, n in ((k_t, "k"), (v_t, "v"), (o_t, "o"), (do_t, "dout")):
+        _need(t, torch.bfloat16, n, shape=q_t.shape)
+    _need(lse, torch.float32, "lse", shape=(B, H, Npad))
+    _need_maps(maps, H, Npad)
+    _need_lists(lists, B, H, nT)
+    if tlists.stride != nT:
+        raise ValueError(f"tlists: stride {tlists.stride}, expected {nT}")
+    _need(tlists.cnt, torch.int32, "tlists.cnt", shape=(B, H, nT))
+    _need(tlists.idx, torch.int32, "tlists.idx", shape=(B, H, nT, nT))
     dq, dk, dv = torch.empty_like(q_t), torch.empty_like(k_t), torch.empty_like(v_t)
     delta = torch.empty(B * H * Npad + 4, dtype=torch.float32, device=q_t.device)   # D + work counters
     _check("veda_block_sparse_attn_bwd", lib().veda_block_sparse_attn_bwd(
@@ -433,13 +492,16 @@ def block_heat(q_t: torch.Tensor, k_t: torch.Tensor, maps: DeviceMaps, lists: Bl
                lse: torch.Tensor, scale: float, out: Optional[torch.Tensor] = None,
                stream=None) -> torch.Tensor:
     """veda_block_heat: per-block attention mass against the given (dense) LSE."""
-    for t, n in ((q_t, "q"), (k_t, "k")):
-        _need(t, torch.bfloat16, n)
-    _need(lse, torch.float32, "lse")
+    _need(q_t, torch.bfloat16, "q")
     B, H, Npad, D = q_t.shape
     nT = Npad // 128
+    _need(k_t, torch.bfloat16, "k", shape=q_t.shape)
+    _need(lse, torch.float32, "lse", shape=(B, H, Npad))
+    _need_maps(maps, H, Npad)
+    _need_lists(lists, B, H, nT)
     if out is None:
         out = torch.empty((B, H, nT, nT), dtype=torch.float32, device=q_t.device)
+    _need(out, torch.float32, "out", shape=(B, H, nT, nT))
     _check("veda_block_heat", lib().veda_block_heat(
         _ptr(q_t), _ptr(k_t), _ptr(maps.tile_valid), _ptr(lists.full_cnt), _ptr(lists.full_idx),
         _ptr(lists.part_cnt), _ptr(lists.part_idx), lists.stride, _ptr(lse), float(scale),
@@ -470,7 +532,12 @@ def mask_quality(heat: torch.Tensor, maps: DeviceMaps, pred: BlockLists, oracle:
                  stream=None) -> MaskQuality:
     """veda_mask_quality: kept attention mass of `pred` and its recall against `oracle`."""
     _need(heat, torch.float32, "heat")
-    B, H, nT, _ = heat.shape
+    B, H, nT, nT2 = heat.shape
+    if nT2 != nT:
+        raise ValueError("heat: expected shape [B, H, nT, nT]")
+    _need_maps(maps, H, nT * 128)
+    _need_lists(pred, B, H, nT, "pred")
+    _need_lists(oracle, B, H, nT, "oracle")
     dev = heat.device
     q = MaskQuality(torch.empty((B, H, nT), dtype=torch.float32, device=dev),
                     torch.empty((B, H, nT), dtype=torch.float32, device=dev),
@@ -487,7 +554,7 @@ def mask_quality(heat: torch.Tensor, maps: DeviceMaps, pred: BlockLists, oracle:
 def rel_error(o: torch.Tensor, o_ref: torch.Tensor, stream=None) -> torch.Tensor:
     """veda_rel_error: [H, 2] sums of |o - o_ref|^2 and |o_ref|^2 per head (raster bf16)."""
     _need(o, torch.bfloat16, "o")
-    _need(o_ref, torch.bfloat16, "o_ref")
+    _need(o_ref, torch.bfloat16, "o_ref", shape=o.shape)
     B, N, H, D = o.shape
     sums = torch.empty((H, 2), dtype=torch.float32, device=o.device)
     _check("veda_rel_error", lib().veda_rel_error(_ptr(o), _ptr(o_ref), _ptr(sums), B, N, H, D,
@@ -514,8 +581,10 @@ def unpermute(o_t: torch.Tensor, maps: DeviceMaps, N: int, out: Optional[torch.T
               stream=None) -> torch.Tensor:
     _need(o_t, torch.bfloat16, "o_tiled")
     B, H, Npad, D = o_t.shape
+    _need_maps(maps, H, Npad)
     if out is None:
         out = torch.empty((B, N, H, D), dtype=torch.bfloat16, device=o_t.device)
+    _need(out, torch.bfloat16, "out", shape=(B, N, H, D))
     _check("veda_unpermute", lib().veda_unpermute(
         _ptr(o_t), _ptr(out), _ptr(maps.tile_map), B, N, H, D, Npad, _stream(stream)))
     return out

@@ -155,3 +155,30 @@ def test_tile_plan_vote_rejects_nan_and_bad_sizes(L):
         veda.tile_plan_vote(np.array([[0.1, np.nan]]))
     with pytest.raises(veda.VedaError):
         veda.tile_plan_vote(np.zeros((2, 3)), max_shapes=0)
+
+
+def test_binding_checks_shapes_before_passing_pointers():
+    """A buffer of the wrong shape would send a kernel outside it: the binding compares every
+    tensor's shape with the call's sizes (and the tile map's and the lists') before the call."""
+    maps = veda.build_tile_map((2, 8, 16), [(1, 8, 16), (1, 8, 16)], 0).to("cpu")   # H = 2, nT = 2
+    veda._need_maps(maps, 2, 256, cuda=False)
+    with pytest.raises(ValueError, match="slots per head"):
+        veda._need_maps(maps, 2, 384, cuda=False)
+    with pytest.raises(ValueError, match="expected shape"):
+        veda._need_maps(maps, 3, 256, cuda=False)                  # three heads, map of two
+    z = lambda *s: torch.zeros(s, dtype=torch.int32)
+    lists = veda.BlockLists(z(1, 2, 2), z(1, 2, 2, 2), z(1, 2, 2), z(1, 2, 2, 2), 2)
+    veda._need_lists(lists, 1, 2, 2, cuda=False)
+    with pytest.raises(ValueError, match="stride"):
+        veda._need_lists(veda.BlockLists(z(1, 2, 2), z(1, 2, 2, 3), z(1, 2, 2), z(1, 2, 2, 3), 3), 1, 2, 2,
+                         cuda=False)
+    with pytest.raises(ValueError, match="expected shape"):
+        veda._need_lists(lists, 2, 2, 2, cuda=False)                # batch 2, lists of batch 1
+    with pytest.raises(ValueError, match="expected shape"):
+        veda._need_lists(veda.BlockLists(z(1, 2, 2), z(1, 2, 2, 1), z(1, 2, 2), z(1, 2, 2, 2), 2), 1, 2, 2,
+                         cuda=False)                                 # full_idx narrower than the stride
+    with pytest.raises(TypeError):
+        veda._need(torch.zeros(4, dtype=torch.float16), torch.bfloat16, "x", cuda=False)
+    with pytest.raises(ValueError, match="expected shape"):
+        veda._need(torch.zeros(4, 3, dtype=torch.bfloat16), torch.bfloat16, "x", cuda=False, shape=(4, 4))
+    veda._need(torch.zeros(4, 4, dtype=torch.bfloat16), torch.bfloat16, "x", cuda=False, shape=(4, 4))
